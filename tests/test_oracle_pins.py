@@ -1,0 +1,420 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each test checks the oracle against a library routine on a special case that reduces
+to it (torch's scaled_dot_product_attention in float64), a closed form, an invariant
+of the method, or a hand-derived fixture under tests/golden/. The mutation tests at
+the end plant plausible mistakes in the oracle and check that a pin catches them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.spark_oracle as orc
+from block_sparse_video_mean_b200.inputs import make_qkv, random_orthogonal
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def sdpa64(q, k, v, scale):
+    """Dense softmax attention of every row, by torch's library routine in float64."""
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(a))[None, None] for a in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=scale)
+    return o[0, 0].numpy()
+
+
+def lse64(q, k, scale):
+    return torch.logsumexp(torch.from_numpy(q @ k.T * scale), dim=1).numpy()
+
+
+def head(nv, ns, d, seed=0, amp=0.5):
+    Q, K, V = make_qkv(1, 1, nv, ns, d, seed=seed, amp=amp)
+    return tuple(orc.to_f64(t[0, 0]) for t in (Q, K, V))
+
+
+# ----------------------------------------------------------------- attention core
+
+@pytest.mark.parametrize("nv,ns,d", [(256, 16, 64), (320, 0, 32), (256 + 37, 5, 64), (30, 8, 16)])
+def test_full_density_no_compression_is_dense_attention(nv, ns, d):
+    """Keep ratio 1.0 with the compressed branch off is dense softmax attention for every
+    row (video, ragged tail and sink rows)."""
+    q, k, v = head(nv, ns, d, seed=3)
+    scale = 1 / math.sqrt(d)
+    O, L, _ = orc.forward_head(q, k, v, ns, "topk", 1.0, compressed=False)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, scale), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(L, lse64(q, k, scale), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mode,param", [("topk", 0.25), ("topk", 0.1), ("tau", 0.5)])
+def test_constant_key_blocks_make_compression_exact(mode, param):
+    """When every key of a video block is the same vector, the pooled entry with the
+    log-mass bias carries exactly the block's attention mass and value, so the split
+    forward equals dense attention at any density."""
+    nv, ns, d = 512, 24, 64
+    q, k, v = head(nv, ns, d, seed=5)
+    kb = k[:nv].reshape(-1, 64, d)
+    kb[:] = kb[:, :1, :]
+    k[:nv] = kb.reshape(nv, d)
+    O, L, info = orc.forward_head(q, k, v, ns, mode, param, compressed=True)
+    scale = 1 / math.sqrt(d)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, scale), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(L, lse64(q, k, scale), atol=1e-10, rtol=0)
+    pooled = info["pooled"]
+    np.testing.assert_allclose(pooled.beta, math.log(64), atol=1e-12)
+    np.testing.assert_allclose(pooled.vtil, v[:nv].reshape(-1, 64, d).mean(1), atol=1e-12)
+
+
+def test_anchor_query_rows_are_exact():
+    """A query equal to the anchor sees, through each compressed entry, exactly the mass
+    and the mass-weighted value of the block it stands for; its output is the dense one
+    at any density. The other rows must differ (the branch is an approximation)."""
+    rng = np.random.default_rng(7)
+    nv, ns, d = 640, 16, 32
+    a = rng.standard_normal(d)
+    delta = rng.standard_normal((nv // 2, d)) * 1.3
+    delta[::9] = 0.0                                   # some rows are exactly the anchor
+    q = np.concatenate([a + delta, a - delta])         # mean of the video rows is a
+    q = q[rng.permutation(nv)]
+    q = np.concatenate([q, rng.standard_normal((ns, d))])
+    k = rng.standard_normal((nv + ns, d)) + 0.4 * np.repeat(rng.standard_normal((nv // 64 + 1, d)), 64, 0)[: nv + ns]
+    v = rng.standard_normal((nv + ns, d))
+    O, L, info = orc.forward_head(q, k, v, ns, "topk", 0.2, compressed=True)
+    np.testing.assert_allclose(info["pooled"].anchor, a, atol=1e-13)
+    scale = 1 / math.sqrt(d)
+    ref = sdpa64(q, k, v, scale)
+    lref = lse64(q, k, scale)
+    rows = np.nonzero(np.all(np.abs(q[:nv] - a) < 1e-15, axis=1))[0]
+    assert rows.size >= 8
+    np.testing.assert_allclose(O[rows], ref[rows], atol=1e-11, rtol=0)
+    np.testing.assert_allclose(L[rows], lref[rows], atol=1e-11, rtol=0)
+    others = np.setdiff1d(np.arange(nv), rows)
+    assert np.abs(O[others] - ref[others]).max() > 1e-3
+
+
+def test_log_mass_identity_at_the_anchor():
+    """exp(a . kbar_b * scale + beta_b) is the block's total anchor mass sum_j exp(s_j)."""
+    q, k, v = head(1024, 32, 64, seed=11)
+    scale = 0.125
+    P = orc.pool_head(q, k, v, 32, scale)
+    kb = k[:1024].reshape(16, 64, 64)
+    mass = np.exp((kb @ q[:1024].mean(0)) * scale).sum(axis=1)
+    np.testing.assert_allclose(np.exp(P.kbar @ P.anchor * scale + P.beta), mass, rtol=1e-13)
+    # the bias is the Jensen gap plus log(64): never below log(64)
+    assert np.all(P.beta >= math.log(64) - 1e-12)
+
+
+def test_pooled_means_and_anchor():
+    rng = np.random.default_rng(1)
+    nb, d = 6, 16
+    rows = rng.standard_normal((nb, d))
+    q = np.repeat(rows, 64, axis=0)                    # every block holds one repeated query
+    k = np.repeat(rows[::-1], 64, axis=0)
+    P = orc.pool_head(q, k, q, 0)
+    np.testing.assert_allclose(P.qbar, rows, atol=1e-14)
+    np.testing.assert_allclose(P.kbar, rows[::-1], atol=1e-14)
+    np.testing.assert_allclose(P.anchor, rows.mean(0), atol=1e-14)
+
+
+@pytest.mark.parametrize("compressed", [True, False])
+@pytest.mark.parametrize("pool_mode", ["reweight", "mean"])
+def test_constant_values_give_constant_output(compressed, pool_mode):
+    """Softmax weights sum to one over both branches, so V = c everywhere gives O = c."""
+    q, k, v = head(384, 20, 32, seed=2)
+    c = np.linspace(-1, 2, 32)
+    v[:] = c
+    O, _, _ = orc.forward_head(q, k, v, 20, "topk", 0.3, compressed=compressed, pool_mode=pool_mode)
+    np.testing.assert_allclose(O, np.broadcast_to(c, O.shape), atol=1e-12)
+
+
+def test_mean_pool_branch_closed_form():
+    """Plain mean pooling: vtil = block mean of v, beta = log 64; with constant key
+    blocks it is exact as well (Jensen's gap vanishes)."""
+    q, k, v = head(256, 8, 32, seed=4)
+    P = orc.pool_head(q, k, v, 8, mode="mean")
+    np.testing.assert_allclose(P.vtil, v[:256].reshape(4, 64, 32).mean(1), atol=1e-14)
+    np.testing.assert_allclose(P.beta, math.log(64), atol=0)
+
+
+def test_empty_row_outputs_zero():
+    """tau so high that nothing is kept, no sinks, no compressed branch: O = 0, LSE = -inf."""
+    q, k, v = head(256, 0, 32, seed=6)
+    O, L, info = orc.forward_head(q, k, v, 0, "tau", 50.0, compressed=False)
+    assert all(len(s) == 0 for s in info["sel"])
+    assert np.all(O == 0) and np.all(np.isneginf(L))
+
+
+# ----------------------------------------------------------------- selection
+
+def _golden_rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def test_topk_hand_derived_fixture():
+    for ln in _golden_rows("topk_tiny.txt"):
+        k, s, e = (p.strip() for p in ln.split("|"))
+        got = orc.select_topk_row(np.array([float(x) for x in s.split(",")]), int(k))
+        assert got.tolist() == [int(x) for x in e.split(",")], ln
+
+
+def test_topk_count_fixture():
+    for ln in _golden_rows("topk_count.txt"):
+        r, nb, k = ln.split()
+        assert orc.topk_count(float(r), int(nb)) == int(k), ln
+
+
+def test_topk_selection_invariants():
+    """Every kept score is >= every dropped one; equal scores are kept lowest index first."""
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        nb = int(rng.integers(1, 90))
+        s = np.round(rng.standard_normal(nb), 1)      # coarse rounding forces ties
+        k = int(rng.integers(1, nb + 1))
+        sel = orc.select_topk_row(s, k)
+        assert len(sel) == k and np.all(np.diff(sel) > 0)
+        drop = np.setdiff1d(np.arange(nb), sel)
+        if drop.size:
+            assert s[sel].min() >= s[drop].max()
+            t = s[sel].min()
+            if np.any(s[drop] == t):                   # a tie at the boundary
+                assert np.nonzero(s == t)[0][: (s[sel] == t).sum()].tolist() == sel[s[sel] == t].tolist()
+
+
+def test_tau_moments_closed_form():
+    """mu = scale * (sum qbar) . (sum kbar) / nb^2 and E[S^2] = scale^2 tr(Mq Mk) / nb^2."""
+    q, k, v = head(64 * 40, 0, 32, seed=9)
+    scale = 1 / math.sqrt(32)
+    P = orc.pool_head(q, k, v, 0, scale)
+    S = orc.block_scores(P.qbar, P.kbar, scale)
+    mu, sigma = orc.tau_stats(S)
+    nb = P.qbar.shape[0]
+    mu_cf = scale * P.qbar.sum(0) @ P.kbar.sum(0) / nb ** 2
+    es2 = scale ** 2 * np.trace((P.qbar.T @ P.qbar) @ (P.kbar.T @ P.kbar)) / nb ** 2
+    assert abs(mu - mu_cf) < 1e-13
+    assert abs(sigma - math.sqrt(es2 - mu_cf ** 2)) < 1e-12
+
+
+def test_tau_kept_fraction_matches_pages_and_gaussian_tail():
+    """On block-correlated synthetic data the block scores are close to Gaussian, so
+    tau = 1.0 / 1.5 / 2.0 keeps about the upper-tail mass; the pages quote ~16/7/2.7%."""
+    Q, K, V = make_qkv(1, 2, 64 * 300, 0, 128, seed=0)
+    fr = {}
+    for h in range(2):
+        q, k, v = (orc.to_f64(t[0, h]) for t in (Q, K, V))
+        P = orc.pool_head(q, k, v, 0)
+        S = orc.block_scores(P.qbar, P.kbar, 1 / math.sqrt(128))
+        for ln in _golden_rows("tau_kept_fraction.txt"):
+            tau, pages, tail = (float(x) for x in ln.split())
+            kept = 100.0 * (S > orc.tau_threshold(S, tau)).mean()
+            fr.setdefault(tau, []).append(kept)
+            assert abs(kept - tail) < 1.0, (tau, kept, tail)
+            assert abs(kept - pages) < 1.5, (tau, kept, pages)
+    assert fr[1.0][0] > fr[1.5][0] > fr[2.0][0]
+
+
+def test_topk_tau_scale_invariance():
+    """Selections do not depend on the softmax scale (top-k) and on a common scaling of
+    K (tau works in sigma units)."""
+    q, k, v = head(64 * 30, 0, 32, seed=12)
+    a = orc.forward_head(q, k, v, 0, "topk", 0.2, scale=0.1)[2]["sel"]
+    b = orc.forward_head(q, k, v, 0, "topk", 0.2, scale=0.7)[2]["sel"]
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    c = orc.forward_head(q, k, v, 0, "tau", 1.2)[2]["sel"]
+    d = orc.forward_head(q, 3.0 * k, v, 0, "tau", 1.2)[2]["sel"]
+    assert all(np.array_equal(x, y) for x, y in zip(c, d))
+
+
+# ----------------------------------------------------------------- Spark-Reblock
+
+def _check_partition(perm, nv):
+    assert sorted(perm.tolist()) == list(range(nv))
+    leaves = perm.reshape(-1, 64)
+    assert np.all(np.diff(leaves, axis=1) > 0)            # ascending inside a leaf
+    assert np.all(np.diff(leaves[:, 0]) > 0)              # leaves by smallest index
+
+
+@pytest.mark.parametrize("nb", [1, 2, 3, 5, 8, 13])
+def test_reblock_leaves_are_exact_blocks(nb):
+    q, k, v = head(64 * nb, 10, 32, seed=nb)
+    rb = orc.reblock_head(q, k, 10)
+    _check_partition(rb.perm, 64 * nb)
+    assert rb.labels.shape[0] == orc.n_levels(nb) + 1
+    _, counts = np.unique(rb.labels[-1], return_counts=True)
+    assert np.all(counts == 64)
+
+
+def _partition_sets(perm):
+    return sorted(tuple(x) for x in perm.reshape(-1, 64).tolist())
+
+
+def test_reblock_invariances():
+    """The partition depends only on the Mahalanobis cosines q_i^T M q_j: unchanged when K
+    is scaled, and when Q and K are rotated together by an orthogonal matrix."""
+    q, k, v = head(64 * 12, 0, 32, seed=21)
+    base = _partition_sets(orc.reblock_head(q, k, 0).perm)
+    assert _partition_sets(orc.reblock_head(q, 3.7 * k, 0).perm) == base
+    assert _partition_sets(orc.reblock_head(2.5 * q, k, 0).perm) == base
+    R = random_orthogonal(32, 5).numpy()
+    assert _partition_sets(orc.reblock_head(q @ R, k @ R, 0).perm) == base
+
+
+def test_whitening_is_mahalanobis_cosine():
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((50, 8))
+    k = rng.standard_normal((400, 8)) @ rng.standard_normal((8, 8))
+    M = orc.key_second_moment(k)
+    x = orc.whiten(q, M)
+    qMq = q @ M @ q.T
+    nrm = np.sqrt(np.diag(qMq))
+    np.testing.assert_allclose(x @ x.T, qMq / np.outer(nrm, nrm), atol=1e-12)
+
+
+def test_reblock_two_clusters_split_first():
+    """Two well separated groups of query directions go to different children at level 0."""
+    rng = np.random.default_rng(8)
+    d = 16
+    e = np.eye(d)
+    q = np.concatenate([e[0] + 0.05 * rng.standard_normal((192, d)),
+                        e[1] + 0.05 * rng.standard_normal((192, d))])
+    idx = rng.permutation(384)
+    q = q[idx]
+    k = rng.standard_normal((384, d))
+    rb = orc.reblock_head(q, k, 0)
+    groupA = set(np.nonzero(idx < 192)[0].tolist())
+    left = set(np.nonzero(rb.labels[1] == 0)[0].tolist())
+    assert left == groupA or left == set(range(384)) - groupA
+
+
+def test_reblock_arc_hand_derived():
+    """Queries on a short arc of a circle with an isotropic key second moment: the
+    principal direction runs along the arc, so the leaves are the consecutive runs of
+    64 angles, whatever the token order (hand-derived; no eigen solver involved)."""
+    rng = np.random.default_rng(4)
+    n, d = 512, 8
+    theta = np.sort(rng.uniform(0.0, 0.6, n))
+    q = np.zeros((n, d))
+    q[:, 0], q[:, 1] = np.cos(theta), np.sin(theta)
+    shuffle = rng.permutation(n)
+    q = q[shuffle]
+    Qo, _ = np.linalg.qr(rng.standard_normal((n, d)))
+    k = Qo * math.sqrt(n)                                   # k^T k / n = I exactly
+    rb = orc.reblock_head(q, k, 0)
+    rank = np.argsort(np.argsort(theta[shuffle]))           # position of each token on the arc
+    expect = sorted(tuple(sorted(np.nonzero(rank // 64 == g)[0].tolist())) for g in range(8))
+    assert _partition_sets(rb.perm) == expect
+
+
+def test_reblock_odd_node_sign_convention():
+    """m = 3: the left child takes the 64 lowest projections, with the eigenvector
+    signed so that the projections have a non-negative third central moment."""
+    rng = np.random.default_rng(5)
+    n, d = 192, 4
+    t = np.concatenate([rng.uniform(-1, 0.3, 150), rng.uniform(2.0, 6.0, 42)])  # long + tail
+    q = np.zeros((n, d))
+    q[:, 0] = 1.0
+    q[:, 1] = 0.05 * t
+    q[:, 2:] = 1e-4 * rng.standard_normal((n, 2))
+    k = np.eye(d)[np.arange(n) % d] * 2.0
+    rb = orc.reblock_head(q, k, 0)
+    sp = rb.splits[(0, 0)]
+    assert sp.skew >= 0
+    assert set(sp.left.tolist()) == set(np.argsort(t)[:64].tolist())
+
+
+def test_reblock_m2_split_matches_svd():
+    """For a two-block node the split is the median of the projection on the top right
+    singular vector of the centred whitened data (numpy SVD, another routine than eigh)."""
+    q, k, v = head(128, 0, 16, seed=30)
+    rb = orc.reblock_head(q, k, 0)
+    x = orc.whiten(q, orc.key_second_moment(k))
+    _, _, Vt = np.linalg.svd(x - x.mean(0))
+    p = x @ Vt[0]
+    low = set(np.argsort(p)[:64].tolist())
+    left = set(rb.splits[(0, 0)].left.tolist())
+    assert left == low or left == set(range(128)) - low
+
+
+def test_reblock_forward_outputs_in_original_order():
+    """With reblocking at full density and no compression the forward is still dense
+    attention, row for row in the original order."""
+    q, k, v = head(64 * 6, 12, 32, seed=13)
+    O, L, info = orc.forward_head(q, k, v, 12, "topk", 1.0, compressed=False, reblock=True)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, 1 / math.sqrt(32)), atol=1e-12)
+
+
+# ----------------------------------------------------------------- planted mistakes
+
+def test_planted_beta_sign_error_is_caught(monkeypatch):
+    real = orc.pool_head
+
+    def bad(*a, **kw):
+        P = real(*a, **kw)
+        P.beta = -P.beta
+        return P
+    monkeypatch.setattr(orc, "pool_head", bad)
+    with pytest.raises(AssertionError):
+        test_constant_key_blocks_make_compression_exact("topk", 0.25)
+
+
+def test_planted_missing_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(orc, "default_scale", lambda d, s=None: 1.0)
+    with pytest.raises(AssertionError):
+        test_full_density_no_compression_is_dense_attention(256, 16, 64)
+
+
+def test_planted_unweighted_summary_is_caught(monkeypatch):
+    real = orc.pool_head
+
+    def bad(q, k, v, n_sink, scale=None, block=64, mode="reweight"):
+        P = real(q, k, v, n_sink, scale, block, mode)
+        nb = P.qbar.shape[0]
+        P.vtil = v[: nb * block].reshape(nb, block, -1).mean(1)
+        return P
+    monkeypatch.setattr(orc, "pool_head", bad)
+    with pytest.raises(AssertionError):
+        test_anchor_query_rows_are_exact()
+
+
+def test_planted_unsorted_split_is_caught(monkeypatch):
+    """Splitting by token order instead of by projection must break the arc pin."""
+    real = orc.split_node
+
+    def bad(x, members, block=64):
+        sp = real(x, members, block)
+        members = np.sort(np.asarray(members))
+        cut = len(sp.left)
+        return orc.Split(members[:cut], members[cut:], sp.split_value, sp.proj, sp.gap, sp.skew)
+    monkeypatch.setattr(orc, "split_node", bad)
+    with pytest.raises(AssertionError):
+        test_reblock_arc_hand_derived()
+
+
+def test_planted_wrong_whitening_side_is_caught(monkeypatch):
+    """Whitening with the queries' own second moment instead of the keys' must break the
+    Mahalanobis-cosine pin."""
+    monkeypatch.setattr(orc, "key_second_moment", lambda kv: np.eye(kv.shape[1]))
+    with pytest.raises(AssertionError):
+        test_whitening_is_mahalanobis_cosine_via_reblock()
+
+
+def test_whitening_is_mahalanobis_cosine_via_reblock():
+    """The partition of a node of two blocks equals the one computed from the
+    Mahalanobis Gram matrix G_ij = q_i^T M q_j / (|q_i|_M |q_j|_M): the top eigenvector of
+    the doubly centred G gives the same projections up to sign (kernel-PCA identity)."""
+    rng = np.random.default_rng(31)
+    d = 12
+    q = rng.standard_normal((128, d)) * np.linspace(0.3, 3.0, d)
+    k = rng.standard_normal((128, d)) @ rng.standard_normal((d, d))
+    rb = orc.reblock_head(q, k, 0)
+    M = k.T @ k / 128.0
+    G = q @ M @ q.T
+    nrm = np.sqrt(np.diag(G))
+    G = G / np.outer(nrm, nrm)
+    J = np.eye(128) - 1.0 / 128
+    w, U = np.linalg.eigh(J @ G @ J)
+    p = U[:, -1]
+    low = set(np.argsort(p)[:64].tolist())
+    left = set(rb.splits[(0, 0)].left.tolist())
+    assert left == low or left == set(range(128)) - low
