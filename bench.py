@@ -1,0 +1,375 @@
+"""Benchmark: block-sparse video attention forward on the 1152x640, 243-frame clip shape.
+
+One step = one whole forward through the C ABI (pool + score/select + exact+compressed
+attention) of B=1, H=24, d=128, 175,680 video tokens (61 x 72 x 40) + 512 sink rows at
+top-k 10% with the Spark-Reweight compressed branch, inputs resident in HBM. Inputs are
+3.2 GB, larger than the 126 MB L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling); the
+only collectives are the timing barrier and the max-over-ranks of the elapsed time.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call & dense-equiv TFLOP/s of sparse attn fwd at 10% density, N=175,680"
+B, H, NV, NS, D = 1, 24, 175680, 512, 128
+N = NV + NS
+RATIO = 0.1
+WORKLOAD = ("1152x640 243-frame clip: B=1 H=24 d=128, 61x72x40=175680 video tokens + 512 sink "
+            "rows, 64-token blocks, top-k 10%, exact + Spark-Reweight compressed branch, bf16 in/out")
+
+
+def flop_counts(nb, k, ns=NS, d=D, h=H, b=B):
+    """Algorithmic FLOPs of one forward (4*d per query-key pair: QK^T and PV)."""
+    nv = nb * 64
+    n = nv + ns
+    exact = b * h * nb * k * 4 * 64 * 64 * d
+    sink_keys = b * h * nv * ns * 4 * d          # video queries x dense keys
+    sink_queries = b * h * ns * n * 4 * d        # dense queries x all keys
+    compressed = b * h * nv * (nb - k) * 4 * d   # video queries x unselected pooled entries
+    dense_equiv = 4 * b * h * n * n * d
+    return dict(exact=exact, sink=sink_keys + sink_queries, compressed=compressed,
+                selected=exact + sink_keys + sink_queries,
+                attn_total=exact + sink_keys + sink_queries + compressed, dense_equiv=dense_equiv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for ln in open(self.path):
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_video_mean_b200.spark as spark
+    from block_sparse_video_mean_b200.inputs import make_qkv
+
+    spark.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    Q, K, V = make_qkv(B, H, NV, NS, D, seed=args.seed + rank, device=dev)
+    cfg = spark.ForwardConfig("topk", RATIO, True)
+    plan = spark.SparkAttention(B, H, N, D, NS, cfg, dev)
+    nb, k = plan.nb, plan.kcap
+    fl = flop_counts(nb, k)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return plan.run(Q, K, V)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    err = spark.device_error(dev)
+    if err != 0:
+        raise RuntimeError(f"device error {err} ({spark.strerror(err)})")
+
+    # per-kernel timing of the dominant kernel (the attention launch), same stream
+    attn_ev = []
+
+    def step_timed():
+        perm = None
+        spark.pool_kv(Q, K, V, NS, spark.POOL_REWEIGHT, None, out=plan.pool)
+        spark.score_select(plan.pool["q_pool"], plan.pool["k_pool"], NS, N, plan.mode, RATIO,
+                           plan.kcap, None, out=(plan.idx, plan.cnt), ws=plan.sel_ws)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        spark.attn_fwd(Q, K, V, plan.idx, plan.cnt, NS, pack=plan.pool["pack"],
+                       beta=plan.pool["beta"], perm=perm, out=(plan.O, plan.lse))
+        e1.record(stream)
+        attn_ev.append((e0, e1))
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step_timed()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+
+    # end to end through the same calls with pinned host buffers
+    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+    hO = torch.empty(plan.O.shape, dtype=plan.O.dtype).pin_memory()
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+    def e2e_step():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        O, _ = plan.run(dQ, dK, dV)
+        hO.copy_(O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(2, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_ms /= e2e_steps
+
+    if rank != 0:
+        return None
+    hbm, bf16_peak, bf16_sust, peak_src = load_peaks()
+    achieved = fl["attn_total"] / (attn_ms * 1e-3) / 1e12
+    value = world * fl["dense_equiv"] / (ms_step * 1e-3) / 1e12
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s dense-equivalent (4*B*H*N^2*d / time, N=176,192)",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded block-correlated N(0,1) Q/K/V, generated on the device)",
+        "config": {"workload": WORKLOAD, "global_batch": world * B, "heads": H, "seq_len": N,
+                   "head_dim": D, "kept_blocks_per_query_block": k, "video_blocks": nb,
+                   "parallelism": f"independent problem per GPU x{world}",
+                   "l2": "inputs 3.2 GB > 126 MB L2; no flush needed"},
+        "selected_tflops": round(fl["selected"] / (ms_step * 1e-3) / 1e12, 2),
+        "attn_kernel_ms": round(attn_ms, 3),
+        "roofline": {"bound": "tensor", "kernel": "attn_mma_kernel<128>",
+                     "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / bf16_peak, 4),
+                     "peak_source": f"{peak_src} bf16 burst (sustained {bf16_sust})",
+                     "algorithmic_flops_per_launch": fl["attn_total"], "traffic": None},
+        "e2e": {"value": round(world * fl["dense_equiv"] / (e2e_ms * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s dense-equivalent, host buffers, copies inside the timed region",
+                "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
+                "d2h_bytes_per_step": plan.O.numel() * plan.O.element_size()},
+        "gpu_launches": args.steps * 5,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(Q[:, :1].cpu(), K[:, :1].cpu(), V[:, :1].cpu(),
+                                            args.cpu_blocks or 200)
+    return line
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(Qc, Kc, Vc, n_blocks, seed=0):
+    """The fp64 oracle, as it stands, on one head: pooling of all blocks, scores and top-k
+    of n_blocks sampled query blocks, and their exact + compressed attention. Reported as
+    dense-equivalent TFLOP/s of the sampled query rows (their share of 4*N^2*d)."""
+    import numpy as np
+
+    import oracle.spark_oracle as orc
+
+    t_start = time.perf_counter()
+    q, k, v = (orc.to_f64(t[0, 0]) for t in (Qc, Kc, Vc))
+    scale = 1.0 / math.sqrt(D)
+    P = orc.pool_head(q, k, v, NS, scale)
+    nb = P.qbar.shape[0]
+    rng = np.random.default_rng(seed)
+    blocks = rng.choice(nb, n_blocks, replace=False)
+    sel = orc.select_head(P.qbar, P.kbar, scale, "topk", RATIO, blocks)
+    for t, i in enumerate(blocks):
+        orc.attn_video_block(q, k, v, NS, i, sel[t], P, scale)
+    dt = time.perf_counter() - t_start
+    rows = n_blocks * 64
+    flops = 4.0 * rows * N * D
+    threads = None
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads") or 0) for i in threadpool_info()) or None
+    except Exception:
+        pass
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s dense-equivalent",
+            "cores": threads or os.cpu_count(), "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"1 of {H} heads: pooling of all {nb} blocks, top-k of {n_blocks} random "
+                      f"query blocks and their exact+compressed attention ({rows} query rows)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import torch
+    from block_sparse_video_mean_b200.inputs import make_qkv
+
+    # one head of the workload, drawn on the host
+    Q, K, V = make_qkv(1, 1, NV, NS, D, seed=args.seed, device="cpu")
+    vals = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = cpu_baseline(Q, K, V, args.cpu_blocks or 64, seed=i)
+        if i >= args.warmup:
+            vals.append(info)
+    value = statistics.mean(v["value"] for v in vals)
+    sec = statistics.mean(v["seconds"] for v in vals)
+    cb = dict(info)
+    cb["value"] = round(value, 6)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6),
+        "unit": "TFLOP/s dense-equivalent", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded block-correlated N(0,1) Q/K/V, one head drawn on the host)",
+        "config": {"workload": WORKLOAD, "sample": info["sample"]},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s dense-equivalent",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="spark", choices=["spark", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-blocks", type=int, default=0,
+                    help="query blocks in the oracle sample (default: 200 for cpu_baseline, 64 per reference step)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "spark" and args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    pg = False
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        pg = True
+    try:
+        line = run_gpu(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,259 @@
+// Block scores and selection: top-k keep ratio and the Sol-Attn per-head threshold.
+//
+// Method: "ComfyUI adds a core sparse-attention node and the Comfy Compiler", section
+// "Block-sparse attention: one node, three backends": top-k keeps a fixed share of key
+// blocks per query block; Sol-Attn keeps the blocks whose score lies tau standard
+// deviations above the head's score mean.
+//
+// Scores S[i, j] = qbar_i . kbar_j * scale are formed in fp32 FMA (not on the tensor
+// pipe: a bf16/tf32 product would move scores by ~1e-3, far beyond the 1e-4 window in
+// which two blocks count as tied). A CTA holds the score rows of RT query blocks in
+// shared memory as order-preserving uint32 keys; one warp per row then finds the k-th
+// largest key by a 4-pass MSB radix select over warp-private 256-bin histograms, and
+// writes the kept indices in ascending order with ballots (ties: lower index first).
+#pragma once
+#include "spark_common.cuh"
+
+namespace spark {
+
+constexpr int kSelThreads = 256;
+constexpr int kSelJT = 64;  // score columns per staged kbar tile
+constexpr int kSelKT = kSelJT + 1;  // padded row stride of the transposed tile (no bank conflicts)
+
+// ---------------------------------------------------------------- tau: per-head moments
+// acc[bh] += sum over the (r, c) entries of one 32 x 32 tile of Mq o Mk, where
+// Mq = sum_i qbar_i qbar_i^T and Mk = sum_j kbar_j kbar_j^T (fp64). Summed over tiles,
+// acc = tr(Mq Mk) = sum_{i,j} (qbar_i . kbar_j)^2.
+template <int D>
+__global__ void __launch_bounds__(256) moments_kernel(const float* __restrict__ q_pool,
+                                                      const float* __restrict__ k_pool, int nb,
+                                                      double* __restrict__ acc) {
+  constexpr int T = 32;
+  constexpr int TPD = D / T;
+  const int tr = blockIdx.x / TPD, tc = blockIdx.x % TPD;
+  const size_t bh = blockIdx.y;
+  __shared__ float qa[T][T + 1], qb[T][T + 1], ka[T][T + 1], kb[T][T + 1];
+  __shared__ double red[8];
+  const int tid = threadIdx.x;
+  const int r = tid / 8, c0 = (tid % 8) * 4;  // each thread: row r, columns c0..c0+3
+  double mq[4] = {0, 0, 0, 0}, mk[4] = {0, 0, 0, 0};
+  const float* qp = q_pool + bh * (size_t)nb * D;
+  const float* kp = k_pool + bh * (size_t)nb * D;
+  for (int b0 = 0; b0 < nb; b0 += T) {
+    // stage 32 blocks x 32 columns of each operand (rows tr*T.., cols tc*T..)
+    for (int e = tid; e < T * T; e += 256) {
+      const int bb = e / T, cc = e % T;
+      const bool ok = b0 + bb < nb;
+      const size_t o = (size_t)(b0 + bb) * D;
+      qa[bb][cc] = ok ? qp[o + tr * T + cc] : 0.f;
+      qb[bb][cc] = ok ? qp[o + tc * T + cc] : 0.f;
+      ka[bb][cc] = ok ? kp[o + tr * T + cc] : 0.f;
+      kb[bb][cc] = ok ? kp[o + tc * T + cc] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int bb = 0; bb < T; ++bb) {
+      const double xq = qa[bb][r], xk = ka[bb][r];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        mq[u] = fma(xq, (double)qb[bb][c0 + u], mq[u]);
+        mk[u] = fma(xk, (double)kb[bb][c0 + u], mk[u]);
+      }
+    }
+    __syncthreads();
+  }
+  double part = 0.0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) part = fma(mq[u], mk[u], part);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+  if ((tid & 31) == 0) red[tid >> 5] = part;
+  __syncthreads();
+  if (tid == 0) {
+    double t = 0.0;
+    for (int w = 0; w < 8; ++w) t += red[w];
+    atomicAdd(acc + bh, t);
+  }
+}
+
+// thr[bh] = mu + tau * sigma with mu = scale * (sum qbar) . (sum kbar) / nb^2 and
+// sigma^2 = scale^2 * tr(Mq Mk) / nb^2 - mu^2 (population moments of all nb^2 scores).
+template <int D>
+__global__ void __launch_bounds__(D) tau_threshold_kernel(const float* __restrict__ q_pool,
+                                                          const float* __restrict__ k_pool, int nb,
+                                                          const double* __restrict__ acc,
+                                                          double scale, double tau,
+                                                          double* __restrict__ thr) {
+  __shared__ double red[D / 32];
+  const size_t bh = blockIdx.x;
+  const int c = threadIdx.x;
+  const float* qp = q_pool + bh * (size_t)nb * D;
+  const float* kp = k_pool + bh * (size_t)nb * D;
+  double sq = 0.0, sk = 0.0;
+  for (int b = 0; b < nb; ++b) {
+    sq += qp[(size_t)b * D + c];
+    sk += kp[(size_t)b * D + c];
+  }
+  double p = sq * sk;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+  if ((c & 31) == 0) red[c >> 5] = p;
+  __syncthreads();
+  if (c == 0) {
+    double dot = 0.0;
+    for (int w = 0; w < D / 32; ++w) dot += red[w];
+    const double n2 = (double)nb * (double)nb;
+    const double mu = scale * dot / n2;
+    const double es2 = scale * scale * acc[bh] / n2;
+    const double var = es2 - mu * mu;
+    thr[bh] = mu + tau * sqrt(var > 0.0 ? var : 0.0);
+  }
+}
+
+// ---------------------------------------------------------------- scores + selection
+struct SelectParams {
+  const float* q_pool;
+  const float* k_pool;
+  int32_t* idx;
+  int32_t* cnt;
+  const double* thr;  // [B*H] (tau mode)
+  int nb, kcap, k, mode, rt;
+  float scale;
+};
+
+// Dynamic shared memory: keys[rt][nbp] | qs[rt][D] | kt[D][kSelKT] | hist[8][256].
+template <int D>
+__global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int RT = p.rt, nb = p.nb;
+  const int nbp = (nb + 3) & ~3;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
+  float* qs = reinterpret_cast<float*>(keys + (size_t)RT * nbp);
+  float* kt = qs + RT * D;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(kt + D * kSelKT);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t bh = blockIdx.y;
+  const int row0 = blockIdx.x * RT;
+  const int nrows = min(RT, nb - row0);
+  const float* qp = p.q_pool + bh * (size_t)nb * D;
+  const float* kp = p.k_pool + bh * (size_t)nb * D;
+
+  for (int e = tid; e < RT * D; e += kSelThreads) {
+    const int r = e / D;
+    qs[e] = r < nrows ? qp[(size_t)(row0 + r) * D + (e % D)] : 0.f;
+  }
+  // ---- scores: thread -> column j = tid % 64 of the tile, rows rg, rg + 4, ...
+  const int jj = tid % kSelJT, rg = tid / kSelJT;  // rg in [0, 4)
+  for (int j0 = 0; j0 < nb; j0 += kSelJT) {
+    __syncthreads();  // kt reuse
+    for (int e = tid; e < kSelJT * D; e += kSelThreads) {
+      const int j = e / D, c = e % D;  // coalesced read of kbar rows, transposed store
+      kt[c * kSelKT + j] = (j0 + j < nb) ? kp[(size_t)(j0 + j) * D + c] : 0.f;
+    }
+    __syncthreads();
+    const int j = j0 + jj;
+    for (int r = rg; r < RT; r += 4) {
+      float acc0 = 0.f, acc1 = 0.f;
+      const float* qr = qs + r * D;
+#pragma unroll 8
+      for (int c = 0; c < D; c += 2) {
+        acc0 = fmaf(qr[c], kt[c * kSelKT + jj], acc0);
+        acc1 = fmaf(qr[c + 1], kt[(c + 1) * kSelKT + jj], acc1);
+      }
+      if (j < nb && r < nrows) keys[(size_t)r * nbp + j] = float_to_key((acc0 + acc1) * p.scale);
+    }
+  }
+  __syncthreads();
+
+  // ---- selection: warp w handles rows w, w + 8, ...
+  uint32_t* h = hist + warp * 256;
+  for (int r = warp; r < nrows; r += kSelThreads / 32) {
+    const uint32_t* kr = keys + (size_t)r * nbp;
+    const size_t orow = bh * (size_t)nb + row0 + r;
+    int32_t* out = p.idx + orow * (size_t)p.kcap;
+    uint32_t T = 0;
+    int take_eq = 0;  // number of elements equal to T to keep (lowest indices first)
+    bool use_thr = (p.mode == SPARK_SELECT_TAU);
+    double thr = use_thr ? p.thr[bh] : 0.0;
+    if (!use_thr) {
+      uint32_t prefix = 0, mask = 0;
+      int kk = p.k;
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int b = lane; b < 256; b += 32) h[b] = 0;
+        __syncwarp();
+        for (int j = lane; j < nb; j += 32) {
+          const uint32_t key = kr[j];
+          if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        // lane l owns bins 255-8l .. 248-8l (descending); find the bin where the count
+        // from the top reaches kk.
+        uint32_t cntb[8];
+        uint32_t tot = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          cntb[t] = h[255 - 8 * lane - t];
+          tot += cntb[t];
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const uint32_t excl = incl - tot;
+        const bool mine = excl < (uint32_t)kk && (uint32_t)kk <= incl;
+        const uint32_t who = __ballot_sync(0xffffffffu, mine);
+        const int src = __ffs(who) - 1;
+        int bin = 0, above = 0;
+        if (lane == src) {
+          uint32_t run = excl;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (run + cntb[t] >= (uint32_t)kk) {
+              bin = 255 - 8 * lane - t;
+              above = (int)run;
+              break;
+            }
+            run += cntb[t];
+          }
+        }
+        bin = __shfl_sync(0xffffffffu, bin, src);
+        above = __shfl_sync(0xffffffffu, above, src);
+        kk -= above;
+        prefix |= (uint32_t)bin << shift;
+        mask |= 255u << shift;
+        __syncwarp();
+      }
+      T = prefix;
+      take_eq = kk;
+    }
+    // ---- ascending output pass
+    int written = 0, eq_seen = 0;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+      const int j = j0 + lane;
+      bool keep = false;
+      if (use_thr) {
+        keep = j < nb && (double)key_to_float(kr[j]) > thr;
+      } else {
+        const uint32_t key = j < nb ? kr[j] : 0u;
+        const bool eq = j < nb && key == T;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+        const int rank = eq_seen + __popc(eqm & lanemask_lt());
+        eq_seen += __popc(eqm);
+        keep = j < nb && (key > T || (eq && rank < take_eq));
+      }
+      const uint32_t km = __ballot_sync(0xffffffffu, keep);
+      const int pos = written + __popc(km & lanemask_lt());
+      if (keep && pos < p.kcap) out[pos] = j;
+      written += __popc(km);
+    }
+    if (lane == 0) {
+      if (written > p.kcap) set_error(SPARK_ECAPACITY);
+      p.cnt[orow] = min(written, p.kcap);
+    }
+  }
+}
+
+}  // namespace spark

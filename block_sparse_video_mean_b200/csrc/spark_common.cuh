@@ -1,0 +1,68 @@
+// Shared device helpers of the sm_100a kernels (no method arithmetic lives here).
+// Included once, by spark_lib.cu.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/spark.h"
+
+namespace spark {
+
+constexpr int kBlock = 64;
+
+// First device-side fault of any kernel (0 = none). Read and cleared by spark_device_error.
+// The library is one translation unit (spark_lib.cu includes every kernel header), so
+// this definition is unique.
+__device__ int g_error_word = 0;
+
+__device__ __forceinline__ void set_error(int code) { atomicCAS(&g_error_word, 0, code); }
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Order-preserving map of an fp32 value to uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_to_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(u);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+}  // namespace spark
+
+#define SPARK_LAUNCH_CHECK()                                  \
+  do {                                                        \
+    if (cudaPeekAtLastError() != cudaSuccess) {               \
+      cudaGetLastError();                                     \
+      return SPARK_ECUDA;                                     \
+    }                                                         \
+  } while (0)

@@ -1,0 +1,306 @@
+// libspark: the C ABI of include/spark.h. Host-side argument validation and launches;
+// every step of the computation runs in the kernels included below. The whole library
+// is this one translation unit.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "spark_common.cuh"
+#include "pool.cuh"
+#include "select.cuh"
+#include "attn_mma.cuh"
+#include "reblock.cuh"
+
+using namespace spark;
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t num_blocks(const spark_shape* s) {
+  const int64_t nv = (int64_t)s->N - s->n_sink;
+  return nv > 0 ? nv / kBlock : 0;
+}
+
+inline float eff_scale(const spark_shape* s) {
+  return s->scale > 0.f ? s->scale : 1.0f / std::sqrt((float)s->d);
+}
+
+// Shape checks shared by every call. Returns SPARK_OK or a negative status.
+int check_shape(const spark_shape* s) {
+  if (s == nullptr) return SPARK_EINVAL;
+  if (s->B < 0 || s->H < 0 || s->N < 0 || s->n_sink < 0 || s->n_sink > s->N) return SPARK_EINVAL;
+  if (!(std::isfinite(s->scale))) return SPARK_EINVAL;
+  if (s->block != kBlock) return SPARK_EUNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return SPARK_EUNSUPPORTED;
+  const int64_t bh = (int64_t)s->B * s->H;
+  if (bh > 65535) return SPARK_EUNSUPPORTED;                       // grid.y of the pooling kernels
+  if ((int64_t)s->N * s->d * bh > ((int64_t)1 << 40)) return SPARK_EUNSUPPORTED;
+  if ((int64_t)s->N > ((int64_t)1 << 30)) return SPARK_EUNSUPPORTED;
+  return SPARK_OK;
+}
+
+inline bool empty(const spark_shape* s) { return (int64_t)s->B * s->H * s->N == 0; }
+
+// Score rows a select CTA keeps in shared memory (largest of 8, 4, 2, 1 that fits).
+int select_rows_per_cta(int nb, int d, size_t* smem) {
+  const size_t nbp = (size_t)((nb + 3) & ~3);
+  for (int rt = 8; rt >= 1; rt >>= 1) {
+    const size_t bytes = (size_t)rt * nbp * 4 + (size_t)rt * d * 4 + (size_t)d * kSelKT * 4 +
+                         (kSelThreads / 32) * 256 * 4;
+    if (bytes <= 200 * 1024) {
+      *smem = bytes;
+      return rt;
+    }
+  }
+  return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t spark_num_blocks(const spark_shape* s) {
+  if (check_shape(s) != SPARK_OK) return 0;
+  return (int32_t)num_blocks(s);
+}
+
+int32_t spark_topk_count(double ratio, int32_t nb) {
+  if (!(ratio > 0.0 && ratio <= 1.0)) return -1;
+  if (nb <= 0) return 0;
+  double k = std::ceil(ratio * (double)nb - 1e-9);
+  if (k < 1.0) k = 1.0;
+  if (k > nb) k = nb;
+  return (int32_t)k;
+}
+
+size_t spark_workspace_bytes(const spark_shape* s, int call_id) {
+  if (check_shape(s) != SPARK_OK) return 0;
+  const size_t bh = (size_t)s->B * s->H;
+  const size_t nb = (size_t)num_blocks(s);
+  switch (call_id) {
+    case SPARK_CALL_POOL:
+      return 2 * bh * nb * s->d * sizeof(uint16_t);
+    case SPARK_CALL_SELECT:
+      return ((2 * bh * sizeof(double)) + 255) & ~(size_t)255;
+    case SPARK_CALL_ATTN:
+      return 0;
+    case SPARK_CALL_REBLOCK:
+      return reblock_workspace_bytes(s->B * s->H, (int)nb, s->d);
+    default:
+      return 0;
+  }
+}
+
+int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                  int pool_mode, float* q_pool, float* k_pool, float* v_summ, float* beta,
+                  float* anchor, void* pool_pack, size_t pool_pack_bytes, void* stream) {
+  int st = check_shape(s);
+  if (st != SPARK_OK) return st;
+  if (pool_mode != SPARK_POOL_REWEIGHT && pool_mode != SPARK_POOL_MEAN) return SPARK_EINVAL;
+  if (empty(s)) return SPARK_OK;
+  const int nb = (int)num_blocks(s);
+  const int bh = s->B * s->H;
+  if (!Q || !K || !V || !anchor) return SPARK_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(anchor)) return SPARK_EINVAL;
+  cudaStream_t cs = as_stream(stream);
+  if (nb == 0) {
+    if (cudaMemsetAsync(anchor, 0, (size_t)bh * s->d * sizeof(float), cs) != cudaSuccess) return SPARK_ECUDA;
+    return SPARK_OK;
+  }
+  if (!q_pool || !k_pool || !v_summ || !beta || !pool_pack) return SPARK_EINVAL;
+  if (!aligned16(q_pool) || !aligned16(k_pool) || !aligned16(v_summ) || !aligned16(pool_pack))
+    return SPARK_EINVAL;
+  if (pool_pack_bytes < spark_workspace_bytes(s, SPARK_CALL_POOL)) return SPARK_EINVAL;
+  uint16_t* k16 = static_cast<uint16_t*>(pool_pack);
+  uint16_t* v16 = k16 + (size_t)bh * nb * s->d;
+  const float scale = eff_scale(s);
+  dim3 grid((nb + kPoolWarps - 1) / kPoolWarps, bh);
+  if (s->d == 128) {
+    pool_q_kernel<128><<<grid, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nb);
+    anchor_kernel<128><<<bh, 256, 0, cs>>>(q_pool, anchor, nb);
+    pool_kv_kernel<128><<<grid, kPoolWarps * 32, 0, cs>>>(K, V, anchor, k_pool, v_summ, beta, k16,
+                                                          v16, s->N, nb, scale, pool_mode);
+  } else {
+    pool_q_kernel<64><<<grid, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nb);
+    anchor_kernel<64><<<bh, 256, 0, cs>>>(q_pool, anchor, nb);
+    pool_kv_kernel<64><<<grid, kPoolWarps * 32, 0, cs>>>(K, V, anchor, k_pool, v_summ, beta, k16,
+                                                         v16, s->N, nb, scale, pool_mode);
+  }
+  SPARK_LAUNCH_CHECK();
+  return SPARK_OK;
+}
+
+int spark_score_select(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
+                       double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
+                       size_t ws_bytes, void* stream) {
+  int st = check_shape(s);
+  if (st != SPARK_OK) return st;
+  const int nb = (int)num_blocks(s);
+  const int bh = s->B * s->H;
+  int k = 0;
+  if (mode == SPARK_SELECT_TOPK_RATIO) {
+    k = spark_topk_count(param, nb);
+    if (k < 0) return SPARK_EINVAL;
+    if (kcap < k) return SPARK_EINVAL;
+  } else if (mode == SPARK_SELECT_TAU) {
+    if (!std::isfinite(param)) return SPARK_EINVAL;
+  } else {
+    return SPARK_EINVAL;
+  }
+  if (kcap < 0) return SPARK_EINVAL;
+  if (empty(s) || nb == 0) return SPARK_OK;
+  if (kcap < 1) return SPARK_EINVAL;
+  if (!q_pool || !k_pool || !idx || !cnt) return SPARK_EINVAL;
+  if (!aligned16(q_pool) || !aligned16(k_pool)) return SPARK_EINVAL;
+  size_t smem = 0;
+  const int rt = select_rows_per_cta(nb, s->d, &smem);
+  if (rt == 0) return SPARK_EUNSUPPORTED;
+  cudaStream_t cs = as_stream(stream);
+  const float scale = eff_scale(s);
+  double* thr = nullptr;
+  if (mode == SPARK_SELECT_TAU) {
+    if (!ws || ws_bytes < spark_workspace_bytes(s, SPARK_CALL_SELECT) || !aligned16(ws))
+      return SPARK_EINVAL;
+    double* acc = static_cast<double*>(ws);
+    thr = acc + bh;
+    if (cudaMemsetAsync(acc, 0, (size_t)bh * sizeof(double), cs) != cudaSuccess) return SPARK_ECUDA;
+    if (s->d == 128) {
+      moments_kernel<128><<<dim3(16, bh), 256, 0, cs>>>(q_pool, k_pool, nb, acc);
+      tau_threshold_kernel<128><<<bh, 128, 0, cs>>>(q_pool, k_pool, nb, acc, scale, param, thr);
+    } else {
+      moments_kernel<64><<<dim3(4, bh), 256, 0, cs>>>(q_pool, k_pool, nb, acc);
+      tau_threshold_kernel<64><<<bh, 64, 0, cs>>>(q_pool, k_pool, nb, acc, scale, param, thr);
+    }
+    SPARK_LAUNCH_CHECK();
+  }
+  SelectParams sp;
+  sp.q_pool = q_pool;
+  sp.k_pool = k_pool;
+  sp.idx = idx;
+  sp.cnt = cnt;
+  sp.thr = thr;
+  sp.nb = nb;
+  sp.kcap = kcap;
+  sp.k = k;
+  sp.mode = mode;
+  sp.rt = rt;
+  sp.scale = scale;
+  dim3 grid((nb + rt - 1) / rt, bh);
+  if (s->d == 128) {
+    cudaFuncSetAttribute(score_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    score_select_kernel<128><<<grid, kSelThreads, smem, cs>>>(sp);
+  } else {
+    cudaFuncSetAttribute(score_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    score_select_kernel<64><<<grid, kSelThreads, smem, cs>>>(sp);
+  }
+  SPARK_LAUNCH_CHECK();
+  return SPARK_OK;
+}
+
+int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                   const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
+                   const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,
+                   size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int st = check_shape(s);
+  if (st != SPARK_OK) return st;
+  if (empty(s)) return SPARK_OK;
+  const int nb = (int)num_blocks(s);
+  const int bh = s->B * s->H;
+  if (!Q || !K || !V || !O) return SPARK_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARK_EINVAL;
+  if (nb > 0) {
+    if (!idx || !cnt || kcap < 1) return SPARK_EINVAL;
+    if (pool_pack && (!beta || !aligned16(pool_pack))) return SPARK_EINVAL;
+  }
+  const int nv = nb * kBlock;
+  const int n_dq = (s->N - nv + kBlock - 1) / kBlock;
+  const int64_t items = (int64_t)bh * (n_dq + nb);
+  if (items > 0x7fffffff) return SPARK_EUNSUPPORTED;
+  AttnParams ap;
+  ap.Q = Q;
+  ap.K = K;
+  ap.V = V;
+  ap.idx = idx;
+  ap.cnt = cnt;
+  ap.kp16 = nb > 0 ? static_cast<const uint16_t*>(pool_pack) : nullptr;
+  ap.vp16 = ap.kp16 ? ap.kp16 + (size_t)bh * nb * s->d : nullptr;
+  ap.beta = beta;
+  ap.perm = perm;
+  ap.O = O;
+  ap.lse = lse;
+  ap.N = s->N;
+  ap.nb = nb;
+  ap.kcap = kcap;
+  ap.BH = bh;
+  ap.n_dq = n_dq;
+  ap.scale_log2 = eff_scale(s) * kLog2e;
+  cudaStream_t cs = as_stream(stream);
+  const size_t bitmap = (size_t)((nb + 31) / 32) * 4;
+  if (s->d == 128) {
+    const size_t smem = MmaAttn<128>::kSmemFixed + bitmap;
+    if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
+    cudaFuncSetAttribute(attn_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_mma_kernel<128><<<(unsigned)items, 128, smem, cs>>>(ap);
+  } else {
+    const size_t smem = MmaAttn<64>::kSmemFixed + bitmap;
+    if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
+    cudaFuncSetAttribute(attn_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_mma_kernel<64><<<(unsigned)items, 128, smem, cs>>>(ap);
+  }
+  SPARK_LAUNCH_CHECK();
+  return SPARK_OK;
+}
+
+int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                  int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
+                  size_t ws_bytes, void* stream) {
+  int st = check_shape(s);
+  if (st != SPARK_OK) return st;
+  if (empty(s)) return SPARK_OK;
+  if (!Q || !K || !V || !Qp || !Kp || !Vp) return SPARK_EINVAL;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(Qp) || !aligned16(Kp) ||
+      !aligned16(Vp))
+    return SPARK_EINVAL;
+  const int nb = (int)num_blocks(s);
+  if (nb > 0 && !perm) return SPARK_EINVAL;
+  if (ws_bytes < spark_workspace_bytes(s, SPARK_CALL_REBLOCK)) return SPARK_EINVAL;
+  if (spark_workspace_bytes(s, SPARK_CALL_REBLOCK) > 0 && (!ws || !aligned16(ws))) return SPARK_EINVAL;
+  return reblock_launch(s->B * s->H, s->N, nb, s->d, Q, K, V, perm, Qp, Kp, Vp, tree, ws,
+                        as_stream(stream));
+}
+
+int spark_device_error(int32_t* host_word, void* stream) {
+  cudaStream_t cs = as_stream(stream);
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_error_word, sizeof(int32_t), 0, cudaMemcpyDeviceToHost, cs) !=
+      cudaSuccess)
+    return SPARK_ECUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return SPARK_ECUDA;
+  const int32_t zero = 0;
+  if (cudaMemcpyToSymbolAsync(g_error_word, &zero, sizeof(int32_t), 0, cudaMemcpyHostToDevice, cs) !=
+      cudaSuccess)
+    return SPARK_ECUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return SPARK_ECUDA;
+  if (host_word) *host_word = v;
+  return SPARK_OK;
+}
+
+const char* spark_strerror(int status) {
+  switch (status) {
+    case SPARK_OK: return "ok";
+    case SPARK_EINVAL: return "invalid argument (shape, pointer, alignment, ratio/tau or kcap)";
+    case SPARK_EUNSUPPORTED: return "unsupported (d must be 64 or 128, block 64, sizes within limits)";
+    case SPARK_ECUDA: return "CUDA launch or copy failed";
+    case SPARK_ETIMEOUT: return "device: a bounded wait gave up";
+    case SPARK_EDEVICE_INDEX: return "device: block index or count out of range (skipped)";
+    case SPARK_ECAPACITY: return "device: more blocks kept than kcap (row truncated)";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,283 @@
+"""Thin Python binding of libspark (include/spark.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA library; this module allocates the
+caller-owned buffers with torch, passes raw device pointers and the current stream, and
+turns negative status codes into exceptions. There is no fallback: without the built
+library (``python -m block_sparse_video_mean_b200.build``) and a CUDA device nothing here
+computes anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libspark.so")
+
+SPARK_OK = 0
+SELECT_TOPK_RATIO = 0
+SELECT_TAU = 1
+POOL_REWEIGHT = 0
+POOL_MEAN = 1
+CALL_POOL, CALL_SELECT, CALL_ATTN, CALL_REBLOCK = 0, 1, 2, 3
+BLOCK = 64
+
+EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
+           "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
+           "spark_strerror")
+
+
+class SparkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: status {status} ({strerror(status)})")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libspark.so from the package directory (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m block_sparse_video_mean_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, Z, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
+    SP = ctypes.POINTER(Shape)
+    lib.spark_num_blocks.argtypes = [SP]
+    lib.spark_num_blocks.restype = ctypes.c_int32
+    lib.spark_workspace_bytes.argtypes = [SP, I]
+    lib.spark_workspace_bytes.restype = Z
+    lib.spark_topk_count.argtypes = [D, ctypes.c_int32]
+    lib.spark_topk_count.restype = ctypes.c_int32
+    lib.spark_pool_kv.argtypes = [SP, P, P, P, I, P, P, P, P, P, P, Z, P]
+    lib.spark_pool_kv.restype = I
+    lib.spark_score_select.argtypes = [SP, P, P, I, D, ctypes.c_int32, P, P, P, Z, P]
+    lib.spark_score_select.restype = I
+    lib.spark_attn_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_int32, P, P, P, P, P, P, Z, P]
+    lib.spark_attn_fwd.restype = I
+    lib.spark_reblock.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
+    lib.spark_reblock.restype = I
+    lib.spark_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
+    lib.spark_device_error.restype = I
+    lib.spark_strerror.argtypes = [I]
+    lib.spark_strerror.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def strerror(status: int) -> str:
+    return load().spark_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != SPARK_OK:
+        raise SparkError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def make_shape(B, H, N, d, n_sink, scale=None) -> Shape:
+    return Shape(B, H, N, d, n_sink, BLOCK, float(scale) if scale else 0.0)
+
+
+def num_blocks(shape: Shape) -> int:
+    return int(load().spark_num_blocks(ctypes.byref(shape)))
+
+
+def topk_count(ratio: float, nb: int) -> int:
+    return int(load().spark_topk_count(float(ratio), int(nb)))
+
+
+def workspace_bytes(shape: Shape, call_id: int) -> int:
+    return int(load().spark_workspace_bytes(ctypes.byref(shape), int(call_id)))
+
+
+def device_error(device=None) -> int:
+    word = ctypes.c_int32(0)
+    _check(load().spark_device_error(ctypes.byref(word), _stream(device)), "spark_device_error")
+    return int(word.value)
+
+
+def _shape_of(Q, n_sink, scale):
+    B, H, N, d = Q.shape
+    return make_shape(B, H, N, d, n_sink, scale)
+
+
+def _need(t, name):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+
+
+# --------------------------------------------------------------------------- the four calls
+
+def pool_kv(Q, K, V, n_sink, pool_mode=POOL_REWEIGHT, scale=None, out=None):
+    """spark_pool_kv: returns dict(q_pool, k_pool, v_summ, beta, anchor, pack)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, n)
+    shape = _shape_of(Q, n_sink, scale)
+    B, H, N, d = Q.shape
+    nb = num_blocks(shape)
+    dev = Q.device
+    if out is None:
+        out = dict(
+            q_pool=torch.empty((B, H, nb, d), dtype=torch.float32, device=dev),
+            k_pool=torch.empty((B, H, nb, d), dtype=torch.float32, device=dev),
+            v_summ=torch.empty((B, H, nb, d), dtype=torch.float32, device=dev),
+            beta=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
+            anchor=torch.empty((B, H, d), dtype=torch.float32, device=dev),
+            pack=torch.empty(max(workspace_bytes(shape, CALL_POOL), 16), dtype=torch.uint8, device=dev),
+        )
+    _check(load().spark_pool_kv(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), int(pool_mode),
+                                _ptr(out["q_pool"]), _ptr(out["k_pool"]), _ptr(out["v_summ"]),
+                                _ptr(out["beta"]), _ptr(out["anchor"]), _ptr(out["pack"]),
+                                out["pack"].numel(), _stream(dev)), "spark_pool_kv")
+    return out
+
+
+def score_select(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, out=None, ws=None):
+    """spark_score_select: returns (idx [B,H,nb,kcap] int32, cnt [B,H,nb] int32)."""
+    B, H, nb, d = q_pool.shape
+    shape = make_shape(B, H, N, d, n_sink, scale)
+    dev = q_pool.device
+    if kcap is None:
+        kcap = topk_count(param, nb) if mode == SELECT_TOPK_RATIO else max(nb, 1)
+    if out is None:
+        out = (torch.empty((B, H, nb, max(kcap, 1)), dtype=torch.int32, device=dev),
+               torch.empty((B, H, nb), dtype=torch.int32, device=dev))
+    if ws is None and mode == SELECT_TAU:
+        ws = torch.empty(max(workspace_bytes(shape, CALL_SELECT), 16), dtype=torch.uint8, device=dev)
+    idx, cnt = out
+    _check(load().spark_score_select(ctypes.byref(shape), _ptr(q_pool), _ptr(k_pool), int(mode),
+                                     float(param), int(kcap), _ptr(idx), _ptr(cnt), _ptr(ws),
+                                     0 if ws is None else ws.numel(), _stream(dev)),
+           "spark_score_select")
+    return idx, cnt
+
+
+def attn_fwd(Q, K, V, idx, cnt, n_sink, pack=None, beta=None, perm=None, scale=None,
+             out=None, lse=True):
+    """spark_attn_fwd: returns (O bf16 [B,H,N,d], LSE fp32 [B,H,N] or None)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, n)
+    shape = _shape_of(Q, n_sink, scale)
+    B, H, N, d = Q.shape
+    dev = Q.device
+    if out is None:
+        out = (torch.empty_like(Q),
+               torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse else None)
+    O, L = out
+    kcap = idx.shape[-1] if idx is not None else 1
+    _check(load().spark_attn_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                                 _ptr(cnt), int(kcap), _ptr(pack), _ptr(beta), _ptr(perm), _ptr(O),
+                                 _ptr(L), None, 0, _stream(dev)), "spark_attn_fwd")
+    return O, L
+
+
+def reblock(Q, K, V, n_sink, tree=False, out=None, ws=None):
+    """spark_reblock: returns dict(perm, Qp, Kp, Vp, tree or None)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, n)
+    shape = _shape_of(Q, n_sink, None)
+    B, H, N, d = Q.shape
+    nb = num_blocks(shape)
+    dev = Q.device
+    levels = 0 if nb <= 1 else math.ceil(math.log2(nb))
+    if out is None:
+        out = dict(perm=torch.empty((B, H, nb * BLOCK), dtype=torch.int32, device=dev),
+                   Qp=torch.empty_like(Q), Kp=torch.empty_like(K), Vp=torch.empty_like(V),
+                   tree=torch.empty((B, H, levels + 1, nb * BLOCK), dtype=torch.int32, device=dev)
+                   if tree else None)
+    if ws is None:
+        ws = torch.empty(max(workspace_bytes(shape, CALL_REBLOCK), 16), dtype=torch.uint8, device=dev)
+    _check(load().spark_reblock(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(out["perm"]),
+                                _ptr(out["Qp"]), _ptr(out["Kp"]), _ptr(out["Vp"]),
+                                _ptr(out.get("tree")), _ptr(ws), ws.numel(), _stream(dev)),
+           "spark_reblock")
+    return out
+
+
+# --------------------------------------------------------------------------- whole forward
+
+@dataclass
+class ForwardConfig:
+    mode: str = "topk"          # "topk" (keep ratio) or "tau" (Sol-Attn threshold)
+    param: float = 0.1          # ratio or tau
+    compressed: bool = True     # Spark-Reweight compressed branch on/off
+    pool_mode: str = "reweight"  # "reweight" or "mean"
+    reblock: bool = False       # Spark-Reblock partition first (q_reuse_k)
+    scale: float | None = None
+    kcap: int | None = None     # slots per selection row (default: k, or nb for tau)
+
+
+class SparkAttention:
+    """A planned forward of one shape: every buffer allocated once, then ``run`` issues the
+    library calls back to back on the current stream (no host synchronisation)."""
+
+    def __init__(self, B, H, N, d, n_sink, cfg: ForwardConfig, device="cuda"):
+        self.cfg = cfg
+        self.n_sink = n_sink
+        self.shape = make_shape(B, H, N, d, n_sink, cfg.scale)
+        self.nb = nb = num_blocks(self.shape)
+        dev = torch.device(device)
+        self.mode = SELECT_TOPK_RATIO if cfg.mode == "topk" else SELECT_TAU
+        if cfg.kcap is not None:
+            self.kcap = cfg.kcap
+        else:
+            self.kcap = max(topk_count(cfg.param, nb) if self.mode == SELECT_TOPK_RATIO else nb, 1)
+        self.pool_mode = POOL_REWEIGHT if cfg.pool_mode == "reweight" else POOL_MEAN
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.pool = dict(q_pool=torch.empty((B, H, nb, d), **f32), k_pool=torch.empty((B, H, nb, d), **f32),
+                         v_summ=torch.empty((B, H, nb, d), **f32), beta=torch.empty((B, H, nb), **f32),
+                         anchor=torch.empty((B, H, d), **f32),
+                         pack=torch.empty(max(workspace_bytes(self.shape, CALL_POOL), 16),
+                                          dtype=torch.uint8, device=dev))
+        self.idx = torch.empty((B, H, nb, self.kcap), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+        self.sel_ws = torch.empty(max(workspace_bytes(self.shape, CALL_SELECT), 16), dtype=torch.uint8, device=dev)
+        self.O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, H, N), **f32)
+        self.rb = None
+        if cfg.reblock:
+            levels = 0 if nb <= 1 else math.ceil(math.log2(nb))
+            self.rb = dict(perm=torch.empty((B, H, nb * BLOCK), dtype=torch.int32, device=dev),
+                           Qp=torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                           Kp=torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                           Vp=torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                           tree=None)
+            self.rb_ws = torch.empty(max(workspace_bytes(self.shape, CALL_REBLOCK), 16),
+                                     dtype=torch.uint8, device=dev)
+            self.levels = levels
+
+    def run(self, Q, K, V):
+        cfg = self.cfg
+        perm = None
+        if self.rb is not None:
+            reblock(Q, K, V, self.n_sink, out=self.rb, ws=self.rb_ws)
+            Q, K, V, perm = self.rb["Qp"], self.rb["Kp"], self.rb["Vp"], self.rb["perm"]
+        pool_kv(Q, K, V, self.n_sink, self.pool_mode, cfg.scale, out=self.pool)
+        score_select(self.pool["q_pool"], self.pool["k_pool"], self.n_sink, Q.shape[2], self.mode,
+                     cfg.param, self.kcap, cfg.scale, out=(self.idx, self.cnt), ws=self.sel_ws)
+        attn_fwd(Q, K, V, self.idx, self.cnt, self.n_sink,
+                 pack=self.pool["pack"] if cfg.compressed else None, beta=self.pool["beta"],
+                 perm=perm, scale=cfg.scale, out=(self.O, self.lse))
+        return self.O, self.lse

@@ -1,0 +1,164 @@
+/*
+ * spark.h — C ABI of the B200 (sm_100a) block-sparse video attention forward.
+ *
+ * The method: "Spark-H3: speeding up MiniMax-H3 in ComfyUI with block-sparse
+ * attention" (comfyui-wiki news, 2026-10-11), section "What Spark-Attn changes":
+ * an exact branch over the top-ranked key/value blocks and a compressed branch that
+ * covers the rest (Spark-Reweight), optionally over a data-dependent block layout
+ * (Spark-Reblock). Block selection follows "ComfyUI adds a core sparse-attention node
+ * and the Comfy Compiler" (comfyui-wiki news, 2026-09-08), section "Block-sparse
+ * attention: one node, three backends" (top-k keep ratio; Sol-Attn per-head tau;
+ * sink_conditioning), and the dense-row policy of the "H3 Optimizations" README,
+ * section "Nodes".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Q, K, V are contiguous [B, H, N, d] bf16 (passed as uint16_t bit patterns),
+ *   16-byte aligned. Per (b, h) the first nb*64 rows are video rows, nb =
+ *   floor((N - n_sink) / 64); all remaining rows (a ragged video tail shorter than
+ *   one block, then the n_sink sink/text rows) are dense rows: their queries attend
+ *   to every key and their keys are attended by every query. Dense rows are never
+ *   pooled, scored, compressed or reblocked.
+ * - block must be 64; d must be 64 or 128; scale <= 0 means 1/sqrt(d).
+ * - Every pointer is a device pointer owned by the caller; the library allocates
+ *   nothing, keeps no state beyond one device-side error word, and never
+ *   synchronises except in spark_device_error. Calls are asynchronous on `stream`
+ *   (a cudaStream_t, NULL = legacy default stream) and re-entrant.
+ * - Return value: SPARK_OK, or a negative status for arguments rejected on the host
+ *   (nothing is launched then). Faults found by a kernel (an out-of-range block index
+ *   supplied by the caller, a capacity overflow, a bounded wait that gave up) do not
+ *   abort the launch: the kernel skips the offending work and records the first such
+ *   status in the device error word, which spark_device_error reads and clears.
+ */
+#ifndef SPARK_H_
+#define SPARK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SPARK_OK 0
+#define SPARK_EINVAL (-1)        /* bad shape, null pointer, alignment, ratio/tau, kcap */
+#define SPARK_EUNSUPPORTED (-2)  /* d or block not supported, sizes beyond the limits */
+#define SPARK_ECUDA (-3)         /* a CUDA launch failed */
+#define SPARK_ETIMEOUT (-4)      /* device: a bounded wait gave up */
+#define SPARK_EDEVICE_INDEX (-5) /* device: a selected block index was out of range */
+#define SPARK_ECAPACITY (-6)     /* device: tau kept more blocks than kcap; list truncated */
+
+#define SPARK_SELECT_TOPK_RATIO 0
+#define SPARK_SELECT_TAU 1
+
+#define SPARK_POOL_REWEIGHT 0 /* Spark-Reweight: softmax-weighted value summary + log-mass bias */
+#define SPARK_POOL_MEAN 1     /* plain mean pooling: mean value, bias log(64) */
+
+#define SPARK_CALL_POOL 0
+#define SPARK_CALL_SELECT 1
+#define SPARK_CALL_ATTN 2
+#define SPARK_CALL_REBLOCK 3
+
+typedef struct spark_shape {
+  int32_t B, H, N, d; /* Q/K/V are [B, H, N, d] */
+  int32_t n_sink;     /* sink/text rows at the end of each (b, h) */
+  int32_t block;      /* video block size; must be 64 */
+  float scale;        /* softmax scale; <= 0 selects 1/sqrt(d) */
+} spark_shape;
+
+/* Number of full video blocks nb = floor((N - n_sink) / 64) (0 when N <= n_sink). */
+int32_t spark_num_blocks(const spark_shape* s);
+
+/* Bytes of the caller-owned buffer that call `call_id` needs:
+ *   SPARK_CALL_POOL    the pooled pack written by spark_pool_kv and read by
+ *                      spark_attn_fwd (bf16 copies of kbar and vtil, 2*B*H*nb*d*2 bytes);
+ *   SPARK_CALL_SELECT  scratch of spark_score_select (tau moments; 0 for top-k is fine
+ *                      but the tau size is returned);
+ *   SPARK_CALL_ATTN    scratch of spark_attn_fwd (0: it needs none);
+ *   SPARK_CALL_REBLOCK scratch of spark_reblock.
+ * Returns 0 for an invalid shape or call id. */
+size_t spark_workspace_bytes(const spark_shape* s, int call_id);
+
+/* Block-count rule of the top-k mode: k = min(nb, max(1, ceil(ratio*nb - 1e-9))),
+ * evaluated in double precision. Returns -1 for ratio outside (0, 1]. */
+int32_t spark_topk_count(double ratio, int32_t nb);
+
+/* Pooling, anchor and compressed-branch summaries ("What Spark-Attn changes",
+ * Spark-Reweight bullet and the figure caption after it).
+ * Per (b, h):  q_pool[i]  = mean of the 64 queries of video block i        fp32 [B,H,nb,d]
+ *              anchor     = mean of all video queries (= mean of q_pool)   fp32 [B,H,d]
+ *              s_j        = anchor . k_j * scale for every video key j
+ *              k_pool[i]  = mean of the 64 keys of block i                  fp32 [B,H,nb,d]
+ *              v_summ[i]  = sum_j softmax_i(s)_j v_j (REWEIGHT) | mean v     fp32 [B,H,nb,d]
+ *              beta[i]    = logsumexp_i(s) - anchor . k_pool[i] * scale      fp32 [B,H,nb]
+ *                           (REWEIGHT) | log(64) (MEAN)
+ * pool_pack (spark_workspace_bytes(s, SPARK_CALL_POOL) bytes) receives bf16 copies of
+ * k_pool and v_summ, the operands of the compressed branch in spark_attn_fwd.
+ * Any of q_pool/k_pool/v_summ/anchor may not be NULL; all are written. */
+int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                  int pool_mode, float* q_pool, float* k_pool, float* v_summ, float* beta,
+                  float* anchor, void* pool_pack, size_t pool_pack_bytes, void* stream);
+
+/* Block scores and selection ("Block-sparse attention: one node, three backends").
+ * S[i, j] = q_pool[i] . k_pool[j] * scale over video blocks, computed in fp32.
+ *   mode SPARK_SELECT_TOPK_RATIO, param = ratio in (0, 1]: keeps the k =
+ *       spark_topk_count(ratio, nb) largest scores of each row, ties to the lower j;
+ *       requires kcap >= k.
+ *   mode SPARK_SELECT_TAU, param = tau (finite): keeps S[i, j] > mu + tau * sigma,
+ *       mu and sigma (population) over all nb^2 scores of the head, obtained in fp64
+ *       from the d x d second moments of q_pool and k_pool. No per-row floor: a row
+ *       may keep nothing. More than kcap kept blocks truncates the row to its first
+ *       kcap indices and records SPARK_ECAPACITY (kcap = nb never overflows).
+ * Outputs: idx int32 [B, H, nb, kcap] (per row, ascending block indices in the first
+ * cnt slots; later slots unspecified), cnt int32 [B, H, nb].
+ * ws: spark_workspace_bytes(s, SPARK_CALL_SELECT) bytes (tau only; may be NULL for top-k). */
+int spark_score_select(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
+                       double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Attention forward ("What Spark-Attn changes": exact + compressed branches merged in
+ * one softmax; sink_conditioning: sink keys attended exactly; "Nodes": dense rows).
+ * A video query of block i attends to the 64 keys of each selected block idx[i, :cnt[i]]
+ * and to every dense key; when pool_pack is not NULL it also attends to one pooled
+ * entry per unselected video block b, with logit q . k_pool[b] * scale + beta[b] and
+ * value v_summ[b] (bf16 operands from pool_pack, beta fp32). Dense query rows attend
+ * to every key and never to pooled entries. A row with nothing to attend to gets
+ * O = 0 and LSE = -inf.
+ * perm (nullable) int32 [B, H, nb*64]: the inputs are in a reblocked order and output
+ * row p of a video query is written to original row perm[p] (dense rows unchanged).
+ * Outputs: O bf16 [B, H, N, d]; lse fp32 [B, H, N] natural-log (nullable).
+ * Block indices outside [0, nb) are skipped and recorded as SPARK_EDEVICE_INDEX. */
+int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                   const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
+                   const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/* Spark-Reblock ("What Spark-Attn changes", Spark-Reblock bullet; "Workflows":
+ * reblock_layout=q_reuse_k). Per (b, h): M = mean over video keys of k k^T;
+ * x_i = L^T q_i / |L^T q_i| with M = L L^T (Mahalanobis cosine geometry); recursive
+ * bisection of the video tokens: a node of m blocks takes the leading eigenvector v of
+ * the centred covariance of its x (signed so the projections' third central moment is
+ * >= 0), orders its tokens by (x . v, token index) and gives the first floor(m/2)*64 to
+ * the left child, until every leaf holds 64 tokens. perm int32 [B, H, nb*64] lists the
+ * leaves by their smallest token index, tokens ascending inside a leaf. Qp/Kp/Vp
+ * (bf16 [B,H,N,d], may not alias the inputs) receive the permuted rows (keys reuse the
+ * query partition), dense rows copied unchanged. tree (nullable) int32
+ * [B, H, L+1, nb*64], L = ceil(log2 nb): node label of every token at every level
+ * (a node c splits into 2c (left) and 2c+1; a leaf moves to 2c).
+ * ws: spark_workspace_bytes(s, SPARK_CALL_REBLOCK) bytes. */
+int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                  int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* Reads the device error word into *host_word (may be NULL) and clears it; synchronises
+ * `stream`. Returns SPARK_OK or SPARK_ECUDA when the copy itself failed. */
+int spark_device_error(int32_t* host_word, void* stream);
+
+/* Human-readable text of a status code. */
+const char* spark_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARK_H_ */

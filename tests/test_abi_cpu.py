@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI (no GPU): the library builds and loads, exports every
+entry point that include/spark.h declares, and rejects bad arguments before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spark.h")
+
+
+@pytest.fixture(scope="module")
+def spark():
+    from block_sparse_video_mean_b200 import build
+    build.build()
+    import block_sparse_video_mean_b200.spark as spark
+    spark.load()
+    return spark
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(spark_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(spark):
+    lib = spark.load()
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(spark.EXPORTS) <= set(names)
+
+
+def test_topk_count_matches_fixture(spark):
+    path = os.path.join(ROOT, "tests", "golden", "topk_count.txt")
+    for ln in open(path):
+        if ln.strip() and not ln.startswith("#"):
+            r, nb, k = ln.split()
+            assert spark.topk_count(float(r), int(nb)) == int(k), ln
+    assert spark.topk_count(0.0, 10) == -1
+    assert spark.topk_count(1.5, 10) == -1
+
+
+def test_num_blocks_and_workspace(spark):
+    s = spark.make_shape(1, 24, 175680 + 512, 128, 512)
+    assert spark.num_blocks(s) == 2745
+    assert spark.workspace_bytes(s, spark.CALL_POOL) == 2 * 24 * 2745 * 128 * 2
+    assert spark.workspace_bytes(s, spark.CALL_ATTN) == 0
+    ragged = spark.make_shape(1, 1, 64 * 3 + 17 + 5, 64, 5)
+    assert spark.num_blocks(ragged) == 3
+    assert spark.num_blocks(spark.make_shape(1, 1, 40, 64, 8)) == 0
+
+
+def test_bad_arguments_are_rejected_on_the_host(spark):
+    lib = spark.load()
+    P = ctypes.c_void_p
+    dummy = P(16)  # never dereferenced: validation fails first
+    bad_d = spark.make_shape(1, 1, 128, 96, 0)
+    assert lib.spark_pool_kv(ctypes.byref(bad_d), dummy, dummy, dummy, 0, dummy, dummy, dummy,
+                             dummy, dummy, dummy, 1 << 20, None) == -2
+    bad_block = spark.Shape(1, 1, 128, 64, 0, 32, 0.0)
+    assert lib.spark_attn_fwd(ctypes.byref(bad_block), dummy, dummy, dummy, dummy, dummy, 1, None,
+                              None, None, dummy, None, None, 0, None) == -2
+    neg = spark.make_shape(1, 1, 128, 64, 200)
+    assert lib.spark_attn_fwd(ctypes.byref(neg), dummy, dummy, dummy, dummy, dummy, 1, None, None,
+                              None, dummy, None, None, 0, None) == -1
+    ok = spark.make_shape(1, 1, 128, 64, 0)
+    # null inputs, misaligned pointers, bad ratio, kcap below k, unknown mode, bad pool mode
+    assert lib.spark_pool_kv(ctypes.byref(ok), None, dummy, dummy, 0, dummy, dummy, dummy, dummy,
+                             dummy, dummy, 1 << 20, None) == -1
+    assert lib.spark_pool_kv(ctypes.byref(ok), P(18), dummy, dummy, 0, dummy, dummy, dummy, dummy,
+                             dummy, dummy, 1 << 20, None) == -1
+    assert lib.spark_pool_kv(ctypes.byref(ok), dummy, dummy, dummy, 7, dummy, dummy, dummy, dummy,
+                             dummy, dummy, 1 << 20, None) == -1
+    assert lib.spark_score_select(ctypes.byref(ok), dummy, dummy, 0, 1.5, 2, dummy, dummy, None, 0,
+                                  None) == -1
+    assert lib.spark_score_select(ctypes.byref(ok), dummy, dummy, 0, 0.5, 0, dummy, dummy, None, 0,
+                                  None) == -1
+    assert lib.spark_score_select(ctypes.byref(ok), dummy, dummy, 5, 0.5, 2, dummy, dummy, None, 0,
+                                  None) == -1
+    assert lib.spark_score_select(ctypes.byref(ok), dummy, dummy, 1, float("nan"), 2, dummy, dummy,
+                                  dummy, 1 << 10, None) == -1
+    # tau needs its workspace
+    assert lib.spark_score_select(ctypes.byref(ok), dummy, dummy, 1, 1.0, 2, dummy, dummy, None, 0,
+                                  None) == -1
+    assert lib.spark_reblock(ctypes.byref(ok), dummy, dummy, dummy, None, dummy, dummy, dummy, None,
+                             dummy, 1 << 30, None) == -1
+
+
+def test_empty_inputs_are_a_no_op(spark):
+    lib = spark.load()
+    empty = spark.make_shape(0, 4, 128, 64, 0)
+    assert lib.spark_attn_fwd(ctypes.byref(empty), None, None, None, None, None, 1, None, None,
+                              None, None, None, None, 0, None) == 0
+    zero_n = spark.make_shape(1, 4, 0, 64, 0)
+    assert lib.spark_pool_kv(ctypes.byref(zero_n), None, None, None, 0, None, None, None, None,
+                             None, None, 0, None) == 0
+
+
+def test_strerror(spark):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert spark.strerror(code) and spark.strerror(code) != "unknown status"

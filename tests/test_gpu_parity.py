@@ -1,0 +1,198 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded
+inputs. Small cases compare every output element; the full-size workloads compare sampled
+heads and query blocks, in the launch configuration the benchmark times."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.spark_oracle as orc
+from block_sparse_video_mean_b200.inputs import make_qkv
+from tests.parity import (check_lse, check_output, check_selection_row, gpu_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def spark():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import block_sparse_video_mean_b200.spark as spark
+    spark.load()
+    return spark
+
+
+DEV = "cuda:0"
+
+
+def run_plan(spark, Q, K, V, ns, cfg):
+    B, H, N, d = Q.shape
+    plan = spark.SparkAttention(B, H, N, d, ns, cfg, DEV)
+    O, L = plan.run(Q.to(DEV), K.to(DEV), V.to(DEV))
+    torch.cuda.synchronize()
+    return plan, O, L
+
+
+def head_f64(Q, K, V, b, h):
+    return tuple(orc.to_f64(t[b, h]) for t in (Q, K, V))
+
+
+def compare_head(plan, O, L, Q, K, V, b, h, ns, cfg, qblocks=None, check_pool=True, dense=True):
+    """Compare one head (all or sampled query blocks) against the oracle."""
+    q, k, v = head_f64(Q, K, V, b, h)
+    scale = cfg.scale or 1.0 / math.sqrt(q.shape[1])
+    P = orc.pool_head(q, k, v, ns, scale, 64, cfg.pool_mode)
+    nb = P.qbar.shape[0]
+    blocks = np.arange(nb) if qblocks is None else np.asarray(qblocks)
+    if check_pool and nb:
+        gp = {n: plan.pool[n][b, h].cpu().double().numpy() for n in ("q_pool", "k_pool", "v_summ", "beta", "anchor")}
+        np.testing.assert_allclose(gp["q_pool"], P.qbar, atol=2e-6, rtol=0)
+        np.testing.assert_allclose(gp["k_pool"], P.kbar, atol=2e-6, rtol=0)
+        np.testing.assert_allclose(gp["anchor"], P.anchor, atol=2e-6, rtol=0)
+        np.testing.assert_allclose(gp["v_summ"], P.vtil, atol=2e-5, rtol=0)
+        np.testing.assert_allclose(gp["beta"], P.beta, atol=2e-5, rtol=0)
+    sel = gpu_rows(plan.idx[b, h].cpu().numpy(), plan.cnt[b, h].cpu().numpy()) if nb else []
+    thr = None
+    if cfg.mode == "tau" and nb:
+        thr = orc.tau_threshold(orc.block_scores(P.qbar, P.kbar, scale), cfg.param)
+    S = orc.block_scores(P.qbar, P.kbar, scale, blocks) if nb else None
+    for t, i in enumerate(blocks):
+        ok, ndiff = check_selection_row(sel[i], S[t], cfg.mode, cfg.param, thr)
+        assert ok, (b, h, i, ndiff)
+    pooled = P if cfg.compressed else None
+    Og = O[b, h].float().cpu().numpy()
+    Lg = L[b, h].cpu().numpy()
+    for i in blocks:
+        o, l = orc.attn_video_block(q, k, v, ns, i, sel[i], pooled, scale)
+        rows = slice(i * 64, (i + 1) * 64)
+        check_output(Og[rows], o, f"head {b},{h} block {i}")
+        check_lse(Lg[rows], l, f"head {b},{h} block {i}")
+    N = q.shape[0]
+    if dense and N > nb * 64:
+        rows = np.arange(nb * 64, N)
+        o, l = orc.attn_dense_rows(q, k, v, rows, scale)
+        check_output(Og[rows], o, f"head {b},{h} dense rows")
+        check_lse(Lg[rows], l, f"head {b},{h} dense rows")
+
+
+# ------------------------------------------------------------------- small, every element
+
+SMALL = [
+    # d, n_video, n_sink, mode, param, compressed, pool_mode
+    (64, 1024, 32, "topk", 0.1, True, "reweight"),       # the tiny 4x16x16 + 32 sink workload
+    (128, 64 * 40, 100, "topk", 0.2, True, "reweight"),
+    (128, 64 * 33 + 17, 64, "topk", 0.1, True, "reweight"),  # ragged video tail
+    (64, 64 * 50, 0, "tau", 1.0, True, "reweight"),          # no sinks
+    (128, 64 * 40, 30, "tau", 1.5, False, "reweight"),
+    (64, 64 * 24, 16, "topk", 0.3, True, "mean"),
+    (128, 64 * 20, 7, "topk", 1.0, False, "reweight"),       # full density: dense attention
+    (64, 40, 24, "topk", 0.1, True, "reweight"),              # no full video block at all
+    (128, 64 * 150, 70, "topk", 0.05, True, "reweight"),     # several pooled tiles, ragged
+]
+
+
+@pytest.mark.parametrize("d,nv,ns,mode,param,compressed,pool_mode", SMALL)
+def test_small_every_element(spark, d, nv, ns, mode, param, compressed, pool_mode):
+    Q, K, V = make_qkv(1, 2, nv, ns, d, seed=0)
+    cfg = spark.ForwardConfig(mode, param, compressed, pool_mode)
+    plan, O, L = run_plan(spark, Q, K, V, ns, cfg)
+    assert spark.device_error() == 0
+    for h in range(2):
+        compare_head(plan, O, L, Q, K, V, 0, h, ns, cfg)
+
+
+def test_empty_rows_give_zero_and_neg_inf(spark):
+    Q, K, V = make_qkv(1, 1, 64 * 16, 0, 64, seed=1)
+    cfg = spark.ForwardConfig("tau", 50.0, False)
+    plan, O, L = run_plan(spark, Q, K, V, 0, cfg)
+    assert int(plan.cnt.sum()) == 0
+    assert torch.all(O == 0) and torch.all(torch.isneginf(L))
+
+
+def test_batch_and_heads_are_independent(spark):
+    Q, K, V = make_qkv(2, 3, 64 * 12, 9, 64, seed=4)
+    cfg = spark.ForwardConfig("topk", 0.25, True)
+    plan, O, L = run_plan(spark, Q, K, V, 9, cfg)
+    for b in range(2):
+        for h in range(3):
+            compare_head(plan, O, L, Q, K, V, b, h, 9, cfg)
+
+
+def test_repeat_calls_are_bitwise_stable(spark):
+    Q, K, V = make_qkv(1, 2, 64 * 30, 20, 128, seed=2)
+    cfg = spark.ForwardConfig("topk", 0.1, True)
+    plan, O, L = run_plan(spark, Q, K, V, 20, cfg)
+    O1, L1, idx1 = O.clone(), L.clone(), plan.idx.clone()
+    plan.run(Q.to(DEV), K.to(DEV), V.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(O1, plan.O) and torch.equal(L1, plan.lse) and torch.equal(idx1, plan.idx)
+
+
+# ------------------------------------------------------------------- device-side faults
+
+def test_out_of_range_index_is_skipped_and_reported(spark):
+    Q, K, V = make_qkv(1, 1, 64 * 8, 8, 64, seed=3)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    pool = spark.pool_kv(Qd, Kd, Vd, 8)
+    idx, cnt = spark.score_select(pool["q_pool"], pool["k_pool"], 8, Qd.shape[2], spark.SELECT_TOPK_RATIO, 0.25)
+    idx[0, 0, 3, 0] = 1000
+    spark.attn_fwd(Qd, Kd, Vd, idx, cnt, 8, pool["pack"], pool["beta"])
+    assert spark.device_error() == -5
+    assert spark.device_error() == 0          # the word is cleared by the read
+
+
+def test_tau_overflow_truncates_and_reports(spark):
+    Q, K, V = make_qkv(1, 1, 64 * 32, 0, 64, seed=5)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    pool = spark.pool_kv(Qd, Kd, Vd, 0)
+    idx, cnt = spark.score_select(pool["q_pool"], pool["k_pool"], 0, Qd.shape[2], spark.SELECT_TAU, -1.0, kcap=2)
+    assert spark.device_error() == -6
+    assert int(cnt.max()) <= 2
+
+
+# ------------------------------------------------------------------- full-size workloads
+
+def sample_blocks(nb, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, nb - 1], rng.choice(nb, n, replace=False)]))
+
+
+FULL = {
+    "32k": (1, 24, 32768, 512, 128),
+    "1152x640x243": (1, 24, 175680, 512, 128),
+}
+
+
+def full_inputs(name, seed=0):
+    B, H, nv, ns, d = FULL[name]
+    return make_qkv(B, H, nv, ns, d, seed=seed, device=DEV), ns
+
+
+@pytest.mark.parametrize("name,mode,param,compressed", [
+    ("32k", "topk", 0.1, False),
+    ("1152x640x243", "topk", 0.1, True),
+    ("1152x640x243", "topk", 0.2, True),
+    ("1152x640x243", "topk", 0.3, True),
+    ("1152x640x243", "tau", 1.0, True),
+    ("1152x640x243", "tau", 1.5, True),
+    ("1152x640x243", "tau", 2.0, True),
+    ("1152x640x243", "topk", 1.0, False),
+])
+def test_full_size_sampled(spark, name, mode, param, compressed):
+    (Q, K, V), ns = full_inputs(name)
+    B, H, N, d = Q.shape
+    cfg = spark.ForwardConfig(mode, param, compressed)
+    plan = spark.SparkAttention(B, H, N, d, ns, cfg, DEV)
+    O, L = plan.run(Q, K, V)
+    torch.cuda.synchronize()
+    assert spark.device_error() == 0
+    nb = plan.nb
+    if mode == "tau":
+        frac = plan.cnt.double().sum().item() / (B * H * nb * nb)
+        tail = {1.0: 0.15866, 1.5: 0.06681, 2.0: 0.02275}[param]
+        assert abs(frac - tail) < 0.01, (frac, tail)
+    Qc, Kc, Vc = Q.cpu(), K.cpu(), V.cpu()
+    for h in (0, H - 1):
+        compare_head(plan, O, L, Qc, Kc, Vc, 0, h, ns, cfg, qblocks=sample_blocks(nb, 6, h),
+                     check_pool=(h == 0), dense=(mode == "topk" and param == 0.1))
