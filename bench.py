@@ -243,7 +243,7 @@ def run_gpu(args, rank, world, local_rank):
                    "l2": "inputs 3.2 GB > 126 MB L2; no flush needed"},
         "selected_tflops": round(fl["selected"] / (ms_step * 1e-3) / 1e12, 2),
         "attn_kernel_ms": round(attn_ms, 3),
-        "roofline": {"bound": "tensor", "kernel": "attn_mma_kernel<128>",
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>",
                      "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / bf16_peak, 4),
                      "peak_source": f"{peak_src} bf16 burst (sustained {bf16_sust})",

@@ -1,6 +1,8 @@
 // libspark: the C ABI of include/spark.h. Host-side argument validation and launches;
 // every step of the computation runs in the kernels included below. The whole library
 // is this one translation unit.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -9,6 +11,7 @@
 #include "pool.cuh"
 #include "select.cuh"
 #include "attn_mma.cuh"
+#include "attn_tc.cuh"
 #include "reblock.cuh"
 
 using namespace spark;
@@ -56,6 +59,69 @@ int select_rows_per_cta(int nb, int d, size_t* smem) {
     }
   }
   return 0;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over `rows` x d, 64 x 64 boxes, 128-byte swizzle (rows of 64 elements).
+bool bf16_tile_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+template <int D>
+int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, const void* pack,
+                   cudaStream_t cs) {
+  using C = TcCfg<D>;
+  TcMaps maps;
+  const uint64_t rows = (uint64_t)tp.BH * tp.N;
+  if (!bf16_tile_map(&maps.k, K, rows, D) || !bf16_tile_map(&maps.v, V, rows, D)) return SPARK_ECUDA;
+  if (pack != nullptr) {
+    const uint16_t* kp = static_cast<const uint16_t*>(pack);
+    const uint16_t* vp = kp + (size_t)tp.BH * tp.nb * D;
+    const uint64_t prow = (uint64_t)tp.BH * tp.nb;
+    if (!bf16_tile_map(&maps.kp, kp, prow, D) || !bf16_tile_map(&maps.vp, vp, prow, D)) return SPARK_ECUDA;
+  } else {
+    maps.kp = maps.k;
+    maps.vp = maps.v;
+  }
+  const size_t smem = 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes +
+                      8 * (size_t)((tp.nb + 31) / 32) * 4;  // one bitmap per softmax warp
+  if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
+  const int sms = num_sms();
+  if (sms <= 0) return SPARK_ECUDA;
+  const int grid = (int)std::min<int64_t>(sms, ((int64_t)tp.n_items + 1) / 2);
+  if (cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return SPARK_ECUDA;
+  attn_tc_kernel<D><<<grid, C::kThreads, smem, cs>>>(maps, tp);
+  SPARK_LAUNCH_CHECK();
+  return SPARK_OK;
 }
 
 }  // namespace
@@ -221,39 +287,26 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   const int n_dq = (s->N - nv + kBlock - 1) / kBlock;
   const int64_t items = (int64_t)bh * (n_dq + nb);
   if (items > 0x7fffffff) return SPARK_EUNSUPPORTED;
-  AttnParams ap;
-  ap.Q = Q;
-  ap.K = K;
-  ap.V = V;
-  ap.idx = idx;
-  ap.cnt = cnt;
-  ap.kp16 = nb > 0 ? static_cast<const uint16_t*>(pool_pack) : nullptr;
-  ap.vp16 = ap.kp16 ? ap.kp16 + (size_t)bh * nb * s->d : nullptr;
-  ap.beta = beta;
-  ap.perm = perm;
-  ap.O = O;
-  ap.lse = lse;
-  ap.N = s->N;
-  ap.nb = nb;
-  ap.kcap = kcap;
-  ap.BH = bh;
-  ap.n_dq = n_dq;
-  ap.scale_log2 = eff_scale(s) * kLog2e;
+  if ((int64_t)bh * s->N >= ((int64_t)1 << 31)) return SPARK_EUNSUPPORTED;  // TMA row coordinates
+  TcParams tp;
+  tp.Q = Q;
+  tp.idx = idx;
+  tp.cnt = cnt;
+  tp.beta = beta;
+  tp.perm = perm;
+  tp.O = O;
+  tp.lse = lse;
+  tp.N = s->N;
+  tp.nb = nb;
+  tp.kcap = kcap;
+  tp.BH = bh;
+  tp.n_dq = n_dq;
+  tp.pooled = (nb > 0 && pool_pack != nullptr) ? 1 : 0;
+  tp.n_items = (int)items;
+  tp.scale_log2 = eff_scale(s) * kLog2e;
   cudaStream_t cs = as_stream(stream);
-  const size_t bitmap = (size_t)((nb + 31) / 32) * 4;
-  if (s->d == 128) {
-    const size_t smem = MmaAttn<128>::kSmemFixed + bitmap;
-    if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
-    cudaFuncSetAttribute(attn_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_mma_kernel<128><<<(unsigned)items, 128, smem, cs>>>(ap);
-  } else {
-    const size_t smem = MmaAttn<64>::kSmemFixed + bitmap;
-    if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
-    cudaFuncSetAttribute(attn_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attn_mma_kernel<64><<<(unsigned)items, 128, smem, cs>>>(ap);
-  }
-  SPARK_LAUNCH_CHECK();
-  return SPARK_OK;
+  const void* pack = tp.pooled ? pool_pack : nullptr;
+  return s->d == 128 ? launch_attn_tc<128>(tp, K, V, pack, cs) : launch_attn_tc<64>(tp, K, V, pack, cs);
 }
 
 int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
