@@ -19,17 +19,28 @@
 //   (slot 0: lanes 0-15, slot 1: lanes 16-31 of each 32-lane group), so the tensor core
 //   works on one slot while the other slot's softmax runs.
 // * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1 (warp w reads
-//   TMEM sub-partition w % 4), warp 8 issues TMA loads, warp 9 issues MMAs and owns TMEM.
-// * Per 64-key tile: S = Q K^T (8 MMAs 64x64x16 from TMEM Q and a 128B-swizzled K tile),
-//   softmax in base 2 with a lazy running max (O is rescaled only when the row max grows
-//   by more than 2^8), P written back over S as bf16, then O += P V (4 MMAs 64xDx16 with
-//   V as an MN-major operand). Tile order per video query block: selected blocks, dense
-//   key rows, then pooled entries (beta added, selected blocks masked).
+//   TMEM sub-partition w % 4), warp 8 fills the K ring and warp 10 the V ring with TMA,
+//   warp 9 issues MMAs and owns TMEM. K stages are released when their S MMAs complete and
+//   V stages when their PV MMAs complete, so neither producer waits on an MMA that the
+//   issuer can only start later.
+// * A tile is 128 keys made of two 64-key halves (a selected block, 64 dense rows or 64
+//   pooled entries each; per video query block the halves run selected blocks, dense key
+//   rows, then pooled entries). Per tile: S = Q K^T (8 MMAs 64x128x16 from TMEM Q and a
+//   128B-swizzled K tile), softmax in base 2 (each thread owns one half of one row) with a
+//   lazy running max (O is rescaled only when the row max grows by more than 2^8), P
+//   written back over S as bf16, then O += P V (8 MMAs 64xDx16, V as an MN-major operand).
 // * Every mbarrier wait is bounded; a timeout records SPARK_ETIMEOUT, raises the CTA abort
 //   flag, the TMA role drains its copies in flight and TMEM is released.
 #pragma once
 #include "spark_common.cuh"
 #include "tc_util.cuh"
+
+// Timing hooks for out-of-tree instrumented builds; no-ops here.
+#ifndef SPARK_TC_T0
+#define SPARK_TC_T0(v)
+#define SPARK_TC_ACC(slot, v)
+#define SPARK_TC_EV(who, what)
+#endif
 
 namespace spark {
 
@@ -51,23 +62,25 @@ struct TcParams {
 
 template <int D>
 struct TcCfg {
-  static constexpr int kStages = 6;
-  static constexpr int kPanels = D / 64;         // 128-byte swizzle panels per row
-  static constexpr int kPanelBytes = 64 * 128;   // 64 rows x 128 B
-  static constexpr int kTileBytes = 64 * D * 2;  // one K or V tile (64 keys)
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kColS = 0;                // S/P buffers at 0 and 64
-  static constexpr int kColO = 128;
-  static constexpr int kColQ = 128 + D;
-  static constexpr int kTmemCols = (kColQ + D / 2 <= 256) ? 256 : 512;
-  static constexpr int kThreads = 320;
-  static constexpr int kRingBytes = kStages * kStageBytes;
+  // A tile is 128 keys: two 64-key halves (each a selected block, 64 dense rows or 64
+  // pooled entries), so S = Q K^T is one N = 128 MMA per K step.
+  static constexpr int kStages = D == 128 ? 3 : 6;
+  static constexpr int kPanels = D / 64;           // 128-byte swizzle panels per row
+  static constexpr int kHalfBytes = 64 * 128;      // 64 rows x 128 B (one TMA box)
+  static constexpr int kPanelBytes = 128 * 128;    // 128 rows x 128 B
+  static constexpr int kTileBytes = 128 * D * 2;   // K (or V) of one 128-key tile
+  static constexpr int kColS = 0;                  // S/P buffers at 0 and 128
+  static constexpr int kColO = 256;
+  static constexpr int kColQ = 256 + D;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kThreads = 352;
+  static constexpr int kRingBytes = 2 * kStages * kTileBytes;  // K ring, then V ring
   static constexpr int kBarBytes = 1024;
 };
 
 struct TcItem {
-  int bh, q0, nq, dense, cnt, ntiles;
-  size_t row;  // selection row (video items)
+  int bh, q0, nq, dense, cnt, nhalf, ntiles;  // nhalf 64-key halves, ntiles = ceil(nhalf / 2)
+  size_t row;                                  // selection row (video items)
 };
 
 __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
@@ -81,7 +94,7 @@ __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
     r.q0 = nv + (it % p.n_dq) * kBlock;
     r.cnt = 0;
     r.row = 0;
-    r.ntiles = (p.N + kBlock - 1) / kBlock;
+    r.nhalf = (p.N + kBlock - 1) / kBlock;
   } else {
     const int v = it - nd;
     r.bh = v / p.nb;
@@ -91,26 +104,11 @@ __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
     int c = p.cnt[r.row];
     c = c < 0 ? 0 : (c > p.kcap ? p.kcap : c);
     r.cnt = c;
-    r.ntiles = c + n_dk + (p.pooled ? (p.nb + kBlock - 1) / kBlock : 0);
+    r.nhalf = c + n_dk + (p.pooled ? (p.nb + kBlock - 1) / kBlock : 0);
   }
+  r.ntiles = (r.nhalf + 1) / 2;
   r.nq = min(kBlock, p.N - r.q0);
   return r;
-}
-
-// Row coordinate of tile t in the K/V (or pooled pack) tensor map.
-__device__ __forceinline__ int tc_tile_row(const TcParams& p, const TcItem& I, int t, int* pooled) {
-  const int nv = p.nb * kBlock;
-  const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
-  *pooled = 0;
-  if (I.dense) return I.bh * p.N + t * kBlock;
-  if (t < I.cnt) {
-    int b = p.idx[I.row * (size_t)p.kcap + t];
-    if (b < 0 || b >= p.nb) b = 0;  // masked by the softmax, reported there
-    return I.bh * p.N + b * kBlock;
-  }
-  if (t < I.cnt + n_dk) return I.bh * p.N + nv + (t - I.cnt) * kBlock;
-  *pooled = 1;
-  return I.bh * p.nb + (t - I.cnt - n_dk) * kBlock;
 }
 
 // Slot s of CTA c walks items 2c + s, 2c + s + 2G, ... and skips items without tiles.
@@ -141,7 +139,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 
 template <int D>
 __device__ __forceinline__ uint64_t tc_kdesc(uint32_t stage_addr, int kk) {
-  // K tile: K-major, 128B swizzle; k-step kk covers d = 16kk .. 16kk+15
+  // K tile (128 rows): K-major, 128B swizzle; k-step kk covers d = 16kk .. 16kk+15
   return tc::make_sdesc(stage_addr + (kk >> 2) * TcCfg<D>::kPanelBytes + (kk & 3) * 32, 16, 1024,
                         tc::kSwizzle128);
 }
@@ -149,27 +147,29 @@ template <int D>
 __device__ __forceinline__ uint64_t tc_vdesc(uint32_t stage_addr, int kk) {
   // V tile as an MN-major operand (N = d): k-step kk covers keys 16kk .. 16kk+15 (two 8-row
   // atoms of 1 KB); the d panels are kPanelBytes apart.
-  return tc::make_sdesc(stage_addr + TcCfg<D>::kTileBytes + kk * 2048, TcCfg<D>::kPanelBytes, 1024,
-                        tc::kSwizzle128);
+  return tc::make_sdesc(stage_addr + kk * 2048, TcCfg<D>::kPanelBytes, 1024, tc::kSwizzle128);
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     attn_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
   using C = TcCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* ring = smem;
+  unsigned char* vring = ring + C::kStages * C::kTileBytes;
   uint64_t* kfull = reinterpret_cast<uint64_t*>(ring + C::kRingBytes);
   uint64_t* vfull = kfull + C::kStages;
-  uint64_t* kvempty = vfull + C::kStages;
-  uint64_t* sfull = kvempty + C::kStages;  // [slot][buf]
+  uint64_t* kempty = vfull + C::kStages;   // K stage free: its S MMAs completed
+  uint64_t* vempty = kempty + C::kStages;  // V stage free: its PV MMAs completed
+  uint64_t* sfull = vempty + C::kStages;   // [slot][buf]
   uint64_t* pfull = sfull + 4;             // [slot][buf]
   uint64_t* oready = pfull + 4;            // [slot]
   uint64_t* qfull = oready + 2;            // [slot]
   uint64_t* ofree = qfull + 2;             // [slot]
-  uint64_t* finbar = ofree + 2;            // all MMAs of the CTA done
+  uint64_t* odone = ofree + 2;             // [slot]: last PV of an item completed
+  uint64_t* finbar = odone + 2;            // all MMAs of the CTA done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
@@ -180,7 +180,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < C::kStages; ++i) {
       tc::mbar_init(&kfull[i], 1);
       tc::mbar_init(&vfull[i], 1);
-      tc::mbar_init(&kvempty[i], 1);
+      tc::mbar_init(&kempty[i], 1);
+      tc::mbar_init(&vempty[i], 1);
     }
     for (int i = 0; i < 4; ++i) {
       tc::mbar_init(&sfull[i], 1);
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(320, 1)
       tc::mbar_init(&oready[i], 1);
       tc::mbar_init(&qfull[i], 4);
       tc::mbar_init(&ofree[i], 4);
+      tc::mbar_init(&odone[i], 1);
     }
     tc::mbar_init(finbar, 1);
     *abort_flag = 0;
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(320, 1)
     tc::tmem_alloc(tmem_holder, C::kTmemCols);
     tc::tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if ((warp == 8 || warp == 10) && lane == 0) {
     tc::tma_prefetch_desc(&maps.k);
     tc::tma_prefetch_desc(&maps.v);
     tc::tma_prefetch_desc(&maps.kp);
@@ -211,59 +213,102 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tbase = *tmem_holder;
   const int stride = 2 * gridDim.x;
 
-  if (warp == 8) {
-    // ================================================================ TMA producer
-    if (lane == 0) {
-      TcSlotWalk walk[2] = {{2 * (int)blockIdx.x, stride, p.n_items},
-                            {2 * (int)blockIdx.x + 1, stride, p.n_items}};
-      TcItem cur[2];
-      bool have[2];
-      int t[2] = {0, 0};
-      for (int s = 0; s < 2; ++s) have[s] = walk[s].next_nonempty(p, &cur[s]);
-      uint32_t q = 0;
-      bool ok = true;
-      while (ok && (have[0] || have[1])) {
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (!have[s]) continue;
-          const int stage = q % C::kStages;
-          if (q >= (uint32_t)C::kStages &&
-              !tc::mbar_wait(&kvempty[stage], ((q / C::kStages) - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          int pooled;
-          const int y = tc_tile_row(p, cur[s], t[s], &pooled);
-          const CUtensorMap* mk = pooled ? &maps.kp : &maps.k;
-          const CUtensorMap* mv = pooled ? &maps.vp : &maps.v;
-          unsigned char* st = ring + stage * C::kStageBytes;
-          tc::mbar_expect_tx(&kfull[stage], C::kTileBytes);
+  if (warp == 8 || warp == 10) {
+    // ================================================================ TMA producers
+    // warp 8 fills the K ring, warp 10 the V ring, both in the same tile order.
+    const bool is_v = warp == 10;
+    uint64_t* full = is_v ? vfull : kfull;
+    uint64_t* empty = is_v ? vempty : kempty;
+    unsigned char* rbase = is_v ? vring : ring;
+    const CUtensorMap* map_x = is_v ? &maps.v : &maps.k;
+    const CUtensorMap* map_p = is_v ? &maps.vp : &maps.kp;
+    // The whole warp walks the tile sequence; the selected block indices are fetched 32
+    // halves at a time, one chunk ahead, so no global load sits on the issue path.
+    TcSlotWalk walk[2] = {{2 * (int)blockIdx.x, stride, p.n_items},
+                          {2 * (int)blockIdx.x + 1, stride, p.n_items}};
+    TcItem cur[2];
+    bool have[2];
+    int t[2] = {0, 0};
+    int ic[2] = {0, 0}, in[2] = {0, 0};  // idx of halves 32c + lane (current / next chunk)
+    auto chunk = [&](int s, int c) -> int {
+      const int hh = 32 * c + lane;
+      return hh < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + hh] : 0;
+    };
+    for (int s = 0; s < 2; ++s) {
+      have[s] = walk[s].next_nonempty(p, &cur[s]);
+      if (have[s] && !cur[s].dense) {
+        ic[s] = chunk(s, 0);
+        in[s] = chunk(s, 1);
+      }
+    }
+    const int nv = p.nb * kBlock;
+    const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
+    uint32_t q = 0;
+    bool ok = true;
+    while (ok && (have[0] || have[1])) {
+      for (int s = 0; s < 2 && ok; ++s) {
+        if (!have[s]) continue;
+        const int stage = q % C::kStages;
+        SPARK_TC_T0(t_ew);
+        if (q >= (uint32_t)C::kStages &&
+            !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        SPARK_TC_ACC(4, t_ew);
+        const TcItem& I = cur[s];
+        int y[2], pooled[2];
 #pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tc::tma_load_2d(st + pn * C::kPanelBytes, mk, pn * 64, y, &kfull[stage]);
-          tc::mbar_expect_tx(&vfull[stage], C::kTileBytes);
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tc::tma_load_2d(st + C::kTileBytes + pn * C::kPanelBytes, mv, pn * 64, y, &vfull[stage]);
-          ++q;
-          if (++t[s] == cur[s].ntiles) {
-            t[s] = 0;
-            have[s] = walk[s].next_nonempty(p, &cur[s]);
+        for (int hf = 0; hf < 2; ++hf) {
+          int hi = 2 * t[s] + hf;
+          if (hi >= I.nhalf) hi = 2 * t[s];  // a missing second half repeats the first (masked)
+          const int bsel = __shfl_sync(0xffffffffu, ic[s], hi & 31);
+          pooled[hf] = 0;
+          if (I.dense) {
+            y[hf] = I.bh * p.N + hi * kBlock;
+          } else if (hi < I.cnt) {
+            y[hf] = I.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
+          } else if (hi < I.cnt + n_dk) {
+            y[hf] = I.bh * p.N + nv + (hi - I.cnt) * kBlock;
+          } else {
+            pooled[hf] = 1;
+            y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk) * kBlock;
           }
         }
-      }
-      if (!ok || *abort_flag) {
-        // drain every copy that may still be in flight before the CTA leaves
-        const uint32_t first = q > (uint32_t)C::kStages ? q - C::kStages : 0;
-        for (uint32_t j = first; j < q; ++j) {
-          mbar_drain(&kfull[j % C::kStages], (j / C::kStages) & 1);
-          mbar_drain(&vfull[j % C::kStages], (j / C::kStages) & 1);
+        if (lane == 0) {
+          unsigned char* st = rbase + stage * C::kTileBytes;
+          tc::mbar_expect_tx(&full[stage], C::kTileBytes);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int pn = 0; pn < C::kPanels; ++pn)
+              tc::tma_load_2d(st + pn * C::kPanelBytes + hf * C::kHalfBytes,
+                              pooled[hf] ? map_p : map_x, pn * 64, y[hf], &full[stage]);
+        }
+        __syncwarp();
+        ++q;
+        if (++t[s] == cur[s].ntiles) {
+          t[s] = 0;
+          have[s] = walk[s].next_nonempty(p, &cur[s]);
+          if (have[s] && !cur[s].dense) {
+            ic[s] = chunk(s, 0);
+            in[s] = chunk(s, 1);
+          }
+        } else if ((t[s] & 15) == 0 && !cur[s].dense && 2 * t[s] < cur[s].cnt) {
+          ic[s] = in[s];
+          in[s] = chunk(s, (t[s] >> 4) + 1);
         }
       }
+    }
+    if ((!ok || *abort_flag) && lane == 0) {
+      // drain every copy that may still be in flight before the CTA leaves
+      const uint32_t first = q > (uint32_t)C::kStages ? q - C::kStages : 0;
+      for (uint32_t j = first; j < q; ++j) mbar_drain(&full[j % C::kStages], (j / C::kStages) & 1);
     }
   } else if (warp == 9) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = tc::make_idesc_bf16(64, 64, 0, 0);
+      constexpr uint32_t idS = tc::make_idesc_bf16(64, 128, 0, 0);
       constexpr uint32_t idPV = tc::make_idesc_bf16(64, D, 0, 1);
       TcSlotWalk walk[2] = {{2 * (int)blockIdx.x, stride, p.n_items},
                             {2 * (int)blockIdx.x + 1, stride, p.n_items}};
@@ -275,78 +320,110 @@ __global__ void __launch_bounds__(320, 1)
       struct Pend {
         int valid;
         uint32_t q, g, item;
-        int first;
-      } pend[2] = {{0, 0, 0, 0, 0}, {0, 0, 0, 0, 0}};
+        int first, last;
+      } pend[2] = {{0, 0, 0, 0, 0, 0}, {0, 0, 0, 0, 0, 0}};
       for (int s = 0; s < 2; ++s) have[s] = walk[s].next_nonempty(p, &cur[s]);
       const uint32_t ring_addr = tc::smem_addr(ring);
+      const uint32_t vring_addr = tc::smem_addr(vring);
       bool ok = true;
       auto issue_pv = [&](int s, const Pend& pe) -> bool {
         const uint32_t b = pe.g & 1;
+        SPARK_TC_T0(t_pw);
         if (!tc::mbar_wait(&pfull[2 * s + b], (pe.g >> 1) & 1, abort_flag)) return false;
+        SPARK_TC_ACC(0, t_pw);
+        SPARK_TC_EV(0, 30 + s);
         const int stage = pe.q % C::kStages;
+        SPARK_TC_T0(t_vw);
         if (!tc::mbar_wait(&vfull[stage], (pe.q / C::kStages) & 1, abort_flag)) return false;
+        SPARK_TC_ACC(1, t_vw);
+        SPARK_TC_T0(t_ow);
         if (pe.first && pe.item > 0 && !tc::mbar_wait(&ofree[s], (pe.item - 1) & 1, abort_flag))
           return false;
+        SPARK_TC_ACC(9, t_ow);
+        SPARK_TC_T0(t_pv);
         tc::tc_fence_after();
         const uint32_t lanes = (uint32_t)(16 * s) << 16;
-        const uint32_t st = ring_addr + stage * C::kStageBytes;
+        const uint32_t st = vring_addr + stage * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc::mma_ts(tbase + lanes + C::kColO, tbase + lanes + C::kColS + 64 * b + kk * 8,
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_ts(tbase + lanes + C::kColO, tbase + lanes + C::kColS + 128 * b + kk * 8,
                      tc_vdesc<D>(st, kk), idPV, (pe.first && kk == 0) ? 0u : 1u);
-        tc::mma_commit(&kvempty[stage]);
+        tc::mma_commit(&vempty[stage]);
         tc::mma_commit(&oready[s]);
+        if (pe.last) tc::mma_commit(&odone[s]);
+        SPARK_TC_EV(0, 20 + s);
+        SPARK_TC_ACC(10, t_pv);
         return true;
       };
       uint32_t q = 0;
+      SPARK_TC_T0(t_all);
       while (ok && (have[0] || have[1])) {
+        // S of both slots first, so the tensor core has work while a softmax finishes
+        Pend nxt[2] = {{0, 0, 0, 0, 0, 0}, {0, 0, 0, 0, 0, 0}};
         for (int s = 0; s < 2 && ok; ++s) {
           if (!have[s]) continue;
+          SPARK_TC_T0(t_qw);
           if (t[s] == 0 && !tc::mbar_wait(&qfull[s], nitem[s] & 1, abort_flag)) {
             ok = false;
             break;
           }
+          SPARK_TC_ACC(3, t_qw);
           const int stage = q % C::kStages;
+          SPARK_TC_T0(t_kw);
           if (!tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
+          SPARK_TC_ACC(2, t_kw);
+          SPARK_TC_T0(t_si);
           tc::tc_fence_after();
           const uint32_t b = g[s] & 1;
           const uint32_t lanes = (uint32_t)(16 * s) << 16;
-          const uint32_t st = ring_addr + stage * C::kStageBytes;
+          const uint32_t st = ring_addr + stage * C::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_ts(tbase + lanes + C::kColS + 64 * b, tbase + lanes + C::kColQ + kk * 8,
+            tc::mma_ts(tbase + lanes + C::kColS + 128 * b, tbase + lanes + C::kColQ + kk * 8,
                        tc_kdesc<D>(st, kk), idS, kk > 0 ? 1u : 0u);
           tc::mma_commit(&sfull[2 * s + b]);
-          if (pend[s].valid && !issue_pv(s, pend[s])) {
-            ok = false;
-            break;
-          }
-          pend[s].valid = 1;
-          pend[s].q = q;
-          pend[s].g = g[s];
-          pend[s].item = nitem[s];
-          pend[s].first = (t[s] == 0);
+          tc::mma_commit(&kempty[stage]);
+          SPARK_TC_EV(0, 10 + s);
+          SPARK_TC_ACC(11, t_si);
+          nxt[s].valid = 1;
+          nxt[s].q = q;
+          nxt[s].g = g[s];
+          nxt[s].item = nitem[s];
+          nxt[s].first = (t[s] == 0);
+          nxt[s].last = (t[s] + 1 == cur[s].ntiles);
           ++q;
           ++g[s];
           if (++t[s] == cur[s].ntiles) {
             t[s] = 0;
             ++nitem[s];
+            SPARK_TC_T0(t_nx);
             have[s] = walk[s].next_nonempty(p, &cur[s]);
-            if (!have[s]) {  // this slot is done: release its last tile now
-              if (!issue_pv(s, pend[s])) {
-                ok = false;
-                break;
-              }
-              pend[s].valid = 0;
+            SPARK_TC_ACC(12, t_nx);
+          }
+        }
+        // then the PV of each slot's previous tile; a slot that just ran out also
+        // releases its last tile
+        for (int s = 0; s < 2 && ok; ++s) {
+          if (pend[s].valid && !issue_pv(s, pend[s])) {
+            ok = false;
+            break;
+          }
+          pend[s] = nxt[s];
+          if (pend[s].valid && !have[s]) {
+            if (!issue_pv(s, pend[s])) {
+              ok = false;
+              break;
             }
+            pend[s].valid = 0;
           }
         }
       }
       for (int s = 0; s < 2 && ok; ++s)
         if (pend[s].valid && !issue_pv(s, pend[s])) ok = false;
+      SPARK_TC_ACC(13, t_all);
       // every MMA of this CTA must be complete before TMEM is released
       tc::mma_commit(finbar);
       mbar_drain(finbar, 0);
@@ -368,16 +445,15 @@ __global__ void __launch_bounds__(320, 1)
     TcItem prev;
     prev.ntiles = 0;
     float m_prev = -INFINITY, l_prev = 0.f;
-    uint32_t g_prev_last = 0;
     uint32_t nitem = 0;
     int cur_bad = 0;
 
-    auto epilogue = [&](const TcItem& I, float m_run, float l_run, uint32_t g_last) -> bool {
-      // oready completes once per PV. Two PVs may still be outstanding here, and a parity
-      // wait only tells phases apart within one phase of the barrier, so step through
-      // PV(g_last - 1) before PV(g_last).
-      if (g_last > 0 && !tc::mbar_wait(&oready[s], (g_last - 1) & 1, abort_flag)) return false;
-      if (!tc::mbar_wait(&oready[s], g_last & 1, abort_flag)) return false;
+    uint32_t ndone = 0;  // non-empty items whose epilogue ran
+    auto epilogue = [&](const TcItem& I, float m_run, float l_run) -> bool {
+      // odone completes once per item, after its last PV; it cannot run an item ahead
+      // because the next item's PVs need this slot's P tiles.
+      if (!tc::mbar_wait(&odone[s], ndone & 1, abort_flag)) return false;
+      ++ndone;
       tc::tc_fence_after();
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
@@ -492,7 +568,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       // ---- finish the previous item (its last PV was issued after this item's first S)
       if (have_prev) {
-        if (!epilogue(prev, m_prev, l_prev, g_prev_last)) {
+        if (!epilogue(prev, m_prev, l_prev)) {
           ok = false;
           break;
         }
@@ -505,54 +581,73 @@ __global__ void __launch_bounds__(320, 1)
       float m_run = -INFINITY, l_run = 0.f;
       for (int t = 0; t < I.ntiles; ++t, ++g) {
         const uint32_t b = g & 1;
+        SPARK_TC_T0(t_sw);
         if (!tc::mbar_wait(&sfull[2 * s + b], (g >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
+        SPARK_TC_ACC(5, t_sw);
+        SPARK_TC_EV(1 + s, 40);
         tc::tc_fence_after();
-        uint32_t sv[32];
-        tc::tmem_ld_16x32bx2_x16<32>(tbase + lanes + C::kColS + 64 * b, sv);
-        tc::tmem_ld_16x32bx2_x16<32>(tbase + lanes + C::kColS + 64 * b + 16, sv + 16);
+        // this thread's 64 keys: half h of the tile (columns 64h .. 64h+63 of the S buffer)
+        float x[64];
+        SPARK_TC_T0(t_ld);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tc::tmem_ld_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * c,
+                                       reinterpret_cast<uint32_t*>(x) + 16 * c);
         tc::tmem_wait_ld();
-        // ---- logits (base 2) and masks
-        float x[32];
+        SPARK_TC_ACC(6, t_ld);
+        SPARK_TC_T0(t_cp);
+        // ---- logits (base 2) and masks of this half
+        const int hi = 2 * t + h;
         int kind = 0, valid = kBlock, j0 = 0;
-        if (I.dense) {
-          valid = min(kBlock, p.N - t * kBlock);
-        } else if (t < I.cnt) {
+        if (hi >= I.nhalf) {
+          valid = 0;
+        } else if (I.dense) {
+          valid = min(kBlock, p.N - hi * kBlock);
+        } else if (hi < I.cnt) {
           if (bad_idx) {
-            const int bb = p.idx[I.row * (size_t)p.kcap + t];
+            const int bb = p.idx[I.row * (size_t)p.kcap + hi];
             if (bb < 0 || bb >= p.nb) valid = 0;
           }
-        } else if (t < I.cnt + n_dk) {
-          valid = min(kBlock, p.N - (nv + (t - I.cnt) * kBlock));
+        } else if (hi < I.cnt + n_dk) {
+          valid = min(kBlock, p.N - (nv + (hi - I.cnt) * kBlock));
         } else {
           kind = 1;
-          j0 = (t - I.cnt - n_dk) * kBlock;
+          j0 = (hi - I.cnt - n_dk) * kBlock;
           valid = min(kBlock, p.nb - j0);
         }
-        const int kb0 = 32 * h;  // first key of this thread's half
         if (kind == 0) {
           if (valid >= kBlock) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sv[j]) * p.scale_log2;
+            for (int j = 0; j < 64; ++j) x[j] *= p.scale_log2;
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              x[j] = (kb0 + j < valid) ? __uint_as_float(sv[j]) * p.scale_log2 : -INFINITY;
+            for (int j = 0; j < 64; ++j) x[j] = (j < valid) ? x[j] * p.scale_log2 : -INFINITY;
           }
         } else {
           const float* bp = p.beta + (size_t)I.bh * p.nb;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int jj = min(j0 + kb0 + j, p.nb - 1);
-            const bool m = (kb0 + j >= valid) || ((bm[jj >> 5] >> (jj & 31)) & 1u);
-            x[j] = m ? -INFINITY : fmaf(__uint_as_float(sv[j]), p.scale_log2, bp[jj] * kLog2e);
+          for (int j = 0; j < 64; ++j) {
+            const int jj = min(j0 + j, p.nb - 1);
+            const bool m = (j >= valid) || ((bm[jj >> 5] >> (jj & 31)) & 1u);
+            x[j] = m ? -INFINITY : fmaf(x[j], p.scale_log2, bp[jj] * kLog2e);
           }
         }
-        float mx = x[0];
+        // row max: tree over this thread's 64 keys, then the partner half
+        float mx;
+        {
+          float t8[8];
 #pragma unroll
-        for (int j = 1; j < 32; ++j) mx = fmaxf(mx, x[j]);
+          for (int i = 0; i < 8; ++i) {
+            const float a0 = fmaxf(x[i], x[i + 8]), a1 = fmaxf(x[i + 16], x[i + 24]);
+            const float a2 = fmaxf(x[i + 32], x[i + 40]), a3 = fmaxf(x[i + 48], x[i + 56]);
+            t8[i] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          }
+          mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                     fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+        }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + 8.0f;  // also true when m_run = -inf and m_new finite
@@ -579,28 +674,33 @@ __global__ void __launch_bounds__(320, 1)
           m_run = m_new;
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        uint32_t pk[16];
-        float ls = 0.f;
+        uint32_t pk[32];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 32; ++j) {
           const float p0 = ex2f(x[2 * j] - m_use);
           const float p1 = ex2f(x[2 * j + 1] - m_use);
-          ls += p0 + p1;
+          ls[j & 3] += p0 + p1;
           pk[j] = pack_bf16x2(p0, p1);
         }
-        l_run += ls;
-        tc::tmem_st_16x32bx2_x16<16>(tbase + lanes + C::kColS + 64 * b, pk);
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        SPARK_TC_ACC(7, t_cp);
+        SPARK_TC_T0(t_st);
+        // P over S: packed columns 32h .. 32h+31 of the buffer
+        tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b, pk);
+        tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b + 16, pk + 16);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&pfull[2 * s + b]);
+        SPARK_TC_ACC(8, t_st);
+        SPARK_TC_EV(1 + s, 41);
       }
       if (!ok) break;
       have_prev = 1;
       prev = I;
       m_prev = m_run;
       l_prev = l_run;
-      g_prev_last = g - 1;
       ++nitem;
     }
   }

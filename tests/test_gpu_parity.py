@@ -196,3 +196,19 @@ def test_full_size_sampled(spark, name, mode, param, compressed):
     for h in (0, H - 1):
         compare_head(plan, O, L, Qc, Kc, Vc, 0, h, ns, cfg, qblocks=sample_blocks(nb, 6, h),
                      check_pool=(h == 0), dense=(mode == "topk" and param == 0.1))
+
+
+def test_many_items_per_slot_stay_in_sync(spark):
+    """Many short items per CTA slot, repeated: every pipeline barrier must stay in phase
+    (a wait that gives up reports SPARK_ETIMEOUT) and the results must be bitwise stable."""
+    Q, K, V = make_qkv(1, 6, 64 * 700, 40, 128, seed=7, device=DEV)
+    cfg = spark.ForwardConfig("tau", 1.8, False)   # few selected blocks: 1-3 tiles per item
+    plan = spark.SparkAttention(1, 6, Q.shape[2], 128, 40, cfg, DEV)
+    O0, L0 = (t.clone() for t in plan.run(Q, K, V))
+    for _ in range(15):
+        plan.run(Q, K, V)
+        torch.cuda.synchronize()
+        assert spark.device_error() == 0
+        assert torch.equal(plan.O, O0) and torch.equal(plan.lse, L0)
+    Qc, Kc, Vc = Q.cpu(), K.cpu(), V.cpu()
+    compare_head(plan, plan.O, plan.lse, Qc, Kc, Vc, 0, 5, 40, cfg, qblocks=sample_blocks(plan.nb, 6, 1))
