@@ -1,20 +1,1015 @@
-// Spark-Reblock (whitened median bisection) — declared here, implemented below.
+// Spark-Reblock: data-dependent block layout by whitened median bisection.
+//
+// Method: "Spark-H3: speeding up MiniMax-H3 in ComfyUI with block-sparse attention",
+// section "What Spark-Attn changes", Spark-Reblock bullet: two queries are alike when their
+// attention-score patterns over the keys are alike, measured by the Mahalanobis cosine under
+// the opposite side's (the keys') second moment; a hierarchical partitioner splits groups
+// until every leaf holds the block size, in O(N log N), so the layout follows the input,
+// layer and head. Section "Workflows": reblock_layout=q_reuse_k (keys reuse the query
+// partition).
+//
+// Per (batch, head), level-synchronous:
+//   M = mean_j k_j k_j^T (fp32 tile products, fp64 accumulation); M = L L^T (fp64 Cholesky,
+//   retried with 1e-6 tr(M)/d on the diagonal, identity if that fails too);
+//   x_i = L^T q_i / |L^T q_i| (fp32);
+//   every node of m > 1 blocks: centred covariance of its x (fp64 accumulation), leading
+//   eigenvector v (fp64 Householder tridiagonalisation, Sturm multisection, inverse
+//   iteration), projections x.v signed so their third central moment is >= 0, the
+//   floor(m/2)*64-th smallest (projection, token) by radix select, stable partition;
+//   leaves ordered by smallest token, tokens ascending; Q/K/V rows gathered.
+// The tree shape depends only on nb, so the host walks it; nodes at most 64 blocks big are
+// split together with their whole subtree by one CTA, larger nodes (the first few levels)
+// accumulate their covariance over many CTAs with fp64 atomics.
 #pragma once
+#include <vector>
+
 #include "spark_common.cuh"
 
 namespace spark {
+namespace rb {
+
+constexpr int kThreads = 256;
+constexpr int kSmallBlocks = 64;   // nodes up to this many blocks are split by one CTA subtree
+constexpr int kChunkTok = 4096;    // tokens per CTA of the multi-CTA accumulations
+constexpr int kTile = 64;          // tokens staged per covariance step
+
+// Node (level, label) -> first block and block count, following the label bits from the
+// root (bit 1 = right child). Returns false for labels no node carries at that level.
+__host__ __device__ inline bool node_of(int nb, int level, int label, int* start, int* m) {
+  int st = 0, mm = nb;
+  for (int l = level - 1; l >= 0; --l) {
+    const int bit = (label >> l) & 1;
+    if (mm == 1) {
+      if (bit) return false;
+      continue;
+    }
+    const int ml = mm / 2;
+    if (bit) {
+      st += ml;
+      mm -= ml;
+    } else {
+      mm = ml;
+    }
+  }
+  *start = st;
+  *m = mm;
+  return true;
+}
+
+inline int num_levels(int nb) {
+  int L = 0;
+  while ((1 << L) < nb) ++L;
+  return L;
+}
+
+// ------------------------------------------------------------------ block reductions
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// Sum over the CTA; every thread gets the result. `red` holds kThreads/32 doubles.
+__device__ __forceinline__ double block_sum_d(double v, double* red) {
+  v = warp_sum_d(v);
+  const int w = threadIdx.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+  return t;
+}
+
+// ------------------------------------------------------------------ second moments
+// Adds sum over `rows` of r r^T (and sum of r when S1 != nullptr) into fp64 accumulators
+// held in shared memory (S2: D x D, S1: D). Rows are staged 64 at a time as fp32; each
+// thread owns an (D/16) x (D/16) sub-block, sums a tile in fp32, then adds it in fp64.
+// `load_row(i, dst)` writes row i (0 <= i < n) as D floats into dst.
+template <int D, class LoadRow>
+__device__ void accumulate_moments(int n, LoadRow load_row, float* stage, double* S2, double* S1) {
+  constexpr int S = D / 16;
+  constexpr int LD = D + 4;  // padded staging row
+  const int tid = threadIdx.x;
+  const int ti = tid / 16, tj = tid % 16;
+  for (int t0 = 0; t0 < n; t0 += kTile) {
+    const int nt = min(kTile, n - t0);
+    __syncthreads();
+    for (int r = tid / (D / 4); r < kTile; r += kThreads / (D / 4)) {
+      float* dst = stage + r * LD;
+      if (r < nt) {
+        load_row(t0 + r, dst, tid % (D / 4));
+      } else {
+        reinterpret_cast<float4*>(dst)[tid % (D / 4)] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    __syncthreads();
+    float acc[S][S];
+#pragma unroll
+    for (int a = 0; a < S; ++a)
+#pragma unroll
+      for (int b = 0; b < S; ++b) acc[a][b] = 0.f;
+    for (int r = 0; r < kTile; ++r) {
+      const float* row = stage + r * LD;
+      float xa[S], xb[S];
+#pragma unroll
+      for (int a = 0; a < S; ++a) {
+        xa[a] = row[ti * S + a];
+        xb[a] = row[tj * S + a];
+      }
+#pragma unroll
+      for (int a = 0; a < S; ++a)
+#pragma unroll
+        for (int b = 0; b < S; ++b) acc[a][b] = fmaf(xa[a], xb[b], acc[a][b]);
+    }
+#pragma unroll
+    for (int a = 0; a < S; ++a)
+#pragma unroll
+      for (int b = 0; b < S; ++b) S2[(ti * S + a) * D + tj * S + b] += (double)acc[a][b];
+    if (S1 != nullptr && tid < D) {
+      float cs = 0.f;
+      for (int r = 0; r < kTile; ++r) cs += stage[r * LD + tid];
+      S1[tid] += (double)cs;
+    }
+  }
+  __syncthreads();
+}
+
+// Key second moment of one head: grid (chunks, B*H); fp64 atomics into macc[bh][D][D].
+template <int D>
+__global__ void __launch_bounds__(kThreads) kmoment_kernel(const uint16_t* __restrict__ K, int N, int nv,
+                                                           double* __restrict__ macc) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  double* S2 = reinterpret_cast<double*>(smem);
+  float* stage = reinterpret_cast<float*>(S2 + D * D);
+  const size_t bh = blockIdx.y;
+  const int r0 = blockIdx.x * kChunkTok;
+  const int n = min(kChunkTok, nv - r0);
+  if (n <= 0) return;
+  for (int i = threadIdx.x; i < D * D; i += kThreads) S2[i] = 0.0;
+  const uint16_t* kb = K + (bh * N + r0) * D;
+  auto load = [&](int i, float* dst, int c4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(kb + (size_t)i * D + 4 * c4);
+    dst[4 * c4 + 0] = __uint_as_float(u.x << 16);
+    dst[4 * c4 + 1] = __uint_as_float(u.x & 0xffff0000u);
+    dst[4 * c4 + 2] = __uint_as_float(u.y << 16);
+    dst[4 * c4 + 3] = __uint_as_float(u.y & 0xffff0000u);
+  };
+  accumulate_moments<D>(n, load, stage, S2, nullptr);
+  double* dst = macc + bh * D * D;
+  for (int i = threadIdx.x; i < D * D; i += kThreads) atomicAdd(dst + i, S2[i]);
+}
+
+// In-place lower Cholesky of A (fp64, D x D in shared memory). Returns false on a
+// non-positive pivot.
+template <int D>
+__device__ bool cholesky_inplace(double* A, int* fail) {
+  const int tid = threadIdx.x;
+  if (tid == 0) *fail = 0;
+  __syncthreads();
+  for (int j = 0; j < D; ++j) {
+    if (tid == 0) {
+      const double dj = A[j * D + j];
+      if (!(dj > 0.0)) *fail = 1;
+      A[j * D + j] = dj > 0.0 ? sqrt(dj) : 1.0;
+    }
+    __syncthreads();
+    if (*fail) return false;
+    const double piv = A[j * D + j];
+    for (int i = j + 1 + tid; i < D; i += kThreads) A[i * D + j] /= piv;
+    __syncthreads();
+    const int m = D - j - 1;
+    for (int e = tid; e < m * m; e += kThreads) {
+      const int i = j + 1 + e / m, k = j + 1 + e % m;
+      if (k <= i) A[i * D + k] -= A[i * D + j] * A[k * D + j];
+    }
+    __syncthreads();
+  }
+  return true;
+}
+
+// L of each head (fp32 row-major, upper triangle zero): grid B*H.
+template <int D>
+__global__ void __launch_bounds__(kThreads) cholesky_kernel(const double* __restrict__ macc, int nv,
+                                                            float* __restrict__ lmat) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  double* A = reinterpret_cast<double*>(smem);
+  __shared__ int fail;
+  __shared__ double red[kThreads / 32];
+  const size_t bh = blockIdx.x;
+  const double* src = macc + bh * D * D;
+  const double inv_n = nv > 0 ? 1.0 / nv : 0.0;
+  bool ok = false;
+  for (int attempt = 0; attempt < 2 && !ok; ++attempt) {
+    double tr = 0.0;
+    for (int i = threadIdx.x; i < D; i += kThreads) tr += src[i * D + i] * inv_n;
+    tr = block_sum_d(tr, red);
+    const double jitter = attempt == 0 ? 0.0 : 1e-6 * tr / D;
+    for (int e = threadIdx.x; e < D * D; e += kThreads)
+      A[e] = src[e] * inv_n + ((e / D == e % D) ? jitter : 0.0);
+    __syncthreads();
+    ok = cholesky_inplace<D>(A, &fail);
+  }
+  float* L = lmat + bh * D * D;
+  for (int e = threadIdx.x; e < D * D; e += kThreads) {
+    const int i = e / D, k = e % D;
+    L[e] = ok ? (k <= i ? (float)A[e] : 0.f) : (i == k ? 1.f : 0.f);
+  }
+}
+
+// x_i = L^T q_i / |L^T q_i| for the video rows of every head; also tok[i] = i and the
+// level-0 tree labels. grid (ceil(nv / 64), B*H).
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+    whiten_kernel(const uint16_t* __restrict__ Q, int N, int nv, const float* __restrict__ lmat,
+                  float* __restrict__ X, int32_t* __restrict__ tok, int32_t* __restrict__ tree0,
+                  size_t tree_head_stride) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* Ls = reinterpret_cast<float*>(smem);  // D x D
+  float* qs = Ls + D * D;                      // 64 x (D + 4)
+  constexpr int LD = D + 4;
+  constexpr int CG = D / 4;                    // columns per thread
+  const size_t bh = blockIdx.y;
+  const int t0 = blockIdx.x * 64;
+  const int tid = threadIdx.x;
+  const float* L = lmat + bh * D * D;
+  for (int e = tid; e < D * D / 4; e += kThreads)
+    reinterpret_cast<float4*>(Ls)[e] = reinterpret_cast<const float4*>(L)[e];
+  for (int e = tid; e < 64 * D / 2; e += kThreads) {
+    const int r = e / (D / 2), c2 = e % (D / 2);
+    const int t = t0 + r;
+    uint32_t u = 0;
+    if (t < nv) u = *reinterpret_cast<const uint32_t*>(Q + (bh * N + t) * D + 2 * c2);
+    qs[r * LD + 2 * c2] = __uint_as_float(u << 16);
+    qs[r * LD + 2 * c2 + 1] = __uint_as_float(u & 0xffff0000u);
+  }
+  __syncthreads();
+  const int r = tid / 4, cg = tid % 4;  // token r of the tile, columns cg*CG ..
+  const int t = t0 + r;
+  float acc[CG];
+#pragma unroll
+  for (int c = 0; c < CG; ++c) acc[c] = 0.f;
+  for (int k = 0; k < D; ++k) {
+    const float qk = qs[r * LD + k];
+    const float* lr = Ls + k * D + cg * CG;
+#pragma unroll
+    for (int c = 0; c < CG; ++c) acc[c] = fmaf(qk, lr[c], acc[c]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < CG; ++c) ss = fmaf(acc[c], acc[c], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+  if (t < nv) {
+    float* xr = X + (bh * nv + t) * D + cg * CG;
+#pragma unroll
+    for (int c = 0; c < CG; c += 4)
+      *reinterpret_cast<float4*>(xr + c) =
+          make_float4(acc[c] * inv, acc[c + 1] * inv, acc[c + 2] * inv, acc[c + 3] * inv);
+    if (cg == 0) {
+      tok[bh * nv + t] = t;
+      if (tree0 != nullptr) tree0[bh * tree_head_stride + t] = 0;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ node covariance
+// C = centred covariance (fp64, D x D) and mu = mean of the n whitened rows x[tok[i]].
+template <int D>
+__device__ void node_covariance(const float* __restrict__ Xh, const int32_t* __restrict__ tseg,
+                                int n, float* stage, double* C, double* mu) {
+  for (int i = threadIdx.x; i < D * D; i += kThreads) C[i] = 0.0;
+  for (int i = threadIdx.x; i < D; i += kThreads) mu[i] = 0.0;
+  auto load = [&](int i, float* dst, int c4) {
+    const int t = tseg[i];
+    reinterpret_cast<float4*>(dst)[c4] = reinterpret_cast<const float4*>(Xh + (size_t)t * D)[c4];
+  };
+  accumulate_moments<D>(n, load, stage, C, mu);
+  const double inv = 1.0 / n;
+  for (int i = threadIdx.x; i < D; i += kThreads) mu[i] *= inv;
+  __syncthreads();
+  for (int e = threadIdx.x; e < D * D; e += kThreads) C[e] = C[e] * inv - mu[e / D] * mu[e % D];
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ leading eigenvector
+// Scratch layout (doubles): a, e, e2, beta, u, w, y, dd, du, du2, dl (D each), red (8),
+// misc (8); piv (D ints) after that.
+template <int D>
+struct EigScratch {
+  static constexpr int kDoubles = 11 * D + 16;
+  static constexpr int kBytes = kDoubles * 8 + D * 4;
+};
+
+__device__ __forceinline__ int sturm_count(const double* a, const double* e2, int n, double x,
+                                           double pivmin) {
+  int c = 0;
+  double q = a[0] - x;
+  if (q < 0.0) ++c;
+  for (int i = 1; i < n; ++i) {
+    const double den = fabs(q) < pivmin ? -pivmin : q;
+    q = (a[i] - x) - e2[i - 1] / den;
+    if (q < 0.0) ++c;
+  }
+  return c;
+}
+
+// Unit eigenvector of the largest eigenvalue of the symmetric matrix C (fp64, shared
+// memory, destroyed) into v (shared). Householder tridiagonalisation T = H^T C H, the
+// largest eigenvalue of T by multisection on Sturm counts, its eigenvector by inverse
+// iteration (tridiagonal LU with partial pivoting), then v = H y.
+template <int D>
+__device__ void eigen_top(double* C, double* scr, double* v) {
+  double* a = scr;
+  double* e = a + D;
+  double* e2 = e + D;
+  double* bt = e2 + D;
+  double* u = bt + D;
+  double* w = u + D;
+  double* y = w + D;
+  double* dd = y + D;
+  double* du = dd + D;
+  double* du2 = du + D;
+  double* dl = du2 + D;
+  double* red = dl + D;
+  double* misc = red + 8;
+  int* piv = reinterpret_cast<int*>(misc + 8);
+  const int tid = threadIdx.x;
+
+  // ---- tridiagonalisation
+  for (int k = 0; k < D - 2; ++k) {
+    const int m = D - k - 1;
+    for (int i = tid; i < m; i += kThreads) u[i] = C[(k + 1 + i) * D + k];
+    __syncthreads();
+    double ss = 0.0;
+    for (int i = tid; i < m; i += kThreads) ss += u[i] * u[i];
+    const double norm2 = block_sum_d(ss, red);
+    const double x0 = u[0];
+    const double tail = norm2 - x0 * x0;
+    __syncthreads();
+    if (!(tail > 1e-300 * (norm2 + 1e-300))) {  // column already reduced
+      if (tid == 0) {
+        bt[k] = 0.0;
+        e[k] = x0;
+      }
+      __syncthreads();
+      continue;
+    }
+    const double alpha = -copysign(sqrt(norm2), x0);
+    const double u0 = x0 - alpha;
+    const double beta = 2.0 / (tail + u0 * u0);
+    if (tid == 0) {
+      u[0] = u0;
+      bt[k] = beta;
+      e[k] = alpha;
+    }
+    __syncthreads();
+    for (int i = tid; i < m; i += kThreads) C[(k + 1 + i) * D + k] = u[i];
+    // w = beta * C' u over the trailing block (column reads; the block is symmetric)
+    {
+      const int i = tid >> 1, h = tid & 1;
+      double s = 0.0;
+      if (i < m)
+        for (int j = h; j < m; j += 2) s += C[(k + 1 + j) * D + (k + 1 + i)] * u[j];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      if (i < m && h == 0) w[i] = beta * s;  // m <= 127 < kThreads / 2 rows
+    }
+    __syncthreads();
+    double dot = 0.0;
+    for (int i = tid; i < m; i += kThreads) dot += u[i] * w[i];
+    const double kc = 0.5 * beta * block_sum_d(dot, red);
+    for (int i = tid; i < m; i += kThreads) w[i] -= kc * u[i];
+    __syncthreads();
+    for (int q = tid; q < m * m; q += kThreads) {
+      const int i = q / m, j = q % m;
+      C[(k + 1 + i) * D + (k + 1 + j)] -= u[i] * w[j] + w[i] * u[j];
+    }
+    __syncthreads();
+  }
+  for (int i = tid; i < D; i += kThreads) a[i] = C[i * D + i];
+  if (tid == 0) e[D - 2] = C[(D - 1) * D + (D - 2)];
+  __syncthreads();
+  for (int i = tid; i < D - 1; i += kThreads) e2[i] = e[i] * e[i];
+
+  // ---- largest eigenvalue of T: Gershgorin interval, then multisection
+  double glo = 1e300, ghi = -1e300, emax = 0.0;
+  for (int i = tid; i < D; i += kThreads) {
+    const double r = (i > 0 ? fabs(e[i - 1]) : 0.0) + (i < D - 1 ? fabs(e[i]) : 0.0);
+    glo = fmin(glo, a[i] - r);
+    ghi = fmax(ghi, a[i] + r);
+    if (i < D - 1) emax = fmax(emax, e[i] * e[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    glo = fmin(glo, __shfl_xor_sync(0xffffffffu, glo, o));
+    ghi = fmax(ghi, __shfl_xor_sync(0xffffffffu, ghi, o));
+    emax = fmax(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  }
+  __syncthreads();
+  if ((tid & 31) == 0) {
+    red[tid >> 5] = glo;
+    w[tid >> 5] = ghi;
+    y[tid >> 5] = emax;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double lo = red[0], hi = w[0], em = y[0];
+    for (int i = 1; i < kThreads / 32; ++i) {
+      lo = fmin(lo, red[i]);
+      hi = fmax(hi, w[i]);
+      em = fmax(em, y[i]);
+    }
+    const double span = fmax(fabs(lo), fabs(hi)) + 1e-300;
+    misc[0] = lo - 1e-12 * span;
+    misc[1] = hi + 1e-12 * span;
+    misc[2] = 2.2250738585072014e-308 * fmax(1.0, em);
+  }
+  __syncthreads();
+  const double pivmin = misc[2];
+  for (int round = 0; round < 12; ++round) {
+    const double lo = misc[0], hi = misc[1];
+    if (hi - lo <= 4e-16 * fmax(fabs(lo), fabs(hi))) break;
+    const double x = lo + (hi - lo) * (double)(tid + 1) / (double)(kThreads + 1);
+    const int c = sturm_count(a, e2, D, x, pivmin);
+    double clo = (c <= D - 1) ? x : -1e300;  // at or below the top eigenvalue
+    double chi = (c == D) ? x : 1e300;       // above it
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      clo = fmax(clo, __shfl_xor_sync(0xffffffffu, clo, o));
+      chi = fmin(chi, __shfl_xor_sync(0xffffffffu, chi, o));
+    }
+    __syncthreads();
+    if ((tid & 31) == 0) {
+      red[tid >> 5] = clo;
+      w[tid >> 5] = chi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double nlo = misc[0], nhi = misc[1];
+      for (int i = 0; i < kThreads / 32; ++i) {
+        nlo = fmax(nlo, red[i]);
+        nhi = fmin(nhi, w[i]);
+      }
+      misc[0] = nlo;
+      misc[1] = nhi;
+    }
+    __syncthreads();
+  }
+  const double theta = 0.5 * (misc[0] + misc[1]);
+
+  // ---- eigenvector of T by inverse iteration (one thread; O(D) per solve)
+  if (tid == 0) {
+    const double tiny = 1e-30 * (fabs(theta) + 1e-300);
+    for (int i = 0; i < D; ++i) {
+      dd[i] = a[i] - theta;
+      if (i < D - 1) dl[i] = du[i] = e[i];
+      du2[i] = 0.0;
+    }
+    for (int i = 0; i < D - 1; ++i) {
+      if (fabs(dd[i]) >= fabs(dl[i])) {
+        if (dd[i] == 0.0) dd[i] = tiny;
+        const double f = dl[i] / dd[i];
+        dl[i] = f;
+        dd[i + 1] -= f * du[i];
+        piv[i] = 0;
+      } else {
+        const double f = dd[i] / dl[i];
+        dd[i] = dl[i];
+        dl[i] = f;
+        const double tmp = du[i];
+        du[i] = dd[i + 1];
+        dd[i + 1] = tmp - f * dd[i + 1];
+        if (i < D - 2) {
+          du2[i] = du[i + 1];
+          du[i + 1] = -f * du[i + 1];
+        }
+        piv[i] = 1;
+      }
+    }
+    if (dd[D - 1] == 0.0) dd[D - 1] = tiny;
+    for (int i = 0; i < D; ++i) y[i] = 1.0 + 0.001 * i;
+    for (int it = 0; it < 3; ++it) {
+      for (int i = 0; i < D - 1; ++i) {
+        if (piv[i] == 0) {
+          y[i + 1] -= dl[i] * y[i];
+        } else {
+          const double tmp = y[i] - dl[i] * y[i + 1];
+          y[i] = y[i + 1];
+          y[i + 1] = tmp;
+        }
+      }
+      y[D - 1] /= dd[D - 1];
+      y[D - 2] = (y[D - 2] - du[D - 2] * y[D - 1]) / dd[D - 2];
+      for (int i = D - 3; i >= 0; --i) y[i] = (y[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) / dd[i];
+      double nn = 0.0;
+      for (int i = 0; i < D; ++i) nn += y[i] * y[i];
+      const double inv = 1.0 / sqrt(nn);
+      for (int i = 0; i < D; ++i) y[i] *= inv;
+    }
+  }
+  __syncthreads();
+
+  // ---- back-transform v = H_0 ... H_{D-3} y (one warp)
+  if (tid < 32) {
+    for (int k = D - 3; k >= 0; --k) {
+      const double b = bt[k];
+      if (b == 0.0) continue;
+      const int m = D - k - 1;
+      double s = 0.0;
+      for (int i = tid; i < m; i += 32) s += C[(k + 1 + i) * D + k] * y[k + 1 + i];
+      s = warp_sum_d(s) * b;
+      for (int i = tid; i < m; i += 32) y[k + 1 + i] -= s * C[(k + 1 + i) * D + k];
+      __syncwarp();
+    }
+    double nn = 0.0;
+    for (int i = tid; i < D; i += 32) nn += y[i] * y[i];
+    nn = warp_sum_d(nn);
+    const double inv = 1.0 / sqrt(nn);
+    for (int i = tid; i < D; i += 32) v[i] = y[i] * inv;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------ one bisection
+struct SplitScratch {
+  int hist[256];
+  int warp_tot[kThreads / 32];
+  double red[kThreads / 32];
+  int sel[4];  // bin, remaining rank, count of equal keys, chosen token
+};
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Radix select over the n values key(i) (uint32) restricted to filt(i): returns the
+// r-th smallest (1-based) and leaves in sc->sel[1] its rank among equal values and in
+// sc->sel[2] how many values equal it.
+template <class KeyF, class FiltF>
+__device__ uint32_t radix_select(int n, int r, KeyF key, FiltF filt, SplitScratch* sc) {
+  uint32_t prefix = 0, mask = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = threadIdx.x; b < 256; b += kThreads) sc->hist[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      if (!filt(i)) continue;
+      const uint32_t k = key(i);
+      if ((k & mask) == prefix) atomicAdd(&sc->hist[(k >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int cum = 0, b = 0;
+      for (; b < 255; ++b) {
+        if (cum + sc->hist[b] >= r) break;
+        cum += sc->hist[b];
+      }
+      sc->sel[0] = b;
+      sc->sel[1] = r - cum;
+      sc->sel[2] = sc->hist[b];
+    }
+    __syncthreads();
+    prefix |= (uint32_t)sc->sel[0] << shift;
+    mask |= 255u << shift;
+    r = sc->sel[1];
+    __syncthreads();
+  }
+  return prefix;
+}
+
+// Splits one node of m > 1 blocks (n = 64 m tokens): projections on v (fp64 dot products,
+// stored as fp32), sign from the third central moment, the floor(m/2)*64-th smallest
+// (projection, token) and a stable partition of tin into tout (left part first). Writes
+// the children's labels 2c / 2c + 1 into tree_next when it is not null.
+template <int D>
+__device__ void split_node(const double* v, const float* __restrict__ Xh, const int32_t* tin,
+                           int32_t* tout, float* proj, int n, int m, int label,
+                           int32_t* tree_next, SplitScratch* sc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int PL = D / 32;  // components per lane
+  double vl[PL];
+#pragma unroll
+  for (int j = 0; j < PL; ++j) vl[j] = v[lane * PL + j];
+  double psum = 0.0;
+  for (int i = warp; i < n; i += kThreads / 32) {
+    const int t = tin[i];
+    const float* xr = Xh + (size_t)t * D + lane * PL;
+    double d = 0.0;
+#pragma unroll
+    for (int j = 0; j < PL; ++j) d = fma((double)xr[j], vl[j], d);
+    d = warp_sum_d(d);
+    if (lane == 0) {
+      proj[i] = (float)d;
+      psum += d;
+    }
+  }
+  __syncthreads();
+  const double pbar = block_sum_d(psum, sc->red) / n;
+  double m3 = 0.0;
+  for (int i = tid; i < n; i += kThreads) {
+    const double c = (double)proj[i] - pbar;
+    m3 += c * c * c;
+  }
+  m3 = block_sum_d(m3, sc->red);
+  const float sgn = m3 < 0.0 ? -1.f : 1.f;
+  const int cut = (m / 2) * kBlock;
+  auto pkey = [&](int i) { return order_key(sgn * proj[i]); };
+  auto all = [](int) { return true; };
+  const uint32_t T = radix_select(n, cut, pkey, all, sc);
+  const int r_eq = sc->sel[1], n_eq = sc->sel[2];
+  __syncthreads();
+  uint32_t Ttok = 0xffffffffu;  // ties at T: the r_eq lowest tokens go left
+  if (n_eq > r_eq) {
+    auto tkey = [&](int i) { return (uint32_t)tin[i]; };
+    auto eq = [&](int i) { return pkey(i) == T; };
+    Ttok = radix_select(n, r_eq, tkey, eq, sc);
+  }
+  // stable partition
+  int nl_base = 0;
+  for (int base = 0; base < n; base += kThreads) {
+    const int i = base + tid;
+    int t = 0;
+    bool left = false;
+    if (i < n) {
+      t = tin[i];
+      const uint32_t k = pkey(i);
+      left = k < T || (k == T && (uint32_t)t <= Ttok);
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, left);
+    const int wrank = __popc(bal & ((1u << lane) - 1u));
+    __syncthreads();
+    if (lane == 0) sc->warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int q = 0; q < kThreads / 32; ++q) {
+      const int c = sc->warp_tot[q];
+      before += q < warp ? c : 0;
+      total += c;
+    }
+    if (i < n) {
+      const int lrank = nl_base + before + wrank;
+      const int pos = left ? lrank : cut + (i - lrank);
+      tout[pos] = t;
+      if (tree_next != nullptr) tree_next[t] = 2 * label + (left ? 0 : 1);
+    }
+    nl_base += total;
+  }
+  __syncthreads();
+}
+
+// A leaf carried to the next level: same tokens, label 2c.
+__device__ __forceinline__ void carry_leaf(const int32_t* tin, int32_t* tout, int label,
+                                           int32_t* tree_next) {
+  for (int i = threadIdx.x; i < kBlock; i += kThreads) {
+    const int t = tin[i];
+    tout[i] = t;
+    if (tree_next != nullptr) tree_next[t] = 2 * label;
+  }
+}
+
+// Shared memory of the split kernels: C (D x D doubles), mu, v, eigen scratch, staging,
+// split scratch.
+template <int D>
+struct SplitSmem {
+  static constexpr int kC = D * D * 8;
+  static constexpr int kVec = 2 * D * 8;
+  static constexpr int kStage = kTile * (D + 4) * 4;
+  static constexpr int kBytes = kC + kVec + EigScratch<D>::kBytes + kStage + (int)sizeof(SplitScratch) + 64;
+};
+
+struct LevelArgs {
+  const float* X;     // [BH][nv][D]
+  const int32_t* tin; // [BH][nv]
+  int32_t* tout;
+  float* proj;        // [BH][nv]
+  int32_t* tree;      // [BH][L+1][nv] or null
+  int nv, nb, level, levels;
+};
+
+template <int D>
+__device__ __forceinline__ void carve(unsigned char* smem, double** C, double** mu, double** v,
+                                      double** scr, float** stage, SplitScratch** sc) {
+  using S = SplitSmem<D>;
+  *C = reinterpret_cast<double*>(smem);
+  *mu = reinterpret_cast<double*>(smem + S::kC);
+  *v = *mu + D;
+  *scr = reinterpret_cast<double*>(smem + S::kC + S::kVec);
+  *stage = reinterpret_cast<float*>(smem + S::kC + S::kVec + EigScratch<D>::kBytes);
+  *sc = reinterpret_cast<SplitScratch*>(smem + S::kC + S::kVec + EigScratch<D>::kBytes + S::kStage);
+}
+
+// Large levels, step 1: covariance sums of every node over chunks of its tokens, fp64
+// atomics into nacc[node][bh] = (S2 [D x D], S1 [D]). grid (nodes * cpn, BH).
+template <int D>
+__global__ void __launch_bounds__(kThreads) node_moments_kernel(LevelArgs a, int cpn, double* __restrict__ nacc) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  double* S2 = reinterpret_cast<double*>(smem);
+  double* S1 = S2 + D * D;
+  float* stage = reinterpret_cast<float*>(S1 + D);
+  const int c = blockIdx.x / cpn, chunk = blockIdx.x % cpn;
+  const size_t bh = blockIdx.y;
+  int st, m;
+  if (!node_of(a.nb, a.level, c, &st, &m) || m <= 1) return;
+  const int t0 = chunk * kChunkTok;
+  const int n = min(kChunkTok, m * kBlock - t0);
+  if (n <= 0) return;
+  for (int i = threadIdx.x; i < D * D + D; i += kThreads) S2[i] = 0.0;
+  const float* Xh = a.X + bh * (size_t)a.nv * D;
+  const int32_t* tseg = a.tin + bh * (size_t)a.nv + st * kBlock + t0;
+  auto load = [&](int i, float* dst, int c4) {
+    const int t = tseg[i];
+    reinterpret_cast<float4*>(dst)[c4] = reinterpret_cast<const float4*>(Xh + (size_t)t * D)[c4];
+  };
+  accumulate_moments<D>(n, load, stage, S2, S1);
+  double* dst = nacc + ((size_t)c * gridDim.y + bh) * (D * D + D);
+  for (int i = threadIdx.x; i < D * D + D; i += kThreads) atomicAdd(dst + i, S2[i]);
+}
+
+// Large levels, step 2: one CTA per node finishes the covariance, finds the eigenvector and
+// splits (or carries a leaf). grid (nodes, BH).
+template <int D>
+__global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, const double* __restrict__ nacc) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  double *C, *mu, *v, *scr;
+  float* stage;
+  SplitScratch* sc;
+  carve<D>(smem, &C, &mu, &v, &scr, &stage, &sc);
+  const int c = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  int st, m;
+  if (!node_of(a.nb, a.level, c, &st, &m)) return;
+  const size_t hoff = bh * (size_t)a.nv + st * kBlock;
+  int32_t* tree_next = a.tree ? a.tree + bh * (size_t)(a.levels + 1) * a.nv + (size_t)(a.level + 1) * a.nv : nullptr;
+  if (m == 1) {
+    carry_leaf(a.tin + hoff, a.tout + hoff, c, tree_next);
+    return;
+  }
+  const int n = m * kBlock;
+  const double* src = nacc + ((size_t)c * gridDim.y + bh) * (D * D + D);
+  const double inv = 1.0 / n;
+  for (int i = threadIdx.x; i < D; i += kThreads) mu[i] = src[D * D + i] * inv;
+  __syncthreads();
+  for (int e = threadIdx.x; e < D * D; e += kThreads) C[e] = src[e] * inv - mu[e / D] * mu[e % D];
+  __syncthreads();
+  eigen_top<D>(C, scr, v);
+  split_node<D>(v, a.X + bh * (size_t)a.nv * D, a.tin + hoff, a.tout + hoff, a.proj + hoff, n, m, c,
+                tree_next, sc);
+}
+
+// Small nodes: one CTA per node of level `level` splits it and its whole subtree down to
+// single blocks, reading and writing the token arrays tok[lev & 1] -> tok[(lev + 1) & 1].
+template <int D>
+__global__ void __launch_bounds__(kThreads) subtree_kernel(LevelArgs a, int32_t* tok0, int32_t* tok1) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  double *C, *mu, *v, *scr;
+  float* stage;
+  SplitScratch* sc;
+  carve<D>(smem, &C, &mu, &v, &scr, &stage, &sc);
+  const int c0 = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  int st0, m0;
+  if (!node_of(a.nb, a.level, c0, &st0, &m0)) return;
+  const float* Xh = a.X + bh * (size_t)a.nv * D;
+  for (int lev = a.level; lev < a.levels; ++lev) {
+    const int span = 1 << (lev - a.level);
+    const int32_t* tin = (lev & 1) ? tok1 : tok0;
+    int32_t* tout = (lev & 1) ? tok0 : tok1;
+    int32_t* tree_next = a.tree ? a.tree + bh * (size_t)(a.levels + 1) * a.nv + (size_t)(lev + 1) * a.nv : nullptr;
+    for (int cc = c0 * span; cc < (c0 + 1) * span; ++cc) {
+      int st, m;
+      if (!node_of(a.nb, lev, cc, &st, &m)) continue;
+      const size_t hoff = bh * (size_t)a.nv + st * kBlock;
+      if (m == 1) {
+        carry_leaf(tin + hoff, tout + hoff, cc, tree_next);
+        __syncthreads();
+        continue;
+      }
+      const int n = m * kBlock;
+      node_covariance<D>(Xh, tin + hoff, n, stage, C, mu);
+      eigen_top<D>(C, scr, v);
+      split_node<D>(v, Xh, tin + hoff, tout + hoff, a.proj + hoff, n, m, cc, tree_next, sc);
+    }
+    __syncthreads();  // the next level reads what this level wrote (same CTA)
+    __threadfence_block();
+  }
+}
+
+// ------------------------------------------------------------------ canonical order
+// Sorts the 64 tokens of every leaf ascending (in place) and marks each leaf's smallest
+// token: mark[bh][token] = leaf + 1. One warp per leaf; grid (ceil(nb / 8), BH).
+__global__ void __launch_bounds__(kThreads) leaf_sort_kernel(int32_t* tok, int nv, int nb, int32_t* mark) {
+  __shared__ int32_t buf[kThreads / 32][kBlock];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int leaf = blockIdx.x * (kThreads / 32) + warp;
+  if (leaf >= nb) return;
+  const size_t bh = blockIdx.y;
+  int32_t* seg = tok + bh * (size_t)nv + (size_t)leaf * kBlock;
+  const int a = seg[lane], b = seg[lane + 32];
+  buf[warp][lane] = a;
+  buf[warp][lane + 32] = b;
+  __syncwarp();
+  int ra = 0, rb = 0;  // tokens are distinct: rank = number of smaller tokens
+  for (int j = 0; j < kBlock; ++j) {
+    const int x = buf[warp][j];
+    ra += x < a;
+    rb += x < b;
+  }
+  __syncwarp();
+  seg[ra] = a;
+  seg[rb] = b;
+  if (ra == 0) mark[bh * (size_t)nv + a] = leaf + 1;
+  if (rb == 0) mark[bh * (size_t)nv + b] = leaf + 1;
+}
+
+// perm lists the leaves by their smallest token: a scan over the marks in token order.
+// One CTA of 1024 threads per head.
+__global__ void __launch_bounds__(1024) leaf_order_kernel(const int32_t* __restrict__ tok,
+                                                          const int32_t* __restrict__ mark, int nv,
+                                                          int32_t* __restrict__ order) {
+  __shared__ int wsum[32];
+  __shared__ int base;
+  const size_t bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) base = 0;
+  __syncthreads();
+  for (int t0 = 0; t0 < nv; t0 += 1024) {
+    const int t = t0 + tid;
+    const int mk = t < nv ? mark[bh * (size_t)nv + t] : 0;
+    const uint32_t bal = __ballot_sync(0xffffffffu, mk != 0);
+    if (lane == 0) wsum[warp] = __popc(bal);
+    __syncthreads();
+    int before = base;
+    for (int q = 0; q < warp; ++q) before += wsum[q];
+    if (mk != 0) order[bh * (size_t)(nv / kBlock) + before + __popc(bal & ((1u << lane) - 1u))] = mk - 1;
+    __syncthreads();
+    if (tid == 0) {
+      int tot = 0;
+      for (int q = 0; q < 32; ++q) tot += wsum[q];
+      base += tot;
+    }
+    __syncthreads();
+  }
+}
+
+// perm[bh][r * 64 + j] = tok[bh][order[r] * 64 + j]. grid (ceil(nv / 256), BH).
+__global__ void __launch_bounds__(kThreads) perm_kernel(const int32_t* __restrict__ tok,
+                                                        const int32_t* __restrict__ order, int nv,
+                                                        int32_t* __restrict__ perm) {
+  const size_t bh = blockIdx.y;
+  const int p = blockIdx.x * kThreads + threadIdx.x;
+  if (p >= nv) return;
+  const int leaf = order[bh * (size_t)(nv / kBlock) + p / kBlock];
+  perm[bh * (size_t)nv + p] = tok[bh * (size_t)nv + (size_t)leaf * kBlock + (p % kBlock)];
+}
+
+// Qp/Kp/Vp rows p < nv come from rows perm[p]; dense rows are copied. 16 bytes per thread.
+template <int D>
+__global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
+                                                          const uint16_t* __restrict__ V, const int32_t* __restrict__ perm,
+                                                          int N, int nv, uint16_t* __restrict__ Qp,
+                                                          uint16_t* __restrict__ Kp, uint16_t* __restrict__ Vp) {
+  constexpr int CH = D / 8;
+  const size_t bh = blockIdx.y;
+  const long long e = (long long)blockIdx.x * kThreads + threadIdx.x;
+  if (e >= (long long)N * CH) return;
+  const int p = (int)(e / CH), c = (int)(e % CH);
+  const int src = p < nv ? perm[bh * (size_t)nv + p] : p;
+  const size_t so = (bh * N + src) * D + c * 8, dof = (bh * N + p) * D + c * 8;
+  *reinterpret_cast<uint4*>(Qp + dof) = ldg_nc_v4(Q + so);
+  *reinterpret_cast<uint4*>(Kp + dof) = ldg_nc_v4(K + so);
+  *reinterpret_cast<uint4*>(Vp + dof) = ldg_nc_v4(V + so);
+}
+
+// ------------------------------------------------------------------ host side
+struct Plan {
+  int levels = 0, first_small = 0;  // levels < first_small use the multi-CTA path
+  int max_large_nodes = 0;
+  std::vector<int> cpn;             // chunks per node at each large level
+  size_t off_macc, off_lmat, off_x, off_tok0, off_tok1, off_proj, off_nacc, off_mark, off_order, total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+inline Plan make_plan(int bh, int nb, int d) {
+  Plan P;
+  const size_t nv = (size_t)nb * kBlock;
+  P.levels = num_levels(nb);
+  P.first_small = P.levels;
+  for (int l = 0; l < P.levels; ++l) {
+    int maxm = 0;
+    for (int c = 0; c < (1 << l); ++c) {
+      int st, m;
+      if (node_of(nb, l, c, &st, &m)) maxm = m > maxm ? m : maxm;
+    }
+    if (maxm <= kSmallBlocks) {
+      P.first_small = l;
+      break;
+    }
+    P.cpn.push_back((maxm * kBlock + kChunkTok - 1) / kChunkTok);
+  }
+  P.max_large_nodes = P.first_small > 0 ? (1 << (P.first_small - 1)) : 0;
+  size_t o = 0;
+  P.off_macc = o;  o = align256(o + (size_t)bh * d * d * 8);
+  P.off_lmat = o;  o = align256(o + (size_t)bh * d * d * 4);
+  P.off_x = o;     o = align256(o + (size_t)bh * nv * d * 4);
+  P.off_tok0 = o;  o = align256(o + (size_t)bh * nv * 4);
+  P.off_tok1 = o;  o = align256(o + (size_t)bh * nv * 4);
+  P.off_proj = o;  o = align256(o + (size_t)bh * nv * 4);
+  P.off_nacc = o;  o = align256(o + (size_t)P.max_large_nodes * bh * ((size_t)d * d + d) * 8);
+  P.off_mark = o;  o = align256(o + (size_t)bh * nv * 4);
+  P.off_order = o; o = align256(o + (size_t)bh * nb * 4);
+  P.total = o;
+  return P;
+}
+
+}  // namespace rb
 
 inline size_t reblock_workspace_bytes(int bh, int nb, int d) {
-  (void)bh; (void)nb; (void)d;
-  return 0;
+  if (nb <= 0) return 0;
+  return rb::make_plan(bh, nb, d).total;
+}
+
+template <int D>
+int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
+                cudaStream_t cs) {
+  using namespace rb;
+  const int nv = nb * kBlock;
+  if (nb > 0) {
+    const Plan P = make_plan(bh, nb, D);
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    double* macc = reinterpret_cast<double*>(w + P.off_macc);
+    float* lmat = reinterpret_cast<float*>(w + P.off_lmat);
+    float* X = reinterpret_cast<float*>(w + P.off_x);
+    int32_t* tok0 = reinterpret_cast<int32_t*>(w + P.off_tok0);
+    int32_t* tok1 = reinterpret_cast<int32_t*>(w + P.off_tok1);
+    float* proj = reinterpret_cast<float*>(w + P.off_proj);
+    double* nacc = reinterpret_cast<double*>(w + P.off_nacc);
+    int32_t* mark = reinterpret_cast<int32_t*>(w + P.off_mark);
+    int32_t* order = reinterpret_cast<int32_t*>(w + P.off_order);
+    const size_t tree_stride = (size_t)(P.levels + 1) * nv;
+
+    if (cudaMemsetAsync(macc, 0, (size_t)bh * D * D * 8, cs) != cudaSuccess) return SPARK_ECUDA;
+    if (cudaMemsetAsync(mark, 0, (size_t)bh * nv * 4, cs) != cudaSuccess) return SPARK_ECUDA;
+    const int smem_km = D * D * 8 + kTile * (D + 4) * 4;
+    cudaFuncSetAttribute(kmoment_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_km);
+    kmoment_kernel<D><<<dim3((nv + kChunkTok - 1) / kChunkTok, bh), kThreads, smem_km, cs>>>(K, N, nv, macc);
+    cudaFuncSetAttribute(cholesky_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, D * D * 8);
+    cholesky_kernel<D><<<bh, kThreads, D * D * 8, cs>>>(macc, nv, lmat);
+    const int smem_wh = D * D * 4 + 64 * (D + 4) * 4;
+    cudaFuncSetAttribute(whiten_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_wh);
+    whiten_kernel<D><<<dim3((nv + 63) / 64, bh), kThreads, smem_wh, cs>>>(Q, N, nv, lmat, X, tok0, tree, tree_stride);
+    SPARK_LAUNCH_CHECK();
+
+    LevelArgs a;
+    a.X = X;
+    a.proj = proj;
+    a.tree = tree;
+    a.nv = nv;
+    a.nb = nb;
+    a.levels = P.levels;
+    const int smem_split = SplitSmem<D>::kBytes;
+    cudaFuncSetAttribute(node_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
+    cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
+    const int smem_nm = (D * D + D) * 8 + kTile * (D + 4) * 4;
+    cudaFuncSetAttribute(node_moments_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_nm);
+    for (int l = 0; l < P.first_small; ++l) {
+      a.level = l;
+      a.tin = (l & 1) ? tok1 : tok0;
+      a.tout = (l & 1) ? tok0 : tok1;
+      const int nodes = 1 << l;
+      if (cudaMemsetAsync(nacc, 0, (size_t)nodes * bh * ((size_t)D * D + D) * 8, cs) != cudaSuccess)
+        return SPARK_ECUDA;
+      node_moments_kernel<D><<<dim3(nodes * P.cpn[l], bh), kThreads, smem_nm, cs>>>(a, P.cpn[l], nacc);
+      node_split_kernel<D><<<dim3(nodes, bh), kThreads, smem_split, cs>>>(a, nacc);
+      SPARK_LAUNCH_CHECK();
+    }
+    if (P.first_small < P.levels) {
+      a.level = P.first_small;
+      subtree_kernel<D><<<dim3(1 << P.first_small, bh), kThreads, smem_split, cs>>>(a, tok0, tok1);
+      SPARK_LAUNCH_CHECK();
+    }
+    int32_t* final_tok = (P.levels & 1) ? tok1 : tok0;
+    leaf_sort_kernel<<<dim3((nb + 7) / 8, bh), kThreads, 0, cs>>>(final_tok, nv, nb, mark);
+    leaf_order_kernel<<<bh, 1024, 0, cs>>>(final_tok, mark, nv, order);
+    perm_kernel<<<dim3((nv + kThreads - 1) / kThreads, bh), kThreads, 0, cs>>>(final_tok, order, nv, perm);
+    SPARK_LAUNCH_CHECK();
+  }
+  const long long chunks = (long long)N * (D / 8);
+  gather_kernel<D><<<dim3((unsigned)((chunks + kThreads - 1) / kThreads), bh), kThreads, 0, cs>>>(
+      Q, K, V, perm, N, nv, Qp, Kp, Vp);
+  SPARK_LAUNCH_CHECK();
+  return SPARK_OK;
 }
 
 inline int reblock_launch(int bh, int N, int nb, int d, const uint16_t* Q, const uint16_t* K,
                           const uint16_t* V, int32_t* perm, uint16_t* Qp, uint16_t* Kp,
                           uint16_t* Vp, int32_t* tree, void* ws, cudaStream_t stream) {
-  (void)bh; (void)N; (void)nb; (void)d; (void)Q; (void)K; (void)V; (void)perm; (void)Qp;
-  (void)Kp; (void)Vp; (void)tree; (void)ws; (void)stream;
-  return SPARK_EUNSUPPORTED;
+  return d == 128 ? reblock_run<128>(bh, N, nb, Q, K, V, perm, Qp, Kp, Vp, tree, ws, stream)
+                  : reblock_run<64>(bh, N, nb, Q, K, V, perm, Qp, Kp, Vp, tree, ws, stream);
 }
 
 }  // namespace spark

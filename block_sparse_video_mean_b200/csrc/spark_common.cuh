@@ -11,6 +11,8 @@
 namespace spark {
 
 constexpr int kBlock = 64;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // First device-side fault of any kernel (0 = none). Read and cleared by spark_device_error.
 // The library is one translation unit (spark_lib.cu includes every kernel header), so

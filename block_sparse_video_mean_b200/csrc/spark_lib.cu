@@ -10,7 +10,6 @@
 #include "spark_common.cuh"
 #include "pool.cuh"
 #include "select.cuh"
-#include "attn_mma.cuh"
 #include "attn_tc.cuh"
 #include "reblock.cuh"
 

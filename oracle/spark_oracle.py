@@ -261,12 +261,16 @@ def key_second_moment(k_video) -> np.ndarray:
 def whiten(q_video, M) -> np.ndarray:
     """Unit vectors x_i = L^T q_i / |L^T q_i| with M = L L^T, so x_i . x_j is the
     Mahalanobis cosine q_i^T M q_j / (|q_i|_M |q_j|_M) ([Spark-H3] Spark-Reblock bullet).
-    A query with zero M-norm maps to the zero vector."""
+    A query with zero M-norm maps to the zero vector. When M is not positive definite the
+    factor of M + 1e-6 tr(M)/d I is used, and the identity when that fails too."""
     d = M.shape[0]
     try:
         L = np.linalg.cholesky(M)
     except np.linalg.LinAlgError:
-        L = np.linalg.cholesky(M + 1e-6 * np.trace(M) / d * np.eye(d))
+        try:
+            L = np.linalg.cholesky(M + 1e-6 * np.trace(M) / d * np.eye(d))
+        except np.linalg.LinAlgError:
+            L = np.eye(d)   # degenerate keys (e.g. all zero): plain cosine
     x = q_video @ L
     nrm = np.linalg.norm(x, axis=1, keepdims=True)
     return np.divide(x, nrm, out=np.zeros_like(x), where=nrm > 0)
@@ -374,7 +378,7 @@ def apply_perm(x, perm, n_sink, block=BLOCK):
 
 def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale=None,
                  block=BLOCK, reblock=False, qblocks=None, sel_override=None,
-                 pool_mode="reweight"):
+                 pool_mode="reweight", perm_override=None):
     """The whole forward of one head, in the original token order.
 
     Returns (O [N, d], LSE [N], info) where info holds the selection lists, the pooled
@@ -386,7 +390,10 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
     scale = default_scale(d, scale)
     info = {}
     if reblock:
-        rb = reblock_head(q, k, n_sink, block)
+        if perm_override is not None:
+            rb = ReblockResult(np.asarray(perm_override, dtype=np.int64), None, {})
+        else:
+            rb = reblock_head(q, k, n_sink, block)
         info["reblock"] = rb
         qp, kp, vp = (apply_perm(t, rb.perm, n_sink, block) for t in (q, k, v))
     else:

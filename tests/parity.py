@@ -66,3 +66,55 @@ def check_lse(l, r, what=""):
 
 def default_scale(d):
     return 1.0 / math.sqrt(d)
+
+
+GAP_TIE = 1e-4      # relative eigengap below which a node's direction is ill-defined
+SKEW_TIE = 1e-6     # |third moment| / sigma^3 below which the sign of v is ambiguous
+
+
+def replay_reblock_tree(x, tree, levels, nodes=None):
+    """Node replay: for every node of the device's tree (its token set given by the labels
+    at `level`, split into the labels 2c / 2c + 1 at level + 1) the oracle recomputes the
+    split in fp64 from the same membership. Returns (n_checked, n_skipped_as_ties); raises
+    AssertionError on a disagreement outside the tie windows. `nodes` limits the check to
+    a list of (level, label)."""
+    checked = skipped = 0
+    todo = nodes
+    if todo is None:
+        todo = [(lev, int(c)) for lev in range(levels) for c in np.unique(tree[lev])]
+    for lev, c in todo:
+        members = np.nonzero(tree[lev] == c)[0]
+        if members.size <= 64:
+            continue
+        left_dev = set(np.nonzero(tree[lev + 1][members] == 2 * c)[0].tolist())
+        left_dev = set(members[list(left_dev)].tolist())
+        assert len(left_dev) == (members.size // 64 // 2) * 64, (lev, c, len(left_dev))
+        sp = orc.split_node(x, members)
+        if sp.gap < GAP_TIE:
+            skipped += 1
+            continue
+        cut = len(left_dev)
+        cands = [(set(sp.left.tolist()), 1.0, sp.split_value)]
+        if abs(sp.skew) < SKEW_TIE:
+            # the other orientation: the lowest projections after flipping the sign
+            pf = -np.array([sp.proj[t] for t in members.tolist()])
+            order = np.lexsort((members, pf))
+            split_f = 0.5 * (pf[order[cut - 1]] + pf[order[cut]])
+            cands.append((set(members[order[:cut]].tolist()), -1.0, split_f))
+        ok = False
+        for cand, sg, split in cands:
+            diff = cand ^ left_dev
+            if all(abs(sg * sp.proj[t] - split) < TIE for t in diff):
+                ok = True
+                break
+        assert ok, (lev, c, len(cands[0][0] ^ left_dev))
+        checked += 1
+    return checked, skipped
+
+
+def check_partition(perm, nv):
+    perm = np.asarray(perm)
+    assert sorted(perm.tolist()) == list(range(nv))
+    leaves = perm.reshape(-1, 64)
+    assert np.all(np.diff(leaves, axis=1) > 0)
+    assert np.all(np.diff(leaves[:, 0]) > 0)
