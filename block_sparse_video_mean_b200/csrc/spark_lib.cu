@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "spark_common.cuh"
 #include "pool.cuh"
@@ -120,6 +121,29 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
     return SPARK_ECUDA;
   attn_tc_kernel<D><<<grid, C::kThreads, smem, cs>>>(maps, tp);
   SPARK_LAUNCH_CHECK();
+  return SPARK_OK;
+}
+
+// Scratch of spark_score_select_noalloc: a file-scope device array (no allocation). In
+// host code its name is only a stand-in, so its device address is looked up per device.
+__device__ __align__(256) double g_noalloc_select_scratch[2 * SPARK_NOALLOC_MAX_HEADS];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[128] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPARK_ECUDA;
+  if (dev < 0 || dev >= 128) return SPARK_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_select_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return SPARK_ECUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
   return SPARK_OK;
 }
 
@@ -265,6 +289,19 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
   return SPARK_OK;
 }
 
+int spark_score_select_noalloc(const spark_shape* s, const float* q_pool, const float* k_pool,
+                               int mode, double param, int32_t kcap, int32_t* idx, int32_t* cnt,
+                               void* stream) {
+  int st = check_shape(s);
+  if (st != SPARK_OK) return st;
+  if ((int64_t)s->B * s->H > SPARK_NOALLOC_MAX_HEADS) return SPARK_ESCRATCH;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != SPARK_OK) return st;
+  return spark_score_select(s, q_pool, k_pool, mode, param, kcap, idx, cnt, scratch,
+                            sizeof(g_noalloc_select_scratch), stream);
+}
+
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
                    const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,
@@ -351,6 +388,7 @@ const char* spark_strerror(int status) {
     case SPARK_ETIMEOUT: return "device: a bounded wait gave up";
     case SPARK_EDEVICE_INDEX: return "device: block index or count out of range (skipped)";
     case SPARK_ECAPACITY: return "device: more blocks kept than kcap (row truncated)";
+    case SPARK_ESCRATCH: return "B*H exceeds the static scratch of spark_score_select_noalloc";
     default: return "unknown status";
   }
 }

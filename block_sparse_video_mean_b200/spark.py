@@ -28,7 +28,8 @@ BLOCK = 64
 
 EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
            "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
-           "spark_strerror")
+           "spark_strerror", "spark_score_select_noalloc")
+NOALLOC_MAX_HEADS = 4096
 
 
 class SparkError(RuntimeError):
@@ -67,6 +68,8 @@ def load() -> ctypes.CDLL:
     lib.spark_pool_kv.restype = I
     lib.spark_score_select.argtypes = [SP, P, P, I, D, ctypes.c_int32, P, P, P, Z, P]
     lib.spark_score_select.restype = I
+    lib.spark_score_select_noalloc.argtypes = [SP, P, P, I, D, ctypes.c_int32, P, P, P]
+    lib.spark_score_select_noalloc.restype = I
     lib.spark_attn_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_int32, P, P, P, P, P, P, Z, P]
     lib.spark_attn_fwd.restype = I
     lib.spark_reblock.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
@@ -171,6 +174,24 @@ def score_select(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, 
                                      float(param), int(kcap), _ptr(idx), _ptr(cnt), _ptr(ws),
                                      0 if ws is None else ws.numel(), _stream(dev)),
            "spark_score_select")
+    return idx, cnt
+
+
+def score_select_noalloc(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, out=None):
+    """spark_score_select_noalloc: the selection without a scratch argument (the library
+    uses its own fixed device array); returns (idx, cnt) like score_select."""
+    B, H, nb, d = q_pool.shape
+    shape = make_shape(B, H, N, d, n_sink, scale)
+    dev = q_pool.device
+    if kcap is None:
+        kcap = topk_count(param, nb) if mode == SELECT_TOPK_RATIO else max(nb, 1)
+    if out is None:
+        out = (torch.empty((B, H, nb, max(kcap, 1)), dtype=torch.int32, device=dev),
+               torch.empty((B, H, nb), dtype=torch.int32, device=dev))
+    idx, cnt = out
+    _check(load().spark_score_select_noalloc(ctypes.byref(shape), _ptr(q_pool), _ptr(k_pool),
+                                             int(mode), float(param), int(kcap), _ptr(idx),
+                                             _ptr(cnt), _stream(dev)), "spark_score_select_noalloc")
     return idx, cnt
 
 

@@ -21,7 +21,8 @@
  *   pooled, scored, compressed or reblocked.
  * - block must be 64; d must be 64 or 128; scale <= 0 means 1/sqrt(d).
  * - Every pointer is a device pointer owned by the caller; the library allocates
- *   nothing, keeps no state beyond one device-side error word, and never
+ *   nothing, keeps no state beyond one device-side error word (and the fixed scratch
+ *   array of spark_score_select_noalloc), and never
  *   synchronises except in spark_device_error. Calls are asynchronous on `stream`
  *   (a cudaStream_t, NULL = legacy default stream) and re-entrant.
  * - Return value: SPARK_OK, or a negative status for arguments rejected on the host
@@ -47,6 +48,7 @@ extern "C" {
 #define SPARK_ETIMEOUT (-4)      /* device: a bounded wait gave up */
 #define SPARK_EDEVICE_INDEX (-5) /* device: a selected block index was out of range */
 #define SPARK_ECAPACITY (-6)     /* device: tau kept more blocks than kcap; list truncated */
+#define SPARK_ESCRATCH (-7)      /* B*H beyond the static scratch of spark_score_select_noalloc */
 
 #define SPARK_SELECT_TOPK_RATIO 0
 #define SPARK_SELECT_TAU 1
@@ -149,6 +151,28 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
 int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                   int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
                   size_t ws_bytes, void* stream);
+
+/* spark_score_select without a scratch argument, for callers that cannot allocate device
+ * memory of their own (the paper has no counterpart; this is a library convenience).
+ * Some hosts own every byte of device memory up front - an engine that hands out one
+ * arena at start-up, a plugin running inside another framework's allocator, a real-time
+ * loop that must never reach the driver's allocator - and so cannot provide the tau-mode
+ * moment scratch that spark_score_select asks for. This entry point uses a file-scope
+ * device array of SPARK_NOALLOC_MAX_HEADS * 2 doubles (64 KiB, held by every GPU that
+ * loads the library until the process exits) instead, and otherwise runs exactly the
+ * spark_score_select path with the same arguments and outputs.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - B*H above SPARK_NOALLOC_MAX_HEADS returns SPARK_ESCRATCH before any launch.
+ * - The first call on a device looks the array's device address up (cudaGetSymbolAddress,
+ *   with that device current) and caches it; make that first call before any stream
+ *   capture on the device.
+ * - Every call shares the one array: calls whose work overlaps on the GPU (different
+ *   streams, or different host threads without ordering) race on it. The part that must
+ *   start at zero is cleared by each call. */
+#define SPARK_NOALLOC_MAX_HEADS 4096
+int spark_score_select_noalloc(const spark_shape* s, const float* q_pool, const float* k_pool,
+                               int mode, double param, int32_t kcap, int32_t* idx, int32_t* cnt,
+                               void* stream);
 
 /* Reads the device error word into *host_word (may be NULL) and clears it; synchronises
  * `stream`. Returns SPARK_OK or SPARK_ECUDA when the copy itself failed. */
