@@ -40,6 +40,8 @@
 #define SPARK_TC_T0(v)
 #define SPARK_TC_ACC(slot, v)
 #define SPARK_TC_EV(who, what)
+#define SPARK_TC_DECL
+#define SPARK_TC_FLUSH
 #endif
 
 namespace spark {
@@ -124,6 +126,12 @@ struct TcSlotWalk {
   }
 };
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -176,6 +184,7 @@ __global__ void __launch_bounds__(352, 1)
   const int nbw = (p.nb + 31) / 32;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  SPARK_TC_DECL
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       tc::mbar_init(&kfull[i], 1);
@@ -618,35 +627,49 @@ __global__ void __launch_bounds__(352, 1)
           j0 = (hi - I.cnt - n_dk) * kBlock;
           valid = min(kBlock, p.nb - j0);
         }
+        // Exact halves keep raw scores (the scale is folded into the exponent's FFMA);
+        // pooled halves become scale*logit + beta (base 2), with the selected blocks and
+        // entries past nb masked. The half's bias values are loaded up front, unconditionally
+        // (clamped index), so their latencies overlap.
         if (kind == 0) {
-          if (valid >= kBlock) {
+          if (valid < kBlock) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] *= p.scale_log2;
-          } else {
-#pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] = (j < valid) ? x[j] * p.scale_log2 : -INFINITY;
+            for (int j = 0; j < 64; ++j)
+              if (j >= valid) x[j] = -INFINITY;
           }
         } else {
           const float* bp = p.beta + (size_t)I.bh * p.nb;
+          const int wb = j0 >> 5;  // j0 is a multiple of 64
+          const uint32_t w0 = bm[wb];
+          const uint32_t w1 = (j0 + 32 < p.nb) ? bm[wb + 1] : 0u;
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const int jj = min(j0 + j, p.nb - 1);
-            const bool m = (j >= valid) || ((bm[jj >> 5] >> (jj & 31)) & 1u);
-            x[j] = m ? -INFINITY : fmaf(x[j], p.scale_log2, bp[jj] * kLog2e);
+          for (int q = 0; q < 4; ++q) {
+            float bv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) bv[j] = __ldg(bp + min(j0 + 16 * q + j, p.nb - 1));
+            const uint32_t wm = (q < 2 ? w0 : w1) >> (16 * (q & 1));
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const bool m = (16 * q + j >= valid) || ((wm >> j) & 1u);
+              x[16 * q + j] = m ? -INFINITY : fmaf(x[16 * q + j], p.scale_log2, bv[j] * kLog2e);
+            }
           }
         }
-        // row max: tree over this thread's 64 keys, then the partner half
+        const float xs = kind == 0 ? p.scale_log2 : 1.0f;  // factor still to apply to x
+        SPARK_TC_ACC(14 + kind, t_cp);
+        SPARK_TC_T0(t_mx);
+        // row max: 3-input max tree over this thread's 64 keys, then the partner half
         float mx;
         {
-          float t8[8];
+          float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];  // four independent chains
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a0 = fmaxf(x[i], x[i + 8]), a1 = fmaxf(x[i + 16], x[i + 24]);
-            const float a2 = fmaxf(x[i + 32], x[i + 40]), a3 = fmaxf(x[i + 48], x[i + 56]);
-            t8[i] = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          for (int i = 4; i < 64; i += 8) {
+            a0 = max3f(a0, x[i], x[i + 1]);
+            a1 = max3f(a1, x[i + 2], x[i + 3]);
+            a2 = max3f(a2, x[i + 4], x[i + 5]);
+            a3 = max3f(a3, x[i + 6], x[i + 7]);
           }
-          mx = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
-                     fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+          mx = max3f(max3f(a0, a1, a2), a3, a3) * xs;
         }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run, mx);
@@ -673,17 +696,20 @@ __global__ void __launch_bounds__(352, 1)
           l_run *= alpha;
           m_run = m_new;
         }
+        SPARK_TC_ACC(16, t_mx);
+        SPARK_TC_T0(t_ex);
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         uint32_t pk[32];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2f(x[2 * j] - m_use);
-          const float p1 = ex2f(x[2 * j + 1] - m_use);
+          const float p0 = ex2f(fmaf(x[2 * j], xs, -m_use));
+          const float p1 = ex2f(fmaf(x[2 * j + 1], xs, -m_use));
           ls[j & 3] += p0 + p1;
           pk[j] = pack_bf16x2(p0, p1);
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        SPARK_TC_ACC(17, t_ex);
         SPARK_TC_ACC(7, t_cp);
         SPARK_TC_T0(t_st);
         // P over S: packed columns 32h .. 32h+31 of the buffer
@@ -705,6 +731,7 @@ __global__ void __launch_bounds__(352, 1)
     }
   }
 
+  SPARK_TC_FLUSH
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
