@@ -1,9 +1,15 @@
-"""Benchmark: block-sparse video attention forward on the 1152x640, 243-frame clip shape.
+"""Benchmark: block-sparse video attention forward.
 
-One step = one whole forward through the C ABI (pool + score/select + exact+compressed
-attention) of B=1, H=24, d=128, 175,680 video tokens (61 x 72 x 40) + 512 sink rows at
-top-k 10% with the Spark-Reweight compressed branch, inputs resident in HBM. Inputs are
+Default workload (the headline line): the 1152x640, 243-frame clip shape — B=1, H=24,
+d=128, 61 x 72 x 40 = 175,680 video tokens + 512 sink rows, 64-token blocks, top-k 10%,
+exact + Spark-Reweight compressed branch, bf16 in/out. One step = one whole forward
+through the C ABI (pool + score/select + attention), inputs resident in HBM; inputs are
 3.2 GB, larger than the 126 MB L2, so no flush is needed between steps.
+
+Other workloads (``--workload``) time the remaining configurations the same way: the 32k
+exact-only call, the tau-threshold selection, the full-density run and the 1344x768,
+240-frame Spark-Reblock forward (reblock included in the step). ``--heads`` shrinks a
+workload for profiling.
 
 Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling); the
 only collectives are the timing barrier and the max-over-ranks of the elapsed time.
@@ -22,26 +28,62 @@ import subprocess
 import sys
 import tempfile
 import time
+from dataclasses import dataclass
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ms/call & dense-equiv TFLOP/s of sparse attn fwd at 10% density, N=175,680"
-B, H, NV, NS, D = 1, 24, 175680, 512, 128
-N = NV + NS
-RATIO = 0.1
-WORKLOAD = ("1152x640 243-frame clip: B=1 H=24 d=128, 61x72x40=175680 video tokens + 512 sink "
-            "rows, 64-token blocks, top-k 10%, exact + Spark-Reweight compressed branch, bf16 in/out")
 
 
-def flop_counts(nb, k, ns=NS, d=D, h=H, b=B):
-    """Algorithmic FLOPs of one forward (4*d per query-key pair: QK^T and PV)."""
+@dataclass
+class Workload:
+    name: str
+    desc: str
+    H: int
+    nv: int
+    ns: int
+    mode: str = "topk"
+    param: float = 0.1
+    compressed: bool = True
+    reblock: bool = False
+    B: int = 1
+    d: int = 128
+
+
+WORKLOADS = {w.name: w for w in [
+    Workload("1152x640x243", "1152x640 243-frame clip: B=1 H=24 d=128, 61x72x40=175680 video tokens "
+             "+ 512 sink rows, 64-token blocks, top-k 10%, exact + Spark-Reweight compressed branch, "
+             "bf16 in/out", 24, 175680, 512),
+    Workload("1152x640x243-top20", "as 1152x640x243 at top-k 20%", 24, 175680, 512, param=0.2),
+    Workload("1152x640x243-top30", "as 1152x640x243 at top-k 30%", 24, 175680, 512, param=0.3),
+    Workload("1152x640x243-tau1.0", "as 1152x640x243 with the per-head threshold tau=1.0",
+             24, 175680, 512, mode="tau", param=1.0),
+    Workload("1152x640x243-tau1.5", "as 1152x640x243 with tau=1.5", 24, 175680, 512, mode="tau", param=1.5),
+    Workload("1152x640x243-tau2.0", "as 1152x640x243 with tau=2.0", 24, 175680, 512, mode="tau", param=2.0),
+    Workload("1152x640x243-dense", "as 1152x640x243 at 100% density, compressed branch off",
+             24, 175680, 512, param=1.0, compressed=False),
+    Workload("32k-exact", "single call: B=1 H=24 d=128, 32768 video tokens + 512 text sink rows, "
+             "top-k 10%, exact branch only", 24, 32768, 512, compressed=False),
+    Workload("1344x768x240-reblock", "1344x768 240-frame clip: B=1 H=24 d=128, 61x84x48=245952 video "
+             "tokens + 512 sink rows, Spark-Reblock partition, top-k 10%, exact + compressed; "
+             "the step includes the reblock", 24, 245952, 512, reblock=True),
+]}
+DEFAULT = "1152x640x243"
+
+
+def flop_counts(w: Workload, nb: int, kept_blocks: int, h=None):
+    """Algorithmic FLOPs of one forward (4*d per query-key pair: QK^T and PV).
+
+    kept_blocks = total selected (query block, key block) pairs over all heads."""
+    h = w.H if h is None else h
     nv = nb * 64
-    n = nv + ns
-    exact = b * h * nb * k * 4 * 64 * 64 * d
-    sink_keys = b * h * nv * ns * 4 * d          # video queries x dense keys
-    sink_queries = b * h * ns * n * 4 * d        # dense queries x all keys
-    compressed = b * h * nv * (nb - k) * 4 * d   # video queries x unselected pooled entries
+    n = nv + w.ns
+    d, b = w.d, w.B
+    exact = kept_blocks * 4 * 64 * 64 * d
+    sink_keys = b * h * nv * w.ns * 4 * d          # video queries x dense keys
+    sink_queries = b * h * w.ns * n * 4 * d        # dense queries x all keys
+    compressed = (b * h * nb * nb - kept_blocks) * 64 * 4 * d if w.compressed else 0
     dense_equiv = 4 * b * h * n * n * d
     return dict(exact=exact, sink=sink_keys + sink_queries, compressed=compressed,
                 selected=exact + sink_keys + sink_queries,
@@ -56,6 +98,12 @@ def load_peaks():
         return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# DRAM bytes (read + write) of one attention launch at the default workload, from
+# `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` (summary under profiles/);
+# None once the kernel has changed since it was measured.
+ATTN_TRAFFIC_BYTES = None
 
 
 class ClockSampler:
@@ -120,9 +168,22 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+def phase_bytes(w: Workload, h: int, nb: int, kept_blocks: int, kcap: int):
+    """Algorithmic HBM bytes of the bandwidth-bound calls (each input read once, each
+    output written once)."""
+    bh = w.B * h
+    nv = nb * 64
+    n = nv + w.ns
+    row = w.d * 2
+    pool = 3 * bh * nv * row + 3 * bh * nb * w.d * 4 + bh * nb * 4 + 2 * bh * nb * w.d * 2 + bh * w.d * 4
+    select = 2 * bh * nb * w.d * 4 + kept_blocks * 4 + bh * nb * 4
+    gather = 6 * bh * n * row + bh * nv * 4          # permute Q,K,V (read + write) + perm
+    return dict(pool=pool, select=select, reblock_gather=gather)
+
+
 # --------------------------------------------------------------------------- GPU arm
 
-def run_gpu(args, rank, world, local_rank):
+def run_gpu(args, w: Workload, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
@@ -132,61 +193,55 @@ def run_gpu(args, rank, world, local_rank):
     spark.load()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    Q, K, V = make_qkv(B, H, NV, NS, D, seed=args.seed + rank, device=dev)
-    cfg = spark.ForwardConfig("topk", RATIO, True)
-    plan = spark.SparkAttention(B, H, N, D, NS, cfg, dev)
-    nb, k = plan.nb, plan.kcap
-    fl = flop_counts(nb, k)
+    h = args.heads or w.H
+    N = w.nv + w.ns
+    Q, K, V = make_qkv(w.B, h, w.nv, w.ns, w.d, seed=args.seed + rank, device=dev)
+    cfg = spark.ForwardConfig(w.mode, w.param, w.compressed, reblock=w.reblock)
+    plan = spark.SparkAttention(w.B, h, N, w.d, w.ns, cfg, dev)
+    nb = plan.nb
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        return plan.run(Q, K, V)
-
     for _ in range(args.warmup):
-        step()
+        plan.run(Q, K, V)
     torch.cuda.synchronize(dev)
     err = spark.device_error(dev)
     if err != 0:
         raise RuntimeError(f"device error {err} ({spark.strerror(err)})")
+    kept = int(plan.cnt.to(torch.int64).sum().item()) if nb > 0 else 0
+    fl = flop_counts(w, nb, kept, h)
+    by = phase_bytes(w, h, nb, kept, plan.kcap)
 
-    # per-kernel timing of the dominant kernel (the attention launch), same stream
-    attn_ev = []
-
-    def step_timed():
-        perm = None
-        spark.pool_kv(Q, K, V, NS, spark.POOL_REWEIGHT, None, out=plan.pool)
-        spark.score_select(plan.pool["q_pool"], plan.pool["k_pool"], NS, N, plan.mode, RATIO,
-                           plan.kcap, None, out=(plan.idx, plan.cnt), ws=plan.sel_ws)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        spark.attn_fwd(Q, K, V, plan.idx, plan.cnt, NS, pack=plan.pool["pack"],
-                       beta=plan.pool["beta"], perm=perm, out=(plan.O, plan.lse))
-        e1.record(stream)
-        attn_ev.append((e0, e1))
-
+    ev = []
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    launches0 = spark.kernel_launches()
     with ClockSampler(local_rank) as clk:
         t0.record(stream)
         for _ in range(args.steps):
-            step_timed()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            plan.run(Q, K, V, events=e)
+            ev.append(e)
         t1.record(stream)
         torch.cuda.synchronize(dev)
+    launches = spark.kernel_launches() - launches0
     if world > 1:
         dist.barrier()
+    err = spark.device_error(dev)
+    if err != 0:
+        raise RuntimeError(f"device error {err} ({spark.strerror(err)})")
     ms = t0.elapsed_time(t1)
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    phase_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev)
+                for i, name in enumerate(("reblock", "pool", "select", "attn"))}
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     ms_step = ms / args.steps
 
-    # end to end through the same calls with pinned host buffers
+    # end to end through the same public call with pinned host buffers
     hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
     hO = torch.empty(plan.O.shape, dtype=plan.O.dtype).pin_memory()
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
@@ -217,17 +272,37 @@ def run_gpu(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_ms /= e2e_steps
+    del dQ, dK, dV
 
     if rank != 0:
         return None
     hbm, bf16_peak, bf16_sust, peak_src = load_peaks()
+    attn_ms = phase_ms["attn"]
     achieved = fl["attn_total"] / (attn_ms * 1e-3) / 1e12
     value = world * fl["dense_equiv"] / (ms_step * 1e-3) / 1e12
     clocks = clk.summary()
+    default = (w.name == DEFAULT and h == w.H)
+
+    def gbs(nbytes, t_ms):
+        return round(nbytes / (t_ms * 1e-3) / 1e9, 1) if t_ms > 0 else None
+    phases = {
+        "pool": {"ms": round(phase_ms["pool"], 3), "bytes": by["pool"],
+                 "GB/s": gbs(by["pool"], phase_ms["pool"]),
+                 "frac_hbm": round(by["pool"] / (phase_ms["pool"] * 1e-3) / 1e9 / hbm, 3)},
+        "select": {"ms": round(phase_ms["select"], 3), "bytes": by["select"],
+                   "GB/s": gbs(by["select"], phase_ms["select"]),
+                   "score_flops": 2 * w.B * h * nb * nb * w.d},
+        "attn": {"ms": round(attn_ms, 3), "selected_flops": fl["selected"],
+                 "compressed_flops": fl["compressed"]},
+    }
+    if w.reblock:
+        phases["reblock"] = {"ms": round(phase_ms["reblock"], 3),
+                             "gather_bytes": by["reblock_gather"]}
     line = {
-        "metric": METRIC,
+        "metric": METRIC if w.name == DEFAULT else
+        f"ms/call & dense-equiv TFLOP/s of sparse attn fwd, workload {w.name}",
         "value": round(value, 2),
-        "unit": "TFLOP/s dense-equivalent (4*B*H*N^2*d / time, N=176,192)",
+        "unit": f"TFLOP/s dense-equivalent (4*B*H*N^2*d / time, N={N:,})",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -237,54 +312,61 @@ def run_gpu(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded block-correlated N(0,1) Q/K/V, generated on the device)",
-        "config": {"workload": WORKLOAD, "global_batch": world * B, "heads": H, "seq_len": N,
-                   "head_dim": D, "kept_blocks_per_query_block": k, "video_blocks": nb,
+        "config": {"workload": w.name, "desc": w.desc, "global_batch": world * w.B, "heads": h,
+                   "seq_len": N, "head_dim": w.d, "select": f"{w.mode} {w.param}",
+                   "compressed": w.compressed, "reblock": w.reblock, "video_blocks": nb,
+                   "kept_blocks_mean_per_query_block": round(kept / max(w.B * h * nb, 1), 2),
                    "parallelism": f"independent problem per GPU x{world}",
-                   "l2": "inputs 3.2 GB > 126 MB L2; no flush needed"},
+                   "l2": f"inputs {3 * Q.numel() * 2 / 1e9:.2f} GB "
+                         + ("> 126 MB L2; no flush needed" if 3 * Q.numel() * 2 > 126e6
+                            else "(< L2: reduced profiling case)")},
         "selected_tflops": round(fl["selected"] / (ms_step * 1e-3) / 1e12, 2),
-        "attn_kernel_ms": round(attn_ms, 3),
-        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel<128>",
+        "phases": phases,
+        "roofline": {"bound": "tensor", "kernel": f"attn_tc_kernel<{w.d}>",
                      "achieved": round(achieved, 2), "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / bf16_peak, 4),
                      "peak_source": f"{peak_src} bf16 burst (sustained {bf16_sust})",
-                     "algorithmic_flops_per_launch": fl["attn_total"], "traffic": None},
+                     "algorithmic_flops_per_launch": fl["attn_total"],
+                     "traffic": ATTN_TRAFFIC_BYTES if default else None},
         "e2e": {"value": round(world * fl["dense_equiv"] / (e2e_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s dense-equivalent, host buffers, copies inside the timed region",
                 "ms_per_step": round(e2e_ms, 3),
                 "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                 "d2h_bytes_per_step": plan.O.numel() * plan.O.element_size()},
-        "gpu_launches": args.steps * 5,
+        "gpu_launches": launches,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(Q[:, :1].cpu(), K[:, :1].cpu(), V[:, :1].cpu(),
+        line["cpu_baseline"] = cpu_baseline(w, Q[:, :1].cpu(), K[:, :1].cpu(), V[:, :1].cpu(),
                                             args.cpu_blocks or 200)
     return line
 
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(Qc, Kc, Vc, n_blocks, seed=0):
-    """The fp64 oracle, as it stands, on one head: pooling of all blocks, scores and top-k
-    of n_blocks sampled query blocks, and their exact + compressed attention. Reported as
-    dense-equivalent TFLOP/s of the sampled query rows (their share of 4*N^2*d)."""
+def cpu_baseline(w: Workload, Qc, Kc, Vc, n_blocks, seed=0):
+    """The fp64 oracle, as it stands, on one head: pooling of all blocks, scores and
+    selection of n_blocks sampled query blocks, and their exact (+ compressed) attention.
+    Reported as dense-equivalent TFLOP/s of the sampled query rows (their share of
+    4*N^2*d). The reblock stage is not part of the sample."""
     import numpy as np
 
     import oracle.spark_oracle as orc
 
     t_start = time.perf_counter()
     q, k, v = (orc.to_f64(t[0, 0]) for t in (Qc, Kc, Vc))
-    scale = 1.0 / math.sqrt(D)
-    P = orc.pool_head(q, k, v, NS, scale)
+    n = q.shape[0]
+    scale = 1.0 / math.sqrt(w.d)
+    P = orc.pool_head(q, k, v, w.ns, scale)
     nb = P.qbar.shape[0]
     rng = np.random.default_rng(seed)
-    blocks = rng.choice(nb, n_blocks, replace=False)
-    sel = orc.select_head(P.qbar, P.kbar, scale, "topk", RATIO, blocks)
+    blocks = rng.choice(nb, min(n_blocks, nb), replace=False)
+    sel = orc.select_head(P.qbar, P.kbar, scale, w.mode, w.param, blocks)
     for t, i in enumerate(blocks):
-        orc.attn_video_block(q, k, v, NS, i, sel[t], P, scale)
+        orc.attn_video_block(q, k, v, w.ns, i, sel[t], P if w.compressed else None, scale)
     dt = time.perf_counter() - t_start
-    rows = n_blocks * 64
-    flops = 4.0 * rows * N * D
+    rows = len(blocks) * 64
+    flops = 4.0 * rows * n * w.d
     threads = None
     try:
         from threadpoolctl import threadpool_info
@@ -293,22 +375,21 @@ def cpu_baseline(Qc, Kc, Vc, n_blocks, seed=0):
         pass
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s dense-equivalent",
             "cores": threads or os.cpu_count(), "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"1 of {H} heads: pooling of all {nb} blocks, top-k of {n_blocks} random "
-                      f"query blocks and their exact+compressed attention ({rows} query rows)"}
+            "sample": f"1 of {w.H} heads: pooling of all {nb} blocks, {w.mode} {w.param} selection "
+                      f"of {len(blocks)} random query blocks and their attention ({rows} query rows)"}
 
 
-def run_reference(args, rank, world):
+def run_reference(args, w: Workload, rank, world):
     if rank != 0:
         return None
-    import torch
     from block_sparse_video_mean_b200.inputs import make_qkv
 
     # one head of the workload, drawn on the host
-    Q, K, V = make_qkv(1, 1, NV, NS, D, seed=args.seed, device="cpu")
+    Q, K, V = make_qkv(1, 1, w.nv, w.ns, w.d, seed=args.seed, device="cpu")
     vals = []
     info = None
     for i in range(args.warmup + args.steps):
-        info = cpu_baseline(Q, K, V, args.cpu_blocks or 64, seed=i)
+        info = cpu_baseline(w, Q, K, V, args.cpu_blocks or 64, seed=i)
         if i >= args.warmup:
             vals.append(info)
     value = statistics.mean(v["value"] for v in vals)
@@ -316,12 +397,14 @@ def run_reference(args, rank, world):
     cb = dict(info)
     cb["value"] = round(value, 6)
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6),
+        "impl": "reference", "metric": METRIC if w.name == DEFAULT else
+        f"ms/call & dense-equiv TFLOP/s of sparse attn fwd, workload {w.name}",
+        "value": round(value, 6),
         "unit": "TFLOP/s dense-equivalent", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded block-correlated N(0,1) Q/K/V, one head drawn on the host)",
-        "config": {"workload": WORKLOAD, "sample": info["sample"]},
+        "config": {"workload": w.name, "sample": info["sample"]},
         "cpu_baseline": cb,
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s dense-equivalent",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -335,6 +418,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="spark", choices=["spark", "reference"])
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (smaller profiling cases)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-blocks", type=int, default=0,
                     help="query blocks in the oracle sample (default: 200 for cpu_baseline, 64 per reference step)")
@@ -342,12 +428,13 @@ def main():
     args = ap.parse_args()
     if args.impl == "spark" and args.warmup < 3:
         args.warmup = 3
+    w = WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        line = run_reference(args, rank, world)
+        line = run_reference(args, w, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
@@ -362,7 +449,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
         pg = True
     try:
-        line = run_gpu(args, rank, world, local_rank)
+        line = run_gpu(args, w, rank, world, local_rank)
         if line is not None:
             print(json.dumps(line), flush=True)
     finally:

@@ -963,6 +963,7 @@ int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, con
     cudaFuncSetAttribute(whiten_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_wh);
     whiten_kernel<D><<<dim3((nv + 63) / 64, bh), kThreads, smem_wh, cs>>>(Q, N, nv, lmat, X, tok0, tree, tree_stride);
     SPARK_LAUNCH_CHECK();
+    note_launches(3);
 
     LevelArgs a;
     a.X = X;
@@ -986,22 +987,26 @@ int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, con
       node_moments_kernel<D><<<dim3(nodes * P.cpn[l], bh), kThreads, smem_nm, cs>>>(a, P.cpn[l], nacc);
       node_split_kernel<D><<<dim3(nodes, bh), kThreads, smem_split, cs>>>(a, nacc);
       SPARK_LAUNCH_CHECK();
+      note_launches(2);
     }
     if (P.first_small < P.levels) {
       a.level = P.first_small;
       subtree_kernel<D><<<dim3(1 << P.first_small, bh), kThreads, smem_split, cs>>>(a, tok0, tok1);
       SPARK_LAUNCH_CHECK();
+      note_launches(1);
     }
     int32_t* final_tok = (P.levels & 1) ? tok1 : tok0;
     leaf_sort_kernel<<<dim3((nb + 7) / 8, bh), kThreads, 0, cs>>>(final_tok, nv, nb, mark);
     leaf_order_kernel<<<bh, 1024, 0, cs>>>(final_tok, mark, nv, order);
     perm_kernel<<<dim3((nv + kThreads - 1) / kThreads, bh), kThreads, 0, cs>>>(final_tok, order, nv, perm);
     SPARK_LAUNCH_CHECK();
+    note_launches(3);
   }
   const long long chunks = (long long)N * (D / 8);
   gather_kernel<D><<<dim3((unsigned)((chunks + kThreads - 1) / kThreads), bh), kThreads, 0, cs>>>(
       Q, K, V, perm, N, nv, Qp, Kp, Vp);
   SPARK_LAUNCH_CHECK();
+  note_launches(1);
   return SPARK_OK;
 }
 

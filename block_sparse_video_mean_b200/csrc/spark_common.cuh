@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/spark.h"
 
 namespace spark {
@@ -18,6 +20,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 // The library is one translation unit (spark_lib.cu includes every kernel header), so
 // this definition is unique.
 __device__ int g_error_word = 0;
+
+// Host-side count of kernel launches issued by the library (spark_kernel_launches).
+inline std::atomic<uint64_t> g_kernel_launches{0};
+inline void note_launches(int n) { g_kernel_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 __device__ __forceinline__ void set_error(int code) { atomicCAS(&g_error_word, 0, code); }
 

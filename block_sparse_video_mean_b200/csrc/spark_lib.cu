@@ -121,6 +121,7 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
     return SPARK_ECUDA;
   attn_tc_kernel<D><<<grid, C::kThreads, smem, cs>>>(maps, tp);
   SPARK_LAUNCH_CHECK();
+  note_launches(1);
   return SPARK_OK;
 }
 
@@ -219,6 +220,7 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
                                                          v16, s->N, nb, scale, pool_mode);
   }
   SPARK_LAUNCH_CHECK();
+  note_launches(3);
   return SPARK_OK;
 }
 
@@ -264,6 +266,7 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
       tau_threshold_kernel<64><<<bh, 64, 0, cs>>>(q_pool, k_pool, nb, acc, scale, param, thr);
     }
     SPARK_LAUNCH_CHECK();
+    note_launches(2);
   }
   SelectParams sp;
   sp.q_pool = q_pool;
@@ -286,6 +289,7 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
     score_select_kernel<64><<<grid, kSelThreads, smem, cs>>>(sp);
   }
   SPARK_LAUNCH_CHECK();
+  note_launches(1);
   return SPARK_OK;
 }
 
@@ -378,6 +382,8 @@ int spark_device_error(int32_t* host_word, void* stream) {
   if (host_word) *host_word = v;
   return SPARK_OK;
 }
+
+uint64_t spark_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 const char* spark_strerror(int status) {
   switch (status) {

@@ -28,7 +28,7 @@ BLOCK = 64
 
 EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
            "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
-           "spark_strerror", "spark_score_select_noalloc")
+           "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches")
 NOALLOC_MAX_HEADS = 4096
 
 
@@ -78,6 +78,8 @@ def load() -> ctypes.CDLL:
     lib.spark_device_error.restype = I
     lib.spark_strerror.argtypes = [I]
     lib.spark_strerror.restype = ctypes.c_char_p
+    lib.spark_kernel_launches.argtypes = []
+    lib.spark_kernel_launches.restype = ctypes.c_uint64
     _lib = lib
     return lib
 
@@ -113,6 +115,11 @@ def topk_count(ratio: float, nb: int) -> int:
 
 def workspace_bytes(shape: Shape, call_id: int) -> int:
     return int(load().spark_workspace_bytes(ctypes.byref(shape), int(call_id)))
+
+
+def kernel_launches() -> int:
+    """Kernels launched through the library by this process so far (host-side count)."""
+    return int(load().spark_kernel_launches())
 
 
 def device_error(device=None) -> int:
@@ -289,16 +296,29 @@ class SparkAttention:
                                      dtype=torch.uint8, device=dev)
             self.levels = levels
 
-    def run(self, Q, K, V):
+    def run(self, Q, K, V, events=None):
+        """One forward. ``events`` = optional list of five CUDA events, recorded on the
+        current stream before the reblock and after the reblock, the pooling, the
+        selection and the attention launch (for per-call timing)."""
         cfg = self.cfg
+        stream = torch.cuda.current_stream(Q.device)
+
+        def mark(i):
+            if events is not None:
+                events[i].record(stream)
         perm = None
+        mark(0)
         if self.rb is not None:
             reblock(Q, K, V, self.n_sink, out=self.rb, ws=self.rb_ws)
             Q, K, V, perm = self.rb["Qp"], self.rb["Kp"], self.rb["Vp"], self.rb["perm"]
+        mark(1)
         pool_kv(Q, K, V, self.n_sink, self.pool_mode, cfg.scale, out=self.pool)
+        mark(2)
         score_select(self.pool["q_pool"], self.pool["k_pool"], self.n_sink, Q.shape[2], self.mode,
                      cfg.param, self.kcap, cfg.scale, out=(self.idx, self.cnt), ws=self.sel_ws)
+        mark(3)
         attn_fwd(Q, K, V, self.idx, self.cnt, self.n_sink,
                  pack=self.pool["pack"] if cfg.compressed else None, beta=self.pool["beta"],
                  perm=perm, scale=cfg.scale, out=(self.O, self.lse))
+        mark(4)
         return self.O, self.lse

@@ -181,6 +181,11 @@ int spark_device_error(int32_t* host_word, void* stream);
 /* Human-readable text of a status code. */
 const char* spark_strerror(int status);
 
+/* Number of kernels this process has launched through the library so far (all devices
+ * and threads), counted on the host as each launch is issued. No counterpart in the
+ * method: it lets a caller account for the device work of a region of calls. */
+uint64_t spark_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif
