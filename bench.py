@@ -100,10 +100,11 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-# DRAM bytes (read + write) of one attention launch at the default workload, from
-# `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum` (summary under profiles/);
-# None once the kernel has changed since it was measured.
-ATTN_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) of one attention launch at the default workload: the
+# dram__bytes_read.sum + dram__bytes_write.sum of a 2-head capture of the same shape
+# (profiles/attn_tc_1152x640x243_h2_full.md), scaled by 12 to 24 heads. None once the
+# kernel has changed since it was measured.
+ATTN_TRAFFIC_BYTES = 96.1e9
 
 
 class ClockSampler:
