@@ -104,7 +104,7 @@ def load_peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum of a 2-head capture of the same shape
 # (profiles/attn_tc_1152x640x243_h2_full.md), scaled by 12 to 24 heads. None once the
 # kernel has changed since it was measured.
-ATTN_TRAFFIC_BYTES = 96.1e9
+ATTN_TRAFFIC_BYTES = None
 
 
 class ClockSampler:
@@ -176,7 +176,9 @@ def phase_bytes(w: Workload, h: int, nb: int, kept_blocks: int, kcap: int):
     nv = nb * 64
     n = nv + w.ns
     row = w.d * 2
-    pool = 3 * bh * nv * row + 3 * bh * nb * w.d * 4 + bh * nb * 4 + 2 * bh * nb * w.d * 2 + bh * w.d * 4
+    nbp = (nb + 63) // 64 * 64
+    pool = (3 * bh * nv * row + 3 * bh * nb * w.d * 4 + bh * nb * 4 + 2 * bh * nb * w.d * 2
+            + bh * nbp * 4 + bh * w.d * 4)
     select = 2 * bh * nb * w.d * 4 + kept_blocks * 4 + bh * nb * 4
     gather = 6 * bh * n * row + bh * nv * 4          # permute Q,K,V (read + write) + perm
     return dict(pool=pool, select=select, reblock_gather=gather)

@@ -8,29 +8,36 @@
 // README, "Nodes").
 //
 // Design (sm_100a):
-// * The unit of work is one 64-query block: video blocks select their own key blocks,
-//   so two query blocks cannot share an MMA B operand. tcgen05.mma with M = 64 runs at
-//   half the M = 128 rate, and every key of a 64-query block costs >= 1 KB of shared
-//   memory traffic (TMA writes K and V, the tensor core reads them) against a 128 B/clk
-//   port, so the kernel keeps everything else out of shared memory: Q and P live in
-//   tensor memory (A operand of "TS" MMAs), shared memory only carries the K/V ring.
+// * The unit of work is one 64-query block (an item): video blocks select their own key
+//   blocks, so two query blocks cannot share an MMA B operand. tcgen05.mma with M = 64
+//   runs at half the M = 128 rate, and every key of a 64-query block costs >= 1 KB of
+//   shared-memory traffic (TMA writes K and V, the tensor core reads them), so the kernel
+//   keeps everything else out of that path: Q and P live in tensor memory (A operand of
+//   "TS" MMAs), shared memory carries the K/V rings.
 // * Each persistent CTA runs two independent query blocks ("slots") whose M = 64
 //   accumulators share TMEM columns in the two lane halves of every sub-partition
 //   (slot 0: lanes 0-15, slot 1: lanes 16-31 of each 32-lane group), so the tensor core
 //   works on one slot while the other slot's softmax runs.
 // * Warp roles: warps 0-3 softmax of slot 0, warps 4-7 softmax of slot 1 (warp w reads
 //   TMEM sub-partition w % 4), warp 8 fills the K ring and warp 10 the V ring with TMA,
-//   warp 9 issues MMAs and owns TMEM. K stages are released when their S MMAs complete and
-//   V stages when their PV MMAs complete, so neither producer waits on an MMA that the
-//   issuer can only start later.
+//   warps 9 and 11 issue the MMAs of slot 0 and slot 1 (warp 9 owns TMEM). The tensor
+//   pipe queues little more than one MMA, so an issuer's barrier checks between MMA
+//   blocks leave it idle; with one issuer per slot the other slot's MMAs fill that gap.
+//   K stages are released when their S MMAs complete and V stages when their PV MMAs
+//   complete.
 // * A tile is 128 keys made of two 64-key halves (a selected block, 64 dense rows or 64
 //   pooled entries each; per video query block the halves run selected blocks, dense key
 //   rows, then pooled entries). Per tile: S = Q K^T (8 MMAs 64x128x16 from TMEM Q and a
 //   128B-swizzled K tile), softmax in base 2 (each thread owns one half of one row) with a
 //   lazy running max (O is rescaled only when the row max grows by more than 2^8), P
 //   written back over S as bf16, then O += P V (8 MMAs 64xDx16, V as an MN-major operand).
+// * Item transitions stay off the tensor core's path: Q is double-buffered in TMEM and the
+//   next item's Q rows and selection bitmap are fetched a piece per tile during the
+//   current item (loads issued after a tile, consumed after the next tile's S is ready);
+//   the epilogue releases O as soon as it has read it. The compressed branch's biases are
+//   staged per tile into shared memory with cp.async, one tile ahead.
 // * Every mbarrier wait is bounded; a timeout records SPARK_ETIMEOUT, raises the CTA abort
-//   flag, the TMA role drains its copies in flight and TMEM is released.
+//   flag, the TMA roles drain their copies in flight and TMEM is released.
 #pragma once
 #include "spark_common.cuh"
 #include "tc_util.cuh"
@@ -54,11 +61,11 @@ struct TcParams {
   const uint16_t* Q;
   const int32_t* idx;
   const int32_t* cnt;
-  const float* beta;
+  const float* bias;  // pooled bias * log2(e), [B*H, nbp] (-inf past nb); pooled only
   const int32_t* perm;
   uint16_t* O;
   float* lse;
-  int N, nb, kcap, BH, n_dq, pooled, n_items;
+  int N, nb, nbp, kcap, BH, n_dq, pooled, n_items;
   float scale_log2;
 };
 
@@ -73,12 +80,24 @@ struct TcCfg {
   static constexpr int kTileBytes = 128 * D * 2;   // K (or V) of one 128-key tile
   static constexpr int kColS = 0;                  // S/P buffers at 0 and 128
   static constexpr int kColO = 256;
-  static constexpr int kColQ = 256 + D;
+  static constexpr int kColQ = 256 + D;            // Q buffers at kColQ and kColQ + D/2
   static constexpr int kTmemCols = 512;
-  static constexpr int kThreads = 352;
+  static constexpr int kThreads = 384;
   static constexpr int kRingBytes = 2 * kStages * kTileBytes;  // K ring, then V ring
   static constexpr int kBarBytes = 1024;
+  static constexpr int kBiasBytes = 8 * 2 * 512;   // per softmax warp: 2 tiles x 2 halves x 64 fp32
+  static constexpr int kQPieces = D / 64;          // 16-word pieces of a thread's half Q row
 };
+
+// Words of one selection bitmap (even, so a 64-entry pooled half never reads past it).
+__host__ __device__ inline int tc_bitmap_words(int nb) { return ((nb + 31) / 32 + 1) & ~1; }
+
+template <int D>
+__host__ __device__ inline size_t tc_smem_bytes(int nb) {
+  using C = TcCfg<D>;
+  return 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes + C::kBiasBytes +
+         (size_t)8 * 2 * tc_bitmap_words(nb) * 4;  // two bitmaps per softmax warp
+}
 
 struct TcItem {
   int bh, q0, nq, dense, cnt, nhalf, ntiles;  // nhalf 64-key halves, ntiles = ceil(nhalf / 2)
@@ -106,7 +125,7 @@ __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
     int c = p.cnt[r.row];
     c = c < 0 ? 0 : (c > p.kcap ? p.kcap : c);
     r.cnt = c;
-    r.nhalf = c + n_dk + (p.pooled ? (p.nb + kBlock - 1) / kBlock : 0);
+    r.nhalf = c + n_dk + (p.pooled ? p.nbp / kBlock : 0);
   }
   r.ntiles = (r.nhalf + 1) / 2;
   r.nq = min(kBlock, p.N - r.q0);
@@ -158,8 +177,20 @@ __device__ __forceinline__ uint64_t tc_vdesc(uint32_t stage_addr, int kk) {
   return tc::make_sdesc(stage_addr + kk * 2048, TcCfg<D>::kPanelBytes, 1024, tc::kSwizzle128);
 }
 
+// The four 64-key half kinds of a tile.
+enum : int { kHalfExact = 0, kHalfDense = 1, kHalfPooled = 2, kHalfMissing = 3 };
+
+// Kind and first key / pooled entry of half `hi` of item I (video or dense).
+__device__ __forceinline__ int tc_half_kind(const TcItem& I, int hi, int n_dk) {
+  if (hi >= I.nhalf) return kHalfMissing;
+  if (I.dense) return kHalfDense;
+  if (hi < I.cnt) return kHalfExact;
+  if (hi < I.cnt + n_dk) return kHalfDense;
+  return kHalfPooled;
+}
+
 template <int D>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
   using C = TcCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -171,17 +202,17 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t* vfull = kfull + C::kStages;
   uint64_t* kempty = vfull + C::kStages;   // K stage free: its S MMAs completed
   uint64_t* vempty = kempty + C::kStages;  // V stage free: its PV MMAs completed
-  uint64_t* sfull = vempty + C::kStages;   // [slot][buf]
-  uint64_t* pfull = sfull + 4;             // [slot][buf]
-  uint64_t* oready = pfull + 4;            // [slot]
-  uint64_t* qfull = oready + 2;            // [slot]
-  uint64_t* ofree = qfull + 2;             // [slot]
+  uint64_t* sfull = vempty + C::kStages;   // [slot][S buffer]
+  uint64_t* pfull = sfull + 4;             // [slot][S buffer]
+  uint64_t* oready = pfull + 4;            // [slot]: a PV completed
+  uint64_t* qfull = oready + 2;            // [slot][Q buffer]
+  uint64_t* ofree = qfull + 4;             // [slot]: the epilogue has read O
   uint64_t* odone = ofree + 2;             // [slot]: last PV of an item completed
-  uint64_t* finbar = odone + 2;            // all MMAs of the CTA done
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 1);
+  uint64_t* finbar = odone + 2;            // [slot]: all MMAs of that slot's issuer done
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
-  const int nbw = (p.nb + 31) / 32;
+  float* bias_stage = reinterpret_cast<float*>(ring + C::kRingBytes + C::kBarBytes);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes + C::kBiasBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   SPARK_TC_DECL
@@ -195,14 +226,15 @@ __global__ void __launch_bounds__(352, 1)
     for (int i = 0; i < 4; ++i) {
       tc::mbar_init(&sfull[i], 1);
       tc::mbar_init(&pfull[i], 4);
+      tc::mbar_init(&qfull[i], 4);
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&oready[i], 1);
-      tc::mbar_init(&qfull[i], 4);
       tc::mbar_init(&ofree[i], 4);
       tc::mbar_init(&odone[i], 1);
     }
-    tc::mbar_init(finbar, 1);
+    tc::mbar_init(&finbar[0], 1);
+    tc::mbar_init(&finbar[1], 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -221,10 +253,13 @@ __global__ void __launch_bounds__(352, 1)
   tc::tc_fence_after();
   const uint32_t tbase = *tmem_holder;
   const int stride = 2 * gridDim.x;
+  const int nv = p.nb * kBlock;
+  const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
 
   if (warp == 8 || warp == 10) {
     // ================================================================ TMA producers
-    // warp 8 fills the K ring, warp 10 the V ring, both in the same tile order.
+    // warp 8 fills the K ring, warp 10 the V ring, both in the same tile order: per round,
+    // one tile of slot 0 then one of slot 1 (a slot without items is skipped).
     const bool is_v = warp == 10;
     uint64_t* full = is_v ? vfull : kfull;
     uint64_t* empty = is_v ? vempty : kempty;
@@ -239,73 +274,75 @@ __global__ void __launch_bounds__(352, 1)
     bool have[2];
     int t[2] = {0, 0};
     int ic[2] = {0, 0}, in[2] = {0, 0};  // idx of halves 32c + lane (current / next chunk)
-    auto chunk = [&](int s, int c) -> int {
-      const int hh = 32 * c + lane;
-      return hh < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + hh] : 0;
-    };
+#pragma unroll
     for (int s = 0; s < 2; ++s) {
       have[s] = walk[s].next_nonempty(p, &cur[s]);
       if (have[s] && !cur[s].dense) {
-        ic[s] = chunk(s, 0);
-        in[s] = chunk(s, 1);
+        const int h0 = lane, h1 = 32 + lane;
+        ic[s] = h0 < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + h0] : 0;
+        in[s] = h1 < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + h1] : 0;
       }
     }
-    const int nv = p.nb * kBlock;
-    const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
     uint32_t q = 0;
     bool ok = true;
     while (ok && (have[0] || have[1])) {
-      for (int s = 0; s < 2 && ok; ++s) {
-        if (!have[s]) continue;
-        const int stage = q % C::kStages;
-        SPARK_TC_T0(t_ew);
-        if (q >= (uint32_t)C::kStages &&
-            !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        SPARK_TC_ACC(4, t_ew);
-        const TcItem& I = cur[s];
-        int y[2], pooled[2];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          int hi = 2 * t[s] + hf;
-          if (hi >= I.nhalf) hi = 2 * t[s];  // a missing second half repeats the first (masked)
-          const int bsel = __shfl_sync(0xffffffffu, ic[s], hi & 31);
-          pooled[hf] = 0;
-          if (I.dense) {
-            y[hf] = I.bh * p.N + hi * kBlock;
-          } else if (hi < I.cnt) {
-            y[hf] = I.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
-          } else if (hi < I.cnt + n_dk) {
-            y[hf] = I.bh * p.N + nv + (hi - I.cnt) * kBlock;
+      for (int s = 0; s < 2; ++s) {
+        if (ok && have[s]) {
+          const int stage = q % C::kStages;
+          SPARK_TC_T0(t_ew);
+          if (q >= (uint32_t)C::kStages &&
+              !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag)) {
+            ok = false;
           } else {
-            pooled[hf] = 1;
-            y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk) * kBlock;
-          }
-        }
-        if (lane == 0) {
-          unsigned char* st = rbase + stage * C::kTileBytes;
-          tc::mbar_expect_tx(&full[stage], C::kTileBytes);
+            SPARK_TC_ACC(4, t_ew);
+            const TcItem& I = cur[s];
+            int y[2], pooled[2];
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < 2; ++hf) {
+              int hi = 2 * t[s] + hf;
+              if (hi >= I.nhalf) hi = 2 * t[s];  // a missing second half repeats the first (masked)
+              const int bsel = __shfl_sync(0xffffffffu, ic[s], hi & 31);
+              pooled[hf] = 0;
+              if (I.dense) {
+                y[hf] = I.bh * p.N + hi * kBlock;
+              } else if (hi < I.cnt) {
+                y[hf] = I.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
+              } else if (hi < I.cnt + n_dk) {
+                y[hf] = I.bh * p.N + nv + (hi - I.cnt) * kBlock;
+              } else {
+                // pooled entries past nb read rows of the next head (or TMA zero fill);
+                // their bias is -inf, so they carry no weight
+                pooled[hf] = 1;
+                y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk) * kBlock;
+              }
+            }
+            if (lane == 0) {
+              unsigned char* st = rbase + stage * C::kTileBytes;
+              tc::mbar_expect_tx(&full[stage], C::kTileBytes);
 #pragma unroll
-            for (int pn = 0; pn < C::kPanels; ++pn)
-              tc::tma_load_2d(st + pn * C::kPanelBytes + hf * C::kHalfBytes,
-                              pooled[hf] ? map_p : map_x, pn * 64, y[hf], &full[stage]);
-        }
-        __syncwarp();
-        ++q;
-        if (++t[s] == cur[s].ntiles) {
-          t[s] = 0;
-          have[s] = walk[s].next_nonempty(p, &cur[s]);
-          if (have[s] && !cur[s].dense) {
-            ic[s] = chunk(s, 0);
-            in[s] = chunk(s, 1);
+              for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int pn = 0; pn < C::kPanels; ++pn)
+                  tc::tma_load_2d(st + pn * C::kPanelBytes + hf * C::kHalfBytes,
+                                  pooled[hf] ? map_p : map_x, pn * 64, y[hf], &full[stage]);
+            }
+            __syncwarp();
+            ++q;
+            if (++t[s] == cur[s].ntiles) {
+              t[s] = 0;
+              have[s] = walk[s].next_nonempty(p, &cur[s]);
+              if (have[s] && !cur[s].dense) {
+                const int h0 = lane, h1 = 32 + lane;
+                ic[s] = h0 < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + h0] : 0;
+                in[s] = h1 < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + h1] : 0;
+              }
+            } else if ((t[s] & 15) == 0 && !cur[s].dense && 2 * t[s] < cur[s].cnt) {
+              const int hn = 32 * ((t[s] >> 4) + 1) + lane;
+              ic[s] = in[s];
+              in[s] = hn < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + hn] : 0;
+            }
           }
-        } else if ((t[s] & 15) == 0 && !cur[s].dense && 2 * t[s] < cur[s].cnt) {
-          ic[s] = in[s];
-          in[s] = chunk(s, (t[s] >> 4) + 1);
         }
       }
     }
@@ -314,128 +351,98 @@ __global__ void __launch_bounds__(352, 1)
       const uint32_t first = q > (uint32_t)C::kStages ? q - C::kStages : 0;
       for (uint32_t j = first; j < q; ++j) mbar_drain(&full[j % C::kStages], (j / C::kStages) & 1);
     }
-  } else if (warp == 9) {
-    // ================================================================ MMA issuer
+  } else if (warp == 9 || warp == 11) {
+    // ================================================================ MMA issuers
+    // One issuing thread per slot (warp 9: slot 0, warp 11: slot 1): per tile, S of the
+    // slot's next tile then PV of its previous one. Two issuers keep the tensor pipe fed
+    // while either waits on a barrier. Both replay the producers' round-robin tile order
+    // to find the ring stage of each of their tiles.
     if (lane == 0) {
+      const int s = warp == 9 ? 0 : 1;
       constexpr uint32_t idS = tc::make_idesc_bf16(64, 128, 0, 0);
       constexpr uint32_t idPV = tc::make_idesc_bf16(64, D, 0, 1);
+      const uint32_t lanes = (uint32_t)(16 * s) << 16;
       TcSlotWalk walk[2] = {{2 * (int)blockIdx.x, stride, p.n_items},
                             {2 * (int)blockIdx.x + 1, stride, p.n_items}};
       TcItem cur[2];
       bool have[2];
       int t[2] = {0, 0};
-      uint32_t g[2] = {0, 0};       // tiles issued per slot (all items)
-      uint32_t nitem[2] = {0, 0};   // non-empty items started per slot
-      struct Pend {
-        int valid;
-        uint32_t q, g, item;
-        int first, last;
-      } pend[2] = {{0, 0, 0, 0, 0, 0}, {0, 0, 0, 0, 0, 0}};
-      for (int s = 0; s < 2; ++s) have[s] = walk[s].next_nonempty(p, &cur[s]);
+#pragma unroll
+      for (int o = 0; o < 2; ++o) have[o] = walk[o].next_nonempty(p, &cur[o]);
+      uint32_t g = 0;      // tiles of this slot issued (all items)
+      uint32_t nitem = 0;  // non-empty items of this slot started
+      bool pend = false;   // PV of the previous tile still to issue
+      uint32_t pq = 0, pg = 0, pitem = 0;
+      bool pfirst = false, plast = false;
       const uint32_t ring_addr = tc::smem_addr(ring);
       const uint32_t vring_addr = tc::smem_addr(vring);
       bool ok = true;
-      auto issue_pv = [&](int s, const Pend& pe) -> bool {
-        const uint32_t b = pe.g & 1;
-        SPARK_TC_T0(t_pw);
-        if (!tc::mbar_wait(&pfull[2 * s + b], (pe.g >> 1) & 1, abort_flag)) return false;
-        SPARK_TC_ACC(0, t_pw);
-        SPARK_TC_EV(0, 30 + s);
-        const int stage = pe.q % C::kStages;
-        SPARK_TC_T0(t_vw);
-        if (!tc::mbar_wait(&vfull[stage], (pe.q / C::kStages) & 1, abort_flag)) return false;
-        SPARK_TC_ACC(1, t_vw);
-        SPARK_TC_T0(t_ow);
-        if (pe.first && pe.item > 0 && !tc::mbar_wait(&ofree[s], (pe.item - 1) & 1, abort_flag))
-          return false;
-        SPARK_TC_ACC(9, t_ow);
-        SPARK_TC_T0(t_pv);
+      auto issue_pv = [&]() -> bool {
+        const uint32_t b = pg & 1;
+        if (!tc::mbar_wait(&pfull[2 * s + b], (pg >> 1) & 1, abort_flag)) return false;
+        const int stage = pq % C::kStages;
+        if (!tc::mbar_wait(&vfull[stage], (pq / C::kStages) & 1, abort_flag)) return false;
+        if (pfirst && pitem > 0 && !tc::mbar_wait(&ofree[s], (pitem - 1) & 1, abort_flag)) return false;
         tc::tc_fence_after();
-        const uint32_t lanes = (uint32_t)(16 * s) << 16;
         const uint32_t st = vring_addr + stage * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc::mma_ts(tbase + lanes + C::kColO, tbase + lanes + C::kColS + 128 * b + kk * 8,
-                     tc_vdesc<D>(st, kk), idPV, (pe.first && kk == 0) ? 0u : 1u);
+                     tc_vdesc<D>(st, kk), idPV, (pfirst && kk == 0) ? 0u : 1u);
         tc::mma_commit(&vempty[stage]);
         tc::mma_commit(&oready[s]);
-        if (pe.last) tc::mma_commit(&odone[s]);
-        SPARK_TC_EV(0, 20 + s);
-        SPARK_TC_ACC(10, t_pv);
+        if (plast) tc::mma_commit(&odone[s]);
         return true;
       };
-      uint32_t q = 0;
-      SPARK_TC_T0(t_all);
+      uint32_t q = 0;  // ring position of the producers' next tile
       while (ok && (have[0] || have[1])) {
-        // S of both slots first, so the tensor core has work while a softmax finishes
-        Pend nxt[2] = {{0, 0, 0, 0, 0, 0}, {0, 0, 0, 0, 0, 0}};
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (!have[s]) continue;
-          SPARK_TC_T0(t_qw);
-          if (t[s] == 0 && !tc::mbar_wait(&qfull[s], nitem[s] & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          SPARK_TC_ACC(3, t_qw);
-          const int stage = q % C::kStages;
-          SPARK_TC_T0(t_kw);
-          if (!tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          SPARK_TC_ACC(2, t_kw);
-          SPARK_TC_T0(t_si);
-          tc::tc_fence_after();
-          const uint32_t b = g[s] & 1;
-          const uint32_t lanes = (uint32_t)(16 * s) << 16;
-          const uint32_t st = ring_addr + stage * C::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            tc::mma_ts(tbase + lanes + C::kColS + 128 * b, tbase + lanes + C::kColQ + kk * 8,
-                       tc_kdesc<D>(st, kk), idS, kk > 0 ? 1u : 0u);
-          tc::mma_commit(&sfull[2 * s + b]);
-          tc::mma_commit(&kempty[stage]);
-          SPARK_TC_EV(0, 10 + s);
-          SPARK_TC_ACC(11, t_si);
-          nxt[s].valid = 1;
-          nxt[s].q = q;
-          nxt[s].g = g[s];
-          nxt[s].item = nitem[s];
-          nxt[s].first = (t[s] == 0);
-          nxt[s].last = (t[s] + 1 == cur[s].ntiles);
-          ++q;
-          ++g[s];
-          if (++t[s] == cur[s].ntiles) {
-            t[s] = 0;
-            ++nitem[s];
-            SPARK_TC_T0(t_nx);
-            have[s] = walk[s].next_nonempty(p, &cur[s]);
-            SPARK_TC_ACC(12, t_nx);
-          }
-        }
-        // then the PV of each slot's previous tile; a slot that just ran out also
-        // releases its last tile
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (pend[s].valid && !issue_pv(s, pend[s])) {
-            ok = false;
-            break;
-          }
-          pend[s] = nxt[s];
-          if (pend[s].valid && !have[s]) {
-            if (!issue_pv(s, pend[s])) {
-              ok = false;
-              break;
+        for (int o = 0; o < 2; ++o) {
+          if (ok && have[o]) {
+            if (o == s) {
+              const uint32_t qb = nitem & 1;
+              bool good = t[o] != 0 || tc::mbar_wait(&qfull[2 * s + qb], (nitem >> 1) & 1, abort_flag);
+              const int stage = q % C::kStages;
+              good = good && tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag);
+              if (!good) {
+                ok = false;
+              } else {
+                tc::tc_fence_after();
+                const uint32_t b = g & 1;
+                const uint32_t st = ring_addr + stage * C::kTileBytes;
+                const uint32_t qcol = C::kColQ + qb * (D / 2);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                  tc::mma_ts(tbase + lanes + C::kColS + 128 * b, tbase + lanes + qcol + kk * 8,
+                             tc_kdesc<D>(st, kk), idS, kk > 0 ? 1u : 0u);
+                tc::mma_commit(&sfull[2 * s + b]);
+                tc::mma_commit(&kempty[stage]);
+                // then the PV of the previous tile of this slot
+                if (pend) ok = issue_pv();
+                pend = true;
+                pq = q;
+                pg = g;
+                pitem = nitem;
+                pfirst = (t[o] == 0);
+                plast = (t[o] + 1 == cur[o].ntiles);
+                ++g;
+                if (t[o] + 1 == cur[o].ntiles) ++nitem;
+              }
             }
-            pend[s].valid = 0;
+            if (ok) {
+              ++q;
+              if (++t[o] == cur[o].ntiles) {
+                t[o] = 0;
+                have[o] = walk[o].next_nonempty(p, &cur[o]);
+              }
+            }
           }
         }
       }
-      for (int s = 0; s < 2 && ok; ++s)
-        if (pend[s].valid && !issue_pv(s, pend[s])) ok = false;
-      SPARK_TC_ACC(13, t_all);
-      // every MMA of this CTA must be complete before TMEM is released
-      tc::mma_commit(finbar);
-      mbar_drain(finbar, 0);
+      if (ok && pend) ok = issue_pv();
+      // every MMA of this issuer must be complete before TMEM is released
+      tc::mma_commit(&finbar[s]);
+      mbar_drain(&finbar[s], 0);
     }
   } else {
     // ================================================================ softmax (slot s)
@@ -443,19 +450,107 @@ __global__ void __launch_bounds__(352, 1)
     const int w = warp & 3;
     const int r = 16 * w + (lane & 15);  // query row within the block
     const int h = lane >> 4;             // key half (scores) / d half (O, Q)
+    const int lh = lane & 15;
     const uint32_t lanes = (uint32_t)(32 * w + 16 * s) << 16;
-    uint32_t* bm = bitmap + warp * nbw;  // this warp's selection bitmap
-    const int nv = p.nb * kBlock;
-    const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
+    const int nbwp = tc_bitmap_words(p.nb);
+    uint32_t* bm2 = bitmap + warp * 2 * nbwp;  // this warp's two selection bitmaps
+    float* bst = bias_stage + warp * 256;       // [tile parity][half][64] pooled biases
+    bool ok = true;
 
-    TcSlotWalk walk = {2 * (int)blockIdx.x + s, stride, p.n_items};
-    uint32_t g = 0;
-    int have_prev = 0;
-    TcItem prev;
-    prev.ntiles = 0;
-    float m_prev = -INFINITY, l_prev = 0.f;
-    uint32_t nitem = 0;
-    int cur_bad = 0;
+    // ---- preparation of an item, a unit per tile: the thread's Q half row in kQPieces
+    //      16-word pieces into a TMEM Q buffer, then the selection bitmap from its index
+    //      row, 128 indices per unit. Loads are issued after a tile and consumed after
+    //      the next tile's S is ready, so their latency hides behind that wait.
+    TcItem J;                 // the item being prepared
+    int prep_qb = 0, prep_units = 0, prep_u = 0, prep_pend = -1;
+    int bad_next = 0;         // J has a block index out of range
+    uint32_t pf[16];
+    auto prep_setup = [&](const TcItem& It, int qb) {
+      J = It;
+      prep_qb = qb;
+      const bool need_bm = !It.dense && (p.pooled || It.cnt > 0);
+      prep_units = C::kQPieces + (need_bm ? max(1, (It.cnt + 127) / 128) : 0);
+      prep_u = 0;
+      prep_pend = -1;
+    };
+    auto prep_issue = [&](int u) {
+      if (u < C::kQPieces) {
+        const bool rv = r < J.nq;
+        const uint16_t* qrow =
+            p.Q + ((size_t)J.bh * p.N + J.q0 + (rv ? r : 0)) * D + h * (D / 2) + 32 * u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 a = rv ? ldg_nc_v4(qrow + 8 * i) : make_uint4(0, 0, 0, 0);
+          pf[4 * i] = a.x;
+          pf[4 * i + 1] = a.y;
+          pf[4 * i + 2] = a.z;
+          pf[4 * i + 3] = a.w;
+        }
+      } else {
+        const int c = u - C::kQPieces;
+        const int32_t* ip = p.idx + J.row * (size_t)p.kcap;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 128 * c + 32 * i + lane;
+          pf[i] = j < J.cnt ? (uint32_t)ip[j] : 0u;
+        }
+      }
+    };
+    auto prep_consume = [&](int u) {
+      if (u < C::kQPieces) {
+        tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + prep_qb * (D / 2) + 16 * u, pf);
+        if (u == C::kQPieces - 1) {
+          tc::tmem_wait_st();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&qfull[2 * s + prep_qb]);
+        }
+      } else {
+        const int c = u - C::kQPieces;
+        uint32_t* bm = bm2 + prep_qb * nbwp;
+        if (c == 0) {
+          for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
+          __syncwarp();
+          if (lane == 0 && w == 0 && p.cnt[J.row] != J.cnt) set_error(SPARK_EDEVICE_INDEX);
+        }
+        int bad = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 128 * c + 32 * i + lane;
+          const int b = (int)pf[i];
+          if (j < J.cnt) {
+            if (b >= 0 && b < p.nb) atomicOr(&bm[b >> 5], 1u << (b & 31));
+            else bad = 1;
+          }
+        }
+        if (__any_sync(0xffffffffu, bad)) {
+          bad_next = 1;
+          if (lane == 0) set_error(SPARK_EDEVICE_INDEX);
+        }
+        __syncwarp();
+      }
+    };
+    auto prep_flush = [&]() {
+      if (prep_pend >= 0) {
+        prep_consume(prep_pend);
+        prep_pend = -1;
+      }
+      for (; prep_u < prep_units; ++prep_u) {
+        prep_issue(prep_u);
+        prep_consume(prep_u);
+      }
+    };
+    // Pooled biases of half h of tile tt into the staging buffer of tt's parity (one
+    // cp.async group per call, empty when the half is not pooled).
+    auto stage_bias = [&](const TcItem& It, int tt) {
+      const int hi = 2 * tt + h;
+      if (tt < It.ntiles && tc_half_kind(It, hi, n_dk) == kHalfPooled) {
+        const int j0 = (hi - It.cnt - n_dk) * kBlock;
+        tc::cp_async_16(bst + (tt & 1) * 128 + h * 64 + 4 * lh,
+                        p.bias + (size_t)It.bh * p.nbp + j0 + 4 * lh);
+      }
+      tc::cp_async_commit();
+    };
 
     uint32_t ndone = 0;  // non-empty items whose epilogue ran
     auto epilogue = [&](const TcItem& I, float m_run, float l_run) -> bool {
@@ -464,6 +559,15 @@ __global__ void __launch_bounds__(352, 1)
       if (!tc::mbar_wait(&odone[s], ndone & 1, abort_flag)) return false;
       ++ndone;
       tc::tc_fence_after();
+      uint32_t o[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+        tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, o + 16 * c);
+      tc::tmem_wait_ld();
+      // O is in registers: the next item's first PV may overwrite it
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ofree[s]);
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
       int orow = I.q0 + r;
@@ -475,129 +579,85 @@ __global__ void __launch_bounds__(352, 1)
           write = false;
         }
       }
-      uint16_t* dst = p.O + ((size_t)I.bh * p.N + orow) * D + h * (D / 2);
+      if (write) {
+        uint16_t* dst = p.O + ((size_t)I.bh * p.N + orow) * D + h * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[16];
-        tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
-        tc::tmem_wait_ld();
-        if (write) {
-          uint4 o0, o1;
-          o0.x = pack_bf16x2(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
-          o0.y = pack_bf16x2(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv);
-          o0.z = pack_bf16x2(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv);
-          o0.w = pack_bf16x2(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv);
-          o1.x = pack_bf16x2(__uint_as_float(v[8]) * inv, __uint_as_float(v[9]) * inv);
-          o1.y = pack_bf16x2(__uint_as_float(v[10]) * inv, __uint_as_float(v[11]) * inv);
-          o1.z = pack_bf16x2(__uint_as_float(v[12]) * inv, __uint_as_float(v[13]) * inv);
-          o1.w = pack_bf16x2(__uint_as_float(v[14]) * inv, __uint_as_float(v[15]) * inv);
-          *reinterpret_cast<uint4*>(dst + 16 * c) = o0;
-          *reinterpret_cast<uint4*>(dst + 16 * c + 8) = o1;
+        for (int c = 0; c < D / 16; ++c) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[8 * c]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + 8 * c) = v;
         }
+        if (h == 0 && p.lse != nullptr)
+          p.lse[(size_t)I.bh * p.N + orow] = l_tot > 0.f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
       }
-      if (write && h == 0 && p.lse != nullptr)
-        p.lse[(size_t)I.bh * p.N + orow] = l_tot > 0.f ? (m_run + __log2f(l_tot)) * kLn2 : -INFINITY;
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&ofree[s]);
       return true;
     };
 
-    bool ok = true;
-    while (ok) {
-      // ---- next item of this slot (possibly empty)
-      TcItem I;
-      bool more = false;
+    // Items of this slot in order; an item with nothing to attend to gets O = 0, LSE = -inf.
+    TcSlotWalk walk = {2 * (int)blockIdx.x + s, stride, p.n_items};
+    auto next_item = [&](TcItem* I) -> bool {
       while (walk.it < walk.n) {
-        I = tc_item(p, walk.it);
+        *I = tc_item(p, walk.it);
         walk.it += walk.stride;
-        if (I.ntiles > 0) {
-          more = true;
-          break;
-        }
-        // an item with nothing to attend to: O = 0, LSE = -inf
-        if (r < I.nq) {
-          int orow = I.q0 + r;
-          bool write = true;
-          if (!I.dense && p.perm != nullptr) {
-            orow = p.perm[(size_t)I.bh * nv + I.q0 + r];
-            write = orow >= 0 && orow < nv;
+        if (I->ntiles > 0) return true;
+        if (r < I->nq) {
+          int orow = I->q0 + r;
+          bool wr = true;
+          if (!I->dense && p.perm != nullptr) {
+            orow = p.perm[(size_t)I->bh * nv + I->q0 + r];
+            wr = orow >= 0 && orow < nv;
           }
-          if (write) {
-            uint4 z = make_uint4(0, 0, 0, 0);
-            uint16_t* dst = p.O + ((size_t)I.bh * p.N + orow) * D + h * (D / 2);
+          if (wr) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            uint16_t* dst = p.O + ((size_t)I->bh * p.N + orow) * D + h * (D / 2);
 #pragma unroll
             for (int c = 0; c < D / 16; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = z;
-            if (h == 0 && p.lse != nullptr) p.lse[(size_t)I.bh * p.N + orow] = -INFINITY;
+            if (h == 0 && p.lse != nullptr) p.lse[(size_t)I->bh * p.N + orow] = -INFINITY;
           }
         }
       }
-      if (more) {
-        // ---- selection bitmap (pooled masking) and index validity, one copy per warp so
-        //      that no barrier wider than a warp is needed
-        int bad_idx = 0;
-        if (!I.dense && (p.pooled || I.cnt > 0)) {
-          for (int i = lane; i < nbw; i += 32) bm[i] = 0u;
-          __syncwarp();
-          const int32_t* ip = p.idx + I.row * (size_t)p.kcap;
-          int bad = 0;
-          for (int i = lane; i < I.cnt; i += 32) {
-            const int b = ip[i];
-            if (b >= 0 && b < p.nb) atomicOr(&bm[b >> 5], 1u << (b & 31));
-            else bad = 1;
-          }
-          bad_idx = __any_sync(0xffffffffu, bad);
-          if (bad_idx && lane == 0) set_error(SPARK_EDEVICE_INDEX);
-          if (lane == 0 && w == 0 && p.cnt[I.row] != I.cnt) set_error(SPARK_EDEVICE_INDEX);
-          __syncwarp();
-        }
-        cur_bad = bad_idx;
-        // ---- Q block into TMEM (bf16 pairs, A-operand layout of the M = 64 MMA)
-        {
-          const bool rv = r < I.nq;
-          const uint16_t* qrow = p.Q + ((size_t)I.bh * p.N + I.q0 + (rv ? r : 0)) * D + h * (D / 2);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            uint32_t v[16];
-            uint4 a = rv ? ldg_nc_v4(qrow + 32 * c) : make_uint4(0, 0, 0, 0);
-            uint4 b2 = rv ? ldg_nc_v4(qrow + 32 * c + 8) : make_uint4(0, 0, 0, 0);
-            uint4 c2 = rv ? ldg_nc_v4(qrow + 32 * c + 16) : make_uint4(0, 0, 0, 0);
-            uint4 d2 = rv ? ldg_nc_v4(qrow + 32 * c + 24) : make_uint4(0, 0, 0, 0);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-            v[4] = b2.x; v[5] = b2.y; v[6] = b2.z; v[7] = b2.w;
-            v[8] = c2.x; v[9] = c2.y; v[10] = c2.z; v[11] = c2.w;
-            v[12] = d2.x; v[13] = d2.y; v[14] = d2.z; v[15] = d2.w;
-            tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + 16 * c, v);
-          }
-          tc::tmem_wait_st();
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&qfull[s]);
-        }
-      }
-      // ---- finish the previous item (its last PV was issued after this item's first S)
-      if (have_prev) {
-        if (!epilogue(prev, m_prev, l_prev)) {
-          ok = false;
-          break;
-        }
-        have_prev = 0;
-      }
-      if (!more) break;
+      return false;
+    };
 
-      // ---- tiles of this item
-      const int bad_idx = cur_bad;
+    uint32_t g = 0;  // tiles processed by this slot (all items)
+    uint32_t n = 0;  // non-empty items of this slot so far
+    TcItem I, prev;
+    prev.ntiles = 0;
+    bool have_prev = false;
+    float m_prev = -INFINITY, l_prev = 0.f;
+    bool have = next_item(&I);
+    TcSlotWalk ahead = walk;  // finds the next non-empty item one ahead
+    if (have) {
+      prep_setup(I, 0);
+      prep_flush();
+    }
+    int cur_bad = bad_next;
+    bad_next = 0;
+    while (ok && have) {
+      TcItem nxt;
+      if (ahead.next_nonempty(p, &nxt)) prep_setup(nxt, (n + 1) & 1);
+      else prep_units = prep_u = 0, prep_pend = -1;
+      const uint32_t* bm = bm2 + (n & 1) * nbwp;
+
       float m_run = -INFINITY, l_run = 0.f;
       for (int t = 0; t < I.ntiles; ++t, ++g) {
         const uint32_t b = g & 1;
+        if (t == 0) stage_bias(I, 0);
+        stage_bias(I, t + 1);
         SPARK_TC_T0(t_sw);
         if (!tc::mbar_wait(&sfull[2 * s + b], (g >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         SPARK_TC_ACC(5, t_sw);
-        SPARK_TC_EV(1 + s, 40);
         tc::tc_fence_after();
+        if (prep_pend >= 0) {
+          prep_consume(prep_pend);
+          prep_pend = -1;
+        }
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h+63 of the S buffer)
         float x[64];
         SPARK_TC_T0(t_ld);
@@ -610,53 +670,57 @@ __global__ void __launch_bounds__(352, 1)
         SPARK_TC_T0(t_cp);
         // ---- logits (base 2) and masks of this half
         const int hi = 2 * t + h;
-        int kind = 0, valid = kBlock, j0 = 0;
-        if (hi >= I.nhalf) {
-          valid = 0;
-        } else if (I.dense) {
-          valid = min(kBlock, p.N - hi * kBlock);
-        } else if (hi < I.cnt) {
-          if (bad_idx) {
+        const int kind = tc_half_kind(I, hi, n_dk);
+        const bool any_pooled = tc_half_kind(I, 2 * t, n_dk) == kHalfPooled ||
+                                tc_half_kind(I, 2 * t + 1, n_dk) == kHalfPooled;  // warp-uniform
+        // Exact and dense halves keep raw scores (the scale is folded into the exponent's
+        // FFMA); pooled halves become scale*logit + beta*log2(e), with the selected blocks
+        // masked (entries past nb carry a -inf bias).
+        if (kind != kHalfPooled) {
+          int valid = kBlock;
+          if (kind == kHalfMissing) {
+            valid = 0;
+          } else if (kind == kHalfDense) {
+            const int key0 = I.dense ? hi * kBlock : nv + (hi - I.cnt) * kBlock;
+            valid = min(kBlock, p.N - key0);
+          } else if (cur_bad) {
             const int bb = p.idx[I.row * (size_t)p.kcap + hi];
             if (bb < 0 || bb >= p.nb) valid = 0;
           }
-        } else if (hi < I.cnt + n_dk) {
-          valid = min(kBlock, p.N - (nv + (hi - I.cnt) * kBlock));
-        } else {
-          kind = 1;
-          j0 = (hi - I.cnt - n_dk) * kBlock;
-          valid = min(kBlock, p.nb - j0);
-        }
-        // Exact halves keep raw scores (the scale is folded into the exponent's FFMA);
-        // pooled halves become scale*logit + beta (base 2), with the selected blocks and
-        // entries past nb masked. The half's bias values are loaded up front, unconditionally
-        // (clamped index), so their latencies overlap.
-        if (kind == 0) {
           if (valid < kBlock) {
 #pragma unroll
             for (int j = 0; j < 64; ++j)
               if (j >= valid) x[j] = -INFINITY;
           }
-        } else {
-          const float* bp = p.beta + (size_t)I.bh * p.nb;
-          const int wb = j0 >> 5;  // j0 is a multiple of 64
-          const uint32_t w0 = bm[wb];
-          const uint32_t w1 = (j0 + 32 < p.nb) ? bm[wb + 1] : 0u;
+        }
+        if (any_pooled) {
+          tc::cp_async_wait<1>();  // this tile's biases have landed (the next tile's may not)
+          __syncwarp();
+        }
+        if (kind == kHalfPooled) {
+          const float4* bsrc = reinterpret_cast<const float4*>(bst + (t & 1) * 128 + h * 64);
+          const int j0 = (hi - I.cnt - n_dk) * kBlock;
+          const int wb = j0 >> 5;  // j0 is a multiple of 64, wb + 1 < nbwp
+          const uint32_t w0 = bm[wb], w1 = bm[wb + 1];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int qq = 0; qq < 4; ++qq) {
             float bv[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) bv[j] = __ldg(bp + min(j0 + 16 * q + j, p.nb - 1));
-            const uint32_t wm = (q < 2 ? w0 : w1) >> (16 * (q & 1));
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const bool m = (16 * q + j >= valid) || ((wm >> j) & 1u);
-              x[16 * q + j] = m ? -INFINITY : fmaf(x[16 * q + j], p.scale_log2, bv[j] * kLog2e);
+            for (int i = 0; i < 4; ++i) {
+              const float4 f = bsrc[4 * qq + i];
+              bv[4 * i] = f.x;
+              bv[4 * i + 1] = f.y;
+              bv[4 * i + 2] = f.z;
+              bv[4 * i + 3] = f.w;
             }
+            const uint32_t wm = (qq < 2 ? w0 : w1) >> (16 * (qq & 1));
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              x[16 * qq + j] = ((wm >> j) & 1u) ? -INFINITY : fmaf(x[16 * qq + j], p.scale_log2, bv[j]);
           }
         }
-        const float xs = kind == 0 ? p.scale_log2 : 1.0f;  // factor still to apply to x
-        SPARK_TC_ACC(14 + kind, t_cp);
+        const float xs = kind == kHalfPooled ? 1.0f : p.scale_log2;  // factor still to apply
+        SPARK_TC_ACC(14 + (kind == kHalfPooled), t_cp);
         SPARK_TC_T0(t_mx);
         // row max: 3-input max tree over this thread's 64 keys, then the partner half
         float mx;
@@ -720,15 +784,33 @@ __global__ void __launch_bounds__(352, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&pfull[2 * s + b]);
         SPARK_TC_ACC(8, t_st);
-        SPARK_TC_EV(1 + s, 41);
+        // ---- the previous item's epilogue, once this item's first P is on its way
+        if (t == 0 && have_prev) {
+          if (!epilogue(prev, m_prev, l_prev)) {
+            ok = false;
+            break;
+          }
+          have_prev = false;
+        }
+        // ---- next unit of the next item's preparation
+        if (prep_u < prep_units) {
+          prep_issue(prep_u);
+          prep_pend = prep_u++;
+        }
       }
       if (!ok) break;
-      have_prev = 1;
+      prep_flush();
       prev = I;
+      have_prev = true;
       m_prev = m_run;
       l_prev = l_run;
-      ++nitem;
+      cur_bad = bad_next;
+      bad_next = 0;
+      have = next_item(&I);
+      ++n;
     }
+    if (ok && have_prev) epilogue(prev, m_prev, l_prev);
+    tc::cp_async_wait<0>();
   }
 
   SPARK_TC_FLUSH

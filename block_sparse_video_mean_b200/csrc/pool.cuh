@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kPoolWarps * 32)
     pool_kv_kernel(const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
                    const float* __restrict__ anchor, float* __restrict__ k_pool,
                    float* __restrict__ v_summ, float* __restrict__ beta,
-                   uint16_t* __restrict__ k_pool16, uint16_t* __restrict__ v_summ16, int N, int nb,
-                   float scale, int mode) {
+                   uint16_t* __restrict__ k_pool16, uint16_t* __restrict__ v_summ16,
+                   float* __restrict__ beta_l2, int nbp, int N, int nb, float scale, int mode) {
   using L = RowLayout<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bi = blockIdx.x * kPoolWarps + warp;
@@ -198,8 +198,13 @@ __global__ void __launch_bounds__(kPoolWarps * 32)
     v16.z = pack_bf16x2(vacc[4], vacc[5]); v16.w = pack_bf16x2(vacc[6], vacc[7]);
     *reinterpret_cast<uint4*>(k_pool16 + o) = k16;
     *reinterpret_cast<uint4*>(v_summ16 + o) = v16;
-    if (lane == 0)
-      beta[bh * nb + bi] = (mode == SPARK_POOL_REWEIGHT) ? lse - dot * scale : logf((float)kBlock);
+    if (lane == 0) {
+      const float b = (mode == SPARK_POOL_REWEIGHT) ? lse - dot * scale : logf((float)kBlock);
+      beta[bh * nb + bi] = b;
+      // padded log2-scaled copy for the attention kernel; entries past nb are -inf
+      beta_l2[bh * nbp + bi] = b * kLog2e;
+      for (int j = nb + bi; j < nbp; j += nb) beta_l2[bh * nbp + j] = -INFINITY;
+    }
   }
 }
 

@@ -47,6 +47,11 @@ int check_shape(const spark_shape* s) {
 
 inline bool empty(const spark_shape* s) { return (int64_t)s->B * s->H * s->N == 0; }
 
+// Pool pack layout: bf16 k_pool [bh*nb, d], bf16 v_summ [bh*nb, d], then fp32
+// beta*log2(e) [bh, nbp] with nbp = nb rounded up to whole 64-entry tiles.
+inline size_t padded_blocks(size_t nb) { return (nb + kBlock - 1) / kBlock * kBlock; }
+inline size_t pack_bias_offset(size_t bh, size_t nb, int d) { return 2 * bh * nb * d * sizeof(uint16_t); }
+
 // Score rows a select CTA keeps in shared memory (largest of 8, 4, 2, 1 that fits).
 int select_rows_per_cta(int nb, int d, size_t* smem) {
   const size_t nbp = (size_t)((nb + 3) & ~3);
@@ -110,8 +115,7 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
     maps.kp = maps.k;
     maps.vp = maps.v;
   }
-  const size_t smem = 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes +
-                      8 * (size_t)((tp.nb + 31) / 32) * 4;  // one bitmap per softmax warp
+  const size_t smem = tc_smem_bytes<D>(tp.nb);
   if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
   const int sms = num_sms();
   if (sms <= 0) return SPARK_ECUDA;
@@ -172,7 +176,7 @@ size_t spark_workspace_bytes(const spark_shape* s, int call_id) {
   const size_t nb = (size_t)num_blocks(s);
   switch (call_id) {
     case SPARK_CALL_POOL:
-      return 2 * bh * nb * s->d * sizeof(uint16_t);
+      return pack_bias_offset(bh, nb, s->d) + bh * padded_blocks(nb) * sizeof(float);
     case SPARK_CALL_SELECT:
       return ((2 * bh * sizeof(double)) + 255) & ~(size_t)255;
     case SPARK_CALL_ATTN:
@@ -206,18 +210,21 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
   if (pool_pack_bytes < spark_workspace_bytes(s, SPARK_CALL_POOL)) return SPARK_EINVAL;
   uint16_t* k16 = static_cast<uint16_t*>(pool_pack);
   uint16_t* v16 = k16 + (size_t)bh * nb * s->d;
+  float* bl2 = reinterpret_cast<float*>(static_cast<unsigned char*>(pool_pack) +
+                                        pack_bias_offset(bh, nb, s->d));
+  const int nbp = (int)padded_blocks(nb);
   const float scale = eff_scale(s);
   dim3 grid((nb + kPoolWarps - 1) / kPoolWarps, bh);
   if (s->d == 128) {
     pool_q_kernel<128><<<grid, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nb);
     anchor_kernel<128><<<bh, 256, 0, cs>>>(q_pool, anchor, nb);
     pool_kv_kernel<128><<<grid, kPoolWarps * 32, 0, cs>>>(K, V, anchor, k_pool, v_summ, beta, k16,
-                                                          v16, s->N, nb, scale, pool_mode);
+                                                          v16, bl2, nbp, s->N, nb, scale, pool_mode);
   } else {
     pool_q_kernel<64><<<grid, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nb);
     anchor_kernel<64><<<bh, 256, 0, cs>>>(q_pool, anchor, nb);
     pool_kv_kernel<64><<<grid, kPoolWarps * 32, 0, cs>>>(K, V, anchor, k_pool, v_summ, beta, k16,
-                                                         v16, s->N, nb, scale, pool_mode);
+                                                         v16, bl2, nbp, s->N, nb, scale, pool_mode);
   }
   SPARK_LAUNCH_CHECK();
   note_launches(3);
@@ -321,7 +328,7 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SPARK_EINVAL;
   if (nb > 0) {
     if (!idx || !cnt || kcap < 1) return SPARK_EINVAL;
-    if (pool_pack && (!beta || !aligned16(pool_pack))) return SPARK_EINVAL;
+    if (pool_pack && !aligned16(pool_pack)) return SPARK_EINVAL;
   }
   const int nv = nb * kBlock;
   const int n_dq = (s->N - nv + kBlock - 1) / kBlock;
@@ -332,7 +339,12 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   tp.Q = Q;
   tp.idx = idx;
   tp.cnt = cnt;
-  tp.beta = beta;
+  (void)beta;  // the compressed branch reads the pool pack's padded copy
+  tp.bias = nullptr;
+  tp.nbp = (int)padded_blocks(nb);
+  if (nb > 0 && pool_pack != nullptr)
+    tp.bias = reinterpret_cast<const float*>(static_cast<const unsigned char*>(pool_pack) +
+                                             pack_bias_offset(bh, nb, s->d));
   tp.perm = perm;
   tp.O = O;
   tp.lse = lse;

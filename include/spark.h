@@ -73,7 +73,10 @@ int32_t spark_num_blocks(const spark_shape* s);
 
 /* Bytes of the caller-owned buffer that call `call_id` needs:
  *   SPARK_CALL_POOL    the pooled pack written by spark_pool_kv and read by
- *                      spark_attn_fwd (bf16 copies of kbar and vtil, 2*B*H*nb*d*2 bytes);
+ *                      spark_attn_fwd: bf16 copies of k_pool and v_summ ([B*H*nb, d]
+ *                      each) followed by beta * log2(e) in fp32 with each (b, h) row
+ *                      padded to nbp = 64 * ceil(nb / 64) entries (-inf past nb):
+ *                      2*B*H*nb*d*2 + B*H*nbp*4 bytes;
  *   SPARK_CALL_SELECT  scratch of spark_score_select (tau moments; 0 for top-k is fine
  *                      but the tau size is returned);
  *   SPARK_CALL_ATTN    scratch of spark_attn_fwd (0: it needs none);
@@ -94,8 +97,9 @@ int32_t spark_topk_count(double ratio, int32_t nb);
  *              v_summ[i]  = sum_j softmax_i(s)_j v_j (REWEIGHT) | mean v     fp32 [B,H,nb,d]
  *              beta[i]    = logsumexp_i(s) - anchor . k_pool[i] * scale      fp32 [B,H,nb]
  *                           (REWEIGHT) | log(64) (MEAN)
- * pool_pack (spark_workspace_bytes(s, SPARK_CALL_POOL) bytes) receives bf16 copies of
- * k_pool and v_summ, the operands of the compressed branch in spark_attn_fwd.
+ * pool_pack (spark_workspace_bytes(s, SPARK_CALL_POOL) bytes, 16-byte aligned) receives
+ * bf16 copies of k_pool and v_summ and a padded log2-scaled copy of beta, the operands
+ * of the compressed branch in spark_attn_fwd.
  * Any of q_pool/k_pool/v_summ/anchor may not be NULL; all are written. */
 int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                   int pool_mode, float* q_pool, float* k_pool, float* v_summ, float* beta,
@@ -123,7 +127,8 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
  * A video query of block i attends to the 64 keys of each selected block idx[i, :cnt[i]]
  * and to every dense key; when pool_pack is not NULL it also attends to one pooled
  * entry per unselected video block b, with logit q . k_pool[b] * scale + beta[b] and
- * value v_summ[b] (bf16 operands from pool_pack, beta fp32). Dense query rows attend
+ * value v_summ[b] (bf16 k_pool / v_summ and fp32 beta, all read from pool_pack; the
+ * `beta` argument is not read and may be NULL). Dense query rows attend
  * to every key and never to pooled entries. A row with nothing to attend to gets
  * O = 0 and LSE = -inf.
  * perm (nullable) int32 [B, H, nb*64]: the inputs are in a reblocked order and output

@@ -47,7 +47,8 @@ def test_topk_count_matches_fixture(spark):
 def test_num_blocks_and_workspace(spark):
     s = spark.make_shape(1, 24, 175680 + 512, 128, 512)
     assert spark.num_blocks(s) == 2745
-    assert spark.workspace_bytes(s, spark.CALL_POOL) == 2 * 24 * 2745 * 128 * 2
+    # bf16 k_pool and v_summ, then beta*log2(e) padded to 2752 = 43 x 64 entries per head
+    assert spark.workspace_bytes(s, spark.CALL_POOL) == 2 * 24 * 2745 * 128 * 2 + 24 * 2752 * 4
     assert spark.workspace_bytes(s, spark.CALL_ATTN) == 0
     ragged = spark.make_shape(1, 1, 64 * 3 + 17 + 5, 64, 5)
     assert spark.num_blocks(ragged) == 3
