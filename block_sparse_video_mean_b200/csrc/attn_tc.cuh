@@ -31,11 +31,10 @@
 //   128B-swizzled K tile), softmax in base 2 (each thread owns one half of one row) with a
 //   lazy running max (O is rescaled only when the row max grows by more than 2^8), P
 //   written back over S as bf16, then O += P V (8 MMAs 64xDx16, V as an MN-major operand).
-// * Item transitions stay off the tensor core's path: Q is double-buffered in TMEM and the
-//   next item's Q rows and selection bitmap are fetched a piece per tile during the
-//   current item (loads issued after a tile, consumed after the next tile's S is ready);
-//   the epilogue releases O as soon as it has read it. The compressed branch's biases are
-//   staged per tile into shared memory with cp.async, one tile ahead.
+// * Item transitions: Q is double-buffered in TMEM, so a slot's softmax warps store the
+//   next item's Q (and build its selection bitmap) right after the current item's last
+//   tile, while the other slot keeps the tensor pipe busy; the epilogue releases O as soon
+//   as it has read it. A pooled half's biases are warmed into L1 before its S wait.
 // * Every mbarrier wait is bounded; a timeout records SPARK_ETIMEOUT, raises the CTA abort
 //   flag, the TMA roles drain their copies in flight and TMEM is released.
 #pragma once
@@ -85,7 +84,6 @@ struct TcCfg {
   static constexpr int kThreads = 384;
   static constexpr int kRingBytes = 2 * kStages * kTileBytes;  // K ring, then V ring
   static constexpr int kBarBytes = 1024;
-  static constexpr int kBiasBytes = 8 * 2 * 512;   // per softmax warp: 2 tiles x 2 halves x 64 fp32
   static constexpr int kQPieces = D / 64;          // 16-word pieces of a thread's half Q row
 };
 
@@ -95,7 +93,7 @@ __host__ __device__ inline int tc_bitmap_words(int nb) { return ((nb + 31) / 32 
 template <int D>
 __host__ __device__ inline size_t tc_smem_bytes(int nb) {
   using C = TcCfg<D>;
-  return 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes + C::kBiasBytes +
+  return 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes +
          (size_t)8 * 2 * tc_bitmap_words(nb) * 4;  // two bitmaps per softmax warp
 }
 
@@ -157,6 +155,10 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
+}
+
 // Bounded wait that ignores the abort flag (used to drain copies in flight on abort).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -211,8 +213,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* finbar = odone + 2;            // [slot]: all MMAs of that slot's issuer done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* bias_stage = reinterpret_cast<float*>(ring + C::kRingBytes + C::kBarBytes);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes + C::kBiasBytes);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   SPARK_TC_DECL
@@ -256,6 +257,11 @@ __global__ void __launch_bounds__(384, 1)
   const int nv = p.nb * kBlock;
   const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
 
+  // Registers: launched at 168 per thread (384 threads). The producer / issuer warpgroup
+  // (warps 8-11) gives back down to 104 so the two softmax warpgroups (about 186 needed)
+  // can grow to 200: 128 x 104 + 256 x 200 = 64,512 = 384 x 168.
+  if (warp >= 8) {
+  tc::regs_dec<104>();
   if (warp == 8 || warp == 10) {
     // ================================================================ TMA producers
     // warp 8 fills the K ring, warp 10 the V ring, both in the same tile order: per round,
@@ -379,10 +385,17 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       auto issue_pv = [&]() -> bool {
         const uint32_t b = pg & 1;
+        SPARK_TC_T0(t_pw);
         if (!tc::mbar_wait(&pfull[2 * s + b], (pg >> 1) & 1, abort_flag)) return false;
+        SPARK_TC_ACC(0, t_pw);
         const int stage = pq % C::kStages;
+        SPARK_TC_T0(t_vw);
         if (!tc::mbar_wait(&vfull[stage], (pq / C::kStages) & 1, abort_flag)) return false;
+        SPARK_TC_ACC(1, t_vw);
+        SPARK_TC_T0(t_ow);
         if (pfirst && pitem > 0 && !tc::mbar_wait(&ofree[s], (pitem - 1) & 1, abort_flag)) return false;
+        SPARK_TC_ACC(9, t_ow);
+        SPARK_TC_T0(t_pv);
         tc::tc_fence_after();
         const uint32_t st = vring_addr + stage * C::kTileBytes;
 #pragma unroll
@@ -392,6 +405,7 @@ __global__ void __launch_bounds__(384, 1)
         tc::mma_commit(&vempty[stage]);
         tc::mma_commit(&oready[s]);
         if (plast) tc::mma_commit(&odone[s]);
+        SPARK_TC_ACC(10, t_pv);
         return true;
       };
       uint32_t q = 0;  // ring position of the producers' next tile
@@ -401,12 +415,17 @@ __global__ void __launch_bounds__(384, 1)
           if (ok && have[o]) {
             if (o == s) {
               const uint32_t qb = nitem & 1;
+              SPARK_TC_T0(t_qw);
               bool good = t[o] != 0 || tc::mbar_wait(&qfull[2 * s + qb], (nitem >> 1) & 1, abort_flag);
+              SPARK_TC_ACC(3, t_qw);
               const int stage = q % C::kStages;
+              SPARK_TC_T0(t_kw);
               good = good && tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag);
+              SPARK_TC_ACC(2, t_kw);
               if (!good) {
                 ok = false;
               } else {
+                SPARK_TC_T0(t_si);
                 tc::tc_fence_after();
                 const uint32_t b = g & 1;
                 const uint32_t st = ring_addr + stage * C::kTileBytes;
@@ -417,6 +436,7 @@ __global__ void __launch_bounds__(384, 1)
                              tc_kdesc<D>(st, kk), idS, kk > 0 ? 1u : 0u);
                 tc::mma_commit(&sfull[2 * s + b]);
                 tc::mma_commit(&kempty[stage]);
+                SPARK_TC_ACC(11, t_si);
                 // then the PV of the previous tile of this slot
                 if (pend) ok = issue_pv();
                 pend = true;
@@ -444,7 +464,9 @@ __global__ void __launch_bounds__(384, 1)
       tc::mma_commit(&finbar[s]);
       mbar_drain(&finbar[s], 0);
     }
+  }
   } else {
+    tc::regs_inc<200>();
     // ================================================================ softmax (slot s)
     const int s = warp >> 2;
     const int w = warp & 3;
@@ -454,73 +476,54 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lanes = (uint32_t)(32 * w + 16 * s) << 16;
     const int nbwp = tc_bitmap_words(p.nb);
     uint32_t* bm2 = bitmap + warp * 2 * nbwp;  // this warp's two selection bitmaps
-    float* bst = bias_stage + warp * 256;       // [tile parity][half][64] pooled biases
     bool ok = true;
 
-    // ---- preparation of an item, a unit per tile: the thread's Q half row in kQPieces
-    //      16-word pieces into a TMEM Q buffer, then the selection bitmap from its index
-    //      row, 128 indices per unit. Loads are issued after a tile and consumed after
-    //      the next tile's S is ready, so their latency hides behind that wait.
-    TcItem J;                 // the item being prepared
-    int prep_qb = 0, prep_units = 0, prep_u = 0, prep_pend = -1;
-    int bad_next = 0;         // J has a block index out of range
-    uint32_t pf[16];
-    auto prep_setup = [&](const TcItem& It, int qb) {
-      J = It;
-      prep_qb = qb;
-      const bool need_bm = !It.dense && (p.pooled || It.cnt > 0);
-      prep_units = C::kQPieces + (need_bm ? max(1, (It.cnt + 127) / 128) : 0);
-      prep_u = 0;
-      prep_pend = -1;
-    };
-    auto prep_issue = [&](int u) {
-      if (u < C::kQPieces) {
+    // ---- preparation of an item: the thread's Q half row into a TMEM Q buffer (then
+    //      qfull), and the warp's selection bitmap from the item's index row. Runs at the
+    //      end of the previous item; the other slot's MMAs keep the tensor pipe busy.
+    int bad_next = 0;  // the prepared item has a block index out of range
+    auto prepare = [&](const TcItem& J, int qb) {
+      {
         const bool rv = r < J.nq;
-        const uint16_t* qrow =
-            p.Q + ((size_t)J.bh * p.N + J.q0 + (rv ? r : 0)) * D + h * (D / 2) + 32 * u;
+        const uint16_t* qrow = p.Q + ((size_t)J.bh * p.N + J.q0 + (rv ? r : 0)) * D + h * (D / 2);
+        uint32_t qv[D / 4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < D / 16; ++i) {
           const uint4 a = rv ? ldg_nc_v4(qrow + 8 * i) : make_uint4(0, 0, 0, 0);
-          pf[4 * i] = a.x;
-          pf[4 * i + 1] = a.y;
-          pf[4 * i + 2] = a.z;
-          pf[4 * i + 3] = a.w;
+          qv[4 * i] = a.x;
+          qv[4 * i + 1] = a.y;
+          qv[4 * i + 2] = a.z;
+          qv[4 * i + 3] = a.w;
         }
-      } else {
-        const int c = u - C::kQPieces;
-        const int32_t* ip = p.idx + J.row * (size_t)p.kcap;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = 128 * c + 32 * i + lane;
-          pf[i] = j < J.cnt ? (uint32_t)ip[j] : 0u;
-        }
+        for (int c = 0; c < C::kQPieces; ++c)
+          tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + qb * (D / 2) + 16 * c, qv + 16 * c);
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&qfull[2 * s + qb]);
       }
-    };
-    auto prep_consume = [&](int u) {
-      if (u < C::kQPieces) {
-        tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + prep_qb * (D / 2) + 16 * u, pf);
-        if (u == C::kQPieces - 1) {
-          tc::tmem_wait_st();
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&qfull[2 * s + prep_qb]);
-        }
-      } else {
-        const int c = u - C::kQPieces;
-        uint32_t* bm = bm2 + prep_qb * nbwp;
-        if (c == 0) {
-          for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
-          __syncwarp();
-          if (lane == 0 && w == 0 && p.cnt[J.row] != J.cnt) set_error(SPARK_EDEVICE_INDEX);
-        }
+      if (!J.dense && (p.pooled || J.cnt > 0)) {
+        uint32_t* bm = bm2 + qb * nbwp;
+        for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
+        __syncwarp();
+        if (lane == 0 && w == 0 && p.cnt[J.row] != J.cnt) set_error(SPARK_EDEVICE_INDEX);
+        const int32_t* ip = p.idx + J.row * (size_t)p.kcap;
         int bad = 0;
+        for (int j0 = 0; j0 < J.cnt; j0 += 128) {
+          int bv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = 128 * c + 32 * i + lane;
-          const int b = (int)pf[i];
-          if (j < J.cnt) {
-            if (b >= 0 && b < p.nb) atomicOr(&bm[b >> 5], 1u << (b & 31));
-            else bad = 1;
+          for (int i = 0; i < 4; ++i) {
+            const int j = j0 + 32 * i + lane;
+            bv[i] = j < J.cnt ? ip[j] : 0;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = j0 + 32 * i + lane;
+            if (j < J.cnt) {
+              if (bv[i] >= 0 && bv[i] < p.nb) atomicOr(&bm[bv[i] >> 5], 1u << (bv[i] & 31));
+              else bad = 1;
+            }
           }
         }
         if (__any_sync(0xffffffffu, bad)) {
@@ -529,27 +532,6 @@ __global__ void __launch_bounds__(384, 1)
         }
         __syncwarp();
       }
-    };
-    auto prep_flush = [&]() {
-      if (prep_pend >= 0) {
-        prep_consume(prep_pend);
-        prep_pend = -1;
-      }
-      for (; prep_u < prep_units; ++prep_u) {
-        prep_issue(prep_u);
-        prep_consume(prep_u);
-      }
-    };
-    // Pooled biases of half h of tile tt into the staging buffer of tt's parity (one
-    // cp.async group per call, empty when the half is not pooled).
-    auto stage_bias = [&](const TcItem& It, int tt) {
-      const int hi = 2 * tt + h;
-      if (tt < It.ntiles && tc_half_kind(It, hi, n_dk) == kHalfPooled) {
-        const int j0 = (hi - It.cnt - n_dk) * kBlock;
-        tc::cp_async_16(bst + (tt & 1) * 128 + h * 64 + 4 * lh,
-                        p.bias + (size_t)It.bh * p.nbp + j0 + 4 * lh);
-      }
-      tc::cp_async_commit();
     };
 
     uint32_t ndone = 0;  // non-empty items whose epilogue ran
@@ -630,23 +612,23 @@ __global__ void __launch_bounds__(384, 1)
     float m_prev = -INFINITY, l_prev = 0.f;
     bool have = next_item(&I);
     TcSlotWalk ahead = walk;  // finds the next non-empty item one ahead
-    if (have) {
-      prep_setup(I, 0);
-      prep_flush();
-    }
+    if (have) prepare(I, 0);
     int cur_bad = bad_next;
     bad_next = 0;
     while (ok && have) {
       TcItem nxt;
-      if (ahead.next_nonempty(p, &nxt)) prep_setup(nxt, (n + 1) & 1);
-      else prep_units = prep_u = 0, prep_pend = -1;
+      const bool have_nxt = ahead.next_nonempty(p, &nxt);
       const uint32_t* bm = bm2 + (n & 1) * nbwp;
 
       float m_run = -INFINITY, l_run = 0.f;
       for (int t = 0; t < I.ntiles; ++t, ++g) {
         const uint32_t b = g & 1;
-        if (t == 0) stage_bias(I, 0);
-        stage_bias(I, t + 1);
+        // warm L1 with the biases of a pooled half (their loads follow the S wait)
+        const int hi = 2 * t + h;
+        const int kind = tc_half_kind(I, hi, n_dk);
+        const float* bias_src =
+            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk) * kBlock : 0);
+        if (kind == kHalfPooled && lh < 2) prefetch_l1(bias_src + 32 * lh);
         SPARK_TC_T0(t_sw);
         if (!tc::mbar_wait(&sfull[2 * s + b], (g >> 1) & 1, abort_flag)) {
           ok = false;
@@ -654,10 +636,6 @@ __global__ void __launch_bounds__(384, 1)
         }
         SPARK_TC_ACC(5, t_sw);
         tc::tc_fence_after();
-        if (prep_pend >= 0) {
-          prep_consume(prep_pend);
-          prep_pend = -1;
-        }
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h+63 of the S buffer)
         float x[64];
         SPARK_TC_T0(t_ld);
@@ -669,10 +647,6 @@ __global__ void __launch_bounds__(384, 1)
         SPARK_TC_ACC(6, t_ld);
         SPARK_TC_T0(t_cp);
         // ---- logits (base 2) and masks of this half
-        const int hi = 2 * t + h;
-        const int kind = tc_half_kind(I, hi, n_dk);
-        const bool any_pooled = tc_half_kind(I, 2 * t, n_dk) == kHalfPooled ||
-                                tc_half_kind(I, 2 * t + 1, n_dk) == kHalfPooled;  // warp-uniform
         // Exact and dense halves keep raw scores (the scale is folded into the exponent's
         // FFMA); pooled halves become scale*logit + beta*log2(e), with the selected blocks
         // masked (entries past nb carry a -inf bias).
@@ -693,12 +667,8 @@ __global__ void __launch_bounds__(384, 1)
               if (j >= valid) x[j] = -INFINITY;
           }
         }
-        if (any_pooled) {
-          tc::cp_async_wait<1>();  // this tile's biases have landed (the next tile's may not)
-          __syncwarp();
-        }
         if (kind == kHalfPooled) {
-          const float4* bsrc = reinterpret_cast<const float4*>(bst + (t & 1) * 128 + h * 64);
+          const float4* bsrc = reinterpret_cast<const float4*>(bias_src);
           const int j0 = (hi - I.cnt - n_dk) * kBlock;
           const int wb = j0 >> 5;  // j0 is a multiple of 64, wb + 1 < nbwp
           const uint32_t w0 = bm[wb], w1 = bm[wb + 1];
@@ -707,7 +677,7 @@ __global__ void __launch_bounds__(384, 1)
             float bv[16];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const float4 f = bsrc[4 * qq + i];
+              const float4 f = __ldg(bsrc + 4 * qq + i);
               bv[4 * i] = f.x;
               bv[4 * i + 1] = f.y;
               bv[4 * i + 2] = f.z;
@@ -763,22 +733,27 @@ __global__ void __launch_bounds__(384, 1)
         SPARK_TC_ACC(16, t_mx);
         SPARK_TC_T0(t_ex);
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        uint32_t pk[32];
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // P over S (packed columns 32h .. 32h+31 of the buffer), 32 keys at a time
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2f(fmaf(x[2 * j], xs, -m_use));
-          const float p1 = ex2f(fmaf(x[2 * j + 1], xs, -m_use));
-          ls[j & 3] += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int e = 32 * hc + 2 * j;
+            const float a0 = fmaf(x[e], xs, -m_use);
+            const float a1 = fmaf(x[e + 1], xs, -m_use);
+            const float p0 = ex2f(a0);
+            const float p1 = ex2f(a1);
+            ls[j & 3] += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
+          }
+          tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         SPARK_TC_ACC(17, t_ex);
         SPARK_TC_ACC(7, t_cp);
         SPARK_TC_T0(t_st);
-        // P over S: packed columns 32h .. 32h+31 of the buffer
-        tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b, pk);
-        tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b + 16, pk + 16);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
@@ -792,14 +767,9 @@ __global__ void __launch_bounds__(384, 1)
           }
           have_prev = false;
         }
-        // ---- next unit of the next item's preparation
-        if (prep_u < prep_units) {
-          prep_issue(prep_u);
-          prep_pend = prep_u++;
-        }
       }
       if (!ok) break;
-      prep_flush();
+      if (have_nxt) prepare(nxt, (n + 1) & 1);
       prev = I;
       have_prev = true;
       m_prev = m_run;
@@ -810,7 +780,6 @@ __global__ void __launch_bounds__(384, 1)
       ++n;
     }
     if (ok && have_prev) epilogue(prev, m_prev, l_prev);
-    tc::cp_async_wait<0>();
   }
 
   SPARK_TC_FLUSH
