@@ -121,6 +121,98 @@ struct SelectParams {
   float scale;
 };
 
+// One warp selects the kept blocks of one score row kr[0 .. nb) (order-preserving keys):
+// top-k by a 4-pass MSB radix select over a warp-private 256-bin histogram h, or the
+// head's tau threshold; writes the ascending indices of the kept blocks to row orow of
+// idx (at most kcap) and their count to cnt[orow].
+__device__ __forceinline__ void select_row_warp(const SelectParams& p, const uint32_t* kr,
+                                                size_t bh, size_t orow, uint32_t* h, int lane) {
+  const int nb = p.nb;
+  int32_t* out = p.idx + orow * (size_t)p.kcap;
+  uint32_t T = 0;
+  int take_eq = 0;  // number of elements equal to T to keep (lowest indices first)
+  const bool use_thr = (p.mode == SPARK_SELECT_TAU);
+  const double thr = use_thr ? p.thr[bh] : 0.0;
+  if (!use_thr) {
+    uint32_t prefix = 0, mask = 0;
+    int kk = p.k;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int b = lane; b < 256; b += 32) h[b] = 0;
+      __syncwarp();
+      for (int j = lane; j < nb; j += 32) {
+        const uint32_t key = kr[j];
+        if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      // lane l owns bins 255-8l .. 248-8l (descending); find the bin where the count
+      // from the top reaches kk.
+      uint32_t cntb[8];
+      uint32_t tot = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        cntb[t] = h[255 - 8 * lane - t];
+        tot += cntb[t];
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const uint32_t excl = incl - tot;
+      const bool mine = excl < (uint32_t)kk && (uint32_t)kk <= incl;
+      const uint32_t who = __ballot_sync(0xffffffffu, mine);
+      const int src = __ffs(who) - 1;
+      int bin = 0, above = 0;
+      if (lane == src) {
+        uint32_t run = excl;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (run + cntb[t] >= (uint32_t)kk) {
+            bin = 255 - 8 * lane - t;
+            above = (int)run;
+            break;
+          }
+          run += cntb[t];
+        }
+      }
+      bin = __shfl_sync(0xffffffffu, bin, src);
+      above = __shfl_sync(0xffffffffu, above, src);
+      kk -= above;
+      prefix |= (uint32_t)bin << shift;
+      mask |= 255u << shift;
+      __syncwarp();
+    }
+    T = prefix;
+    take_eq = kk;
+  }
+  // ---- ascending output pass
+  int written = 0, eq_seen = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    bool keep = false;
+    if (use_thr) {
+      keep = j < nb && (double)key_to_float(kr[j]) > thr;
+    } else {
+      const uint32_t key = j < nb ? kr[j] : 0u;
+      const bool eq = j < nb && key == T;
+      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+      const int rank = eq_seen + __popc(eqm & lanemask_lt());
+      eq_seen += __popc(eqm);
+      keep = j < nb && (key > T || (eq && rank < take_eq));
+    }
+    const uint32_t km = __ballot_sync(0xffffffffu, keep);
+    const int pos = written + __popc(km & lanemask_lt());
+    if (keep && pos < p.kcap) out[pos] = j;
+    written += __popc(km);
+  }
+  if (lane == 0) {
+    if (written > p.kcap) set_error(SPARK_ECAPACITY);
+    p.cnt[orow] = min(written, p.kcap);
+  }
+}
+
 // Dynamic shared memory: keys[rt][nbp] | qs[rt][D] | kt[D][kSelKT] | hist[8][256].
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams p) {
@@ -167,93 +259,118 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
 
   // ---- selection: warp w handles rows w, w + 8, ...
   uint32_t* h = hist + warp * 256;
-  for (int r = warp; r < nrows; r += kSelThreads / 32) {
-    const uint32_t* kr = keys + (size_t)r * nbp;
-    const size_t orow = bh * (size_t)nb + row0 + r;
-    int32_t* out = p.idx + orow * (size_t)p.kcap;
-    uint32_t T = 0;
-    int take_eq = 0;  // number of elements equal to T to keep (lowest indices first)
-    bool use_thr = (p.mode == SPARK_SELECT_TAU);
-    double thr = use_thr ? p.thr[bh] : 0.0;
-    if (!use_thr) {
-      uint32_t prefix = 0, mask = 0;
-      int kk = p.k;
-      for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int b = lane; b < 256; b += 32) h[b] = 0;
-        __syncwarp();
-        for (int j = lane; j < nb; j += 32) {
-          const uint32_t key = kr[j];
-          if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
-        }
-        __syncwarp();
-        // lane l owns bins 255-8l .. 248-8l (descending); find the bin where the count
-        // from the top reaches kk.
-        uint32_t cntb[8];
-        uint32_t tot = 0;
+  for (int r = warp; r < nrows; r += kSelThreads / 32)
+    select_row_warp(p, keys + (size_t)r * nbp, bh, bh * (size_t)nb + row0 + r, h, lane);
+}
+
+// ---------------------------------------------------------------- scores, tiled
+// Score tile of 64 query blocks x 128 key blocks of one head, written as order-preserving
+// keys to skeys[bh][i][j] (row stride nbp). fp32 FMA with register tiling: each thread
+// owns 4 rows x 8 columns; the d dimension is staged 32 at a time, transposed, so a
+// thread reads its 4 q values and 8 k values of one d with three 16-byte loads. Every
+// score sums its even and its odd d terms in two chains, in increasing d, as the fused
+// kernel does.
+constexpr int kScI = 64, kScJ = 128, kScDC = 32;
+
+template <int D>
+__global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict__ q_pool,
+                                                         const float* __restrict__ k_pool, int nb,
+                                                         int nbp, float scale,
+                                                         uint32_t* __restrict__ skeys) {
+  __shared__ __align__(16) float qs[kScDC][kScI];
+  __shared__ __align__(16) float ks[kScDC][kScJ];
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+  const size_t bh = blockIdx.z;
+  const int i0 = blockIdx.y * kScI, j0 = blockIdx.x * kScJ;
+  const float* qp = q_pool + bh * (size_t)nb * D;
+  const float* kp = k_pool + bh * (size_t)nb * D;
+  float acc0[4][8], acc1[4][8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          cntb[t] = h[255 - 8 * lane - t];
-          tot += cntb[t];
-        }
-        uint32_t incl = tot;
+  for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += o;
-        }
-        const uint32_t excl = incl - tot;
-        const bool mine = excl < (uint32_t)kk && (uint32_t)kk <= incl;
-        const uint32_t who = __ballot_sync(0xffffffffu, mine);
-        const int src = __ffs(who) - 1;
-        int bin = 0, above = 0;
-        if (lane == src) {
-          uint32_t run = excl;
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            if (run + cntb[t] >= (uint32_t)kk) {
-              bin = 255 - 8 * lane - t;
-              above = (int)run;
-              break;
-            }
-            run += cntb[t];
-          }
-        }
-        bin = __shfl_sync(0xffffffffu, bin, src);
-        above = __shfl_sync(0xffffffffu, above, src);
-        kk -= above;
-        prefix |= (uint32_t)bin << shift;
-        mask |= 255u << shift;
-        __syncwarp();
-      }
-      T = prefix;
-      take_eq = kk;
+    for (int u = 0; u < 8; ++u) acc0[r][u] = acc1[r][u] = 0.f;
+  for (int d0 = 0; d0 < D; d0 += kScDC) {
+    __syncthreads();
+    // stage q rows i0.. (64 x 32) and k rows j0.. (128 x 32), transposed to [d][row]
+    for (int e = tid; e < kScI * kScDC / 4; e += 256) {
+      const int rr = e / (kScDC / 4), cc = (e % (kScDC / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i0 + rr < nb) v = *reinterpret_cast<const float4*>(qp + (size_t)(i0 + rr) * D + d0 + cc);
+      qs[cc][rr] = v.x;
+      qs[cc + 1][rr] = v.y;
+      qs[cc + 2][rr] = v.z;
+      qs[cc + 3][rr] = v.w;
     }
-    // ---- ascending output pass
-    int written = 0, eq_seen = 0;
-    for (int j0 = 0; j0 < nb; j0 += 32) {
-      const int j = j0 + lane;
-      bool keep = false;
-      if (use_thr) {
-        keep = j < nb && (double)key_to_float(kr[j]) > thr;
-      } else {
-        const uint32_t key = j < nb ? kr[j] : 0u;
-        const bool eq = j < nb && key == T;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-        const int rank = eq_seen + __popc(eqm & lanemask_lt());
-        eq_seen += __popc(eqm);
-        keep = j < nb && (key > T || (eq && rank < take_eq));
-      }
-      const uint32_t km = __ballot_sync(0xffffffffu, keep);
-      const int pos = written + __popc(km & lanemask_lt());
-      if (keep && pos < p.kcap) out[pos] = j;
-      written += __popc(km);
+    for (int e = tid; e < kScJ * kScDC / 4; e += 256) {
+      const int rr = e / (kScDC / 4), cc = (e % (kScDC / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j0 + rr < nb) v = *reinterpret_cast<const float4*>(kp + (size_t)(j0 + rr) * D + d0 + cc);
+      ks[cc][rr] = v.x;
+      ks[cc + 1][rr] = v.y;
+      ks[cc + 2][rr] = v.z;
+      ks[cc + 3][rr] = v.w;
     }
-    if (lane == 0) {
-      if (written > p.kcap) set_error(SPARK_ECAPACITY);
-      p.cnt[orow] = min(written, p.kcap);
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kScDC; c += 2) {
+      const float4 qa = *reinterpret_cast<const float4*>(&qs[c][4 * ty]);
+      const float4 qb = *reinterpret_cast<const float4*>(&qs[c + 1][4 * ty]);
+      const float4 ka0 = *reinterpret_cast<const float4*>(&ks[c][4 * tx]);
+      const float4 ka1 = *reinterpret_cast<const float4*>(&ks[c][64 + 4 * tx]);
+      const float4 kb0 = *reinterpret_cast<const float4*>(&ks[c + 1][4 * tx]);
+      const float4 kb1 = *reinterpret_cast<const float4*>(&ks[c + 1][64 + 4 * tx]);
+      const float q0[4] = {qa.x, qa.y, qa.z, qa.w}, q1[4] = {qb.x, qb.y, qb.z, qb.w};
+      const float k0[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+      const float k1[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          acc0[r][u] = fmaf(q0[r], k0[u], acc0[r][u]);
+          acc1[r][u] = fmaf(q1[r], k1[u], acc1[r][u]);
+        }
     }
   }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + 4 * ty + r;
+    if (i >= nb) continue;
+    uint32_t* dst = skeys + (bh * (size_t)nb + i) * nbp;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int j = j0 + 64 * half + 4 * tx;
+      uint32_t kv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kv[e] = float_to_key((acc0[r][4 * half + e] + acc1[r][4 * half + e]) * scale);
+      if (j + 3 < nbp) {
+        *reinterpret_cast<uint4*>(dst + j) = make_uint4(kv[0], kv[1], kv[2], kv[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (j + e < nbp) dst[j + e] = kv[e];
+      }
+    }
+  }
+}
+
+// Selection from materialised score rows: warp w of a CTA takes row 8 * blockIdx.x + w of
+// head blockIdx.y, copies it to shared memory and selects (select_row_warp).
+__global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p,
+                                                          const uint32_t* __restrict__ skeys,
+                                                          int nbp) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* rows = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* hist = rows + 8 * (size_t)nbp;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t bh = blockIdx.y;
+  const int i = blockIdx.x * 8 + warp;
+  if (i >= p.nb) return;
+  uint32_t* kr = rows + (size_t)warp * nbp;
+  const uint4* src = reinterpret_cast<const uint4*>(skeys + (bh * (size_t)p.nb + i) * nbp);
+  for (int e = lane; e < nbp / 4; e += 32) reinterpret_cast<uint4*>(kr)[e] = src[e];
+  __syncwarp();
+  select_row_warp(p, kr, bh, bh * (size_t)p.nb + i, hist + warp * 256, lane);
 }
 
 }  // namespace spark

@@ -52,6 +52,11 @@ inline bool empty(const spark_shape* s) { return (int64_t)s->B * s->H * s->N == 
 inline size_t padded_blocks(size_t nb) { return (nb + kBlock - 1) / kBlock * kBlock; }
 inline size_t pack_bias_offset(size_t bh, size_t nb, int d) { return 2 * bh * nb * d * sizeof(uint16_t); }
 
+// Select workspace layout: fp64 tau moments [bh] and thresholds [bh], then (256-byte
+// aligned) the score keys [bh][nb][nbp] with nbp = nb rounded up to 4.
+inline size_t select_row_stride(size_t nb) { return (nb + 3) & ~(size_t)3; }
+inline size_t select_scores_offset(size_t bh) { return ((2 * bh * sizeof(double)) + 255) & ~(size_t)255; }
+
 // Score rows a select CTA keeps in shared memory (largest of 8, 4, 2, 1 that fits).
 int select_rows_per_cta(int nb, int d, size_t* smem) {
   const size_t nbp = (size_t)((nb + 3) & ~3);
@@ -178,7 +183,7 @@ size_t spark_workspace_bytes(const spark_shape* s, int call_id) {
     case SPARK_CALL_POOL:
       return pack_bias_offset(bh, nb, s->d) + bh * padded_blocks(nb) * sizeof(float);
     case SPARK_CALL_SELECT:
-      return ((2 * bh * sizeof(double)) + 255) & ~(size_t)255;
+      return select_scores_offset(bh) + bh * nb * select_row_stride(nb) * sizeof(uint32_t);
     case SPARK_CALL_ATTN:
       return 0;
     case SPARK_CALL_REBLOCK:
@@ -231,9 +236,16 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
   return SPARK_OK;
 }
 
-int spark_score_select(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
-                       double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
-                       size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Scores + selection. `fused`: one kernel keeps each CTA's score rows in shared memory
+// (scratch: the tau moments only); otherwise the scores are first written to the
+// caller's workspace by a tiled kernel and rows are selected from there.
+int score_select_impl(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
+                      double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
+                      size_t ws_bytes, void* stream, bool fused) {
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   const int nb = (int)num_blocks(s);
@@ -259,9 +271,10 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
   cudaStream_t cs = as_stream(stream);
   const float scale = eff_scale(s);
   double* thr = nullptr;
+  const size_t need = fused ? select_scores_offset(bh) : spark_workspace_bytes(s, SPARK_CALL_SELECT);
+  if ((mode == SPARK_SELECT_TAU || !fused) && (!ws || ws_bytes < need || !aligned16(ws)))
+    return SPARK_EINVAL;
   if (mode == SPARK_SELECT_TAU) {
-    if (!ws || ws_bytes < spark_workspace_bytes(s, SPARK_CALL_SELECT) || !aligned16(ws))
-      return SPARK_EINVAL;
     double* acc = static_cast<double*>(ws);
     thr = acc + bh;
     if (cudaMemsetAsync(acc, 0, (size_t)bh * sizeof(double), cs) != cudaSuccess) return SPARK_ECUDA;
@@ -287,6 +300,22 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
   sp.mode = mode;
   sp.rt = rt;
   sp.scale = scale;
+  if (!fused) {
+    const int nbp = (int)select_row_stride(nb);
+    uint32_t* skeys = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + select_scores_offset(bh));
+    dim3 gs((nb + kScJ - 1) / kScJ, (nb + kScI - 1) / kScI, bh);
+    if (s->d == 128)
+      score_tile_kernel<128><<<gs, 256, 0, cs>>>(q_pool, k_pool, nb, nbp, scale, skeys);
+    else
+      score_tile_kernel<64><<<gs, 256, 0, cs>>>(q_pool, k_pool, nb, nbp, scale, skeys);
+    const size_t smem_sel = (size_t)8 * nbp * 4 + 8 * 256 * 4;
+    if (smem_sel > 227 * 1024) return SPARK_EUNSUPPORTED;
+    cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_sel);
+    select_rows_kernel<<<dim3((nb + 7) / 8, bh), 256, smem_sel, cs>>>(sp, skeys, nbp);
+    SPARK_LAUNCH_CHECK();
+    note_launches(2);
+    return SPARK_OK;
+  }
   dim3 grid((nb + rt - 1) / rt, bh);
   if (s->d == 128) {
     cudaFuncSetAttribute(score_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -300,6 +329,17 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
   return SPARK_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int spark_score_select(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
+                       double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
+                       size_t ws_bytes, void* stream) {
+  return score_select_impl(s, q_pool, k_pool, mode, param, kcap, idx, cnt, ws, ws_bytes, stream,
+                           /*fused=*/false);
+}
+
 int spark_score_select_noalloc(const spark_shape* s, const float* q_pool, const float* k_pool,
                                int mode, double param, int32_t kcap, int32_t* idx, int32_t* cnt,
                                void* stream) {
@@ -309,8 +349,8 @@ int spark_score_select_noalloc(const spark_shape* s, const float* q_pool, const 
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != SPARK_OK) return st;
-  return spark_score_select(s, q_pool, k_pool, mode, param, kcap, idx, cnt, scratch,
-                            sizeof(g_noalloc_select_scratch), stream);
+  return score_select_impl(s, q_pool, k_pool, mode, param, kcap, idx, cnt, scratch,
+                           sizeof(g_noalloc_select_scratch), stream, /*fused=*/true);
 }
 
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,

@@ -174,7 +174,7 @@ def score_select(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, 
     if out is None:
         out = (torch.empty((B, H, nb, max(kcap, 1)), dtype=torch.int32, device=dev),
                torch.empty((B, H, nb), dtype=torch.int32, device=dev))
-    if ws is None and mode == SELECT_TAU:
+    if ws is None:
         ws = torch.empty(max(workspace_bytes(shape, CALL_SELECT), 16), dtype=torch.uint8, device=dev)
     idx, cnt = out
     _check(load().spark_score_select(ctypes.byref(shape), _ptr(q_pool), _ptr(k_pool), int(mode),

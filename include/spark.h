@@ -77,8 +77,9 @@ int32_t spark_num_blocks(const spark_shape* s);
  *                      each) followed by beta * log2(e) in fp32 with each (b, h) row
  *                      padded to nbp = 64 * ceil(nb / 64) entries (-inf past nb):
  *                      2*B*H*nb*d*2 + B*H*nbp*4 bytes;
- *   SPARK_CALL_SELECT  scratch of spark_score_select (tau moments; 0 for top-k is fine
- *                      but the tau size is returned);
+ *   SPARK_CALL_SELECT  scratch of spark_score_select: fp64 tau moments (2*B*H doubles,
+ *                      padded to 256 bytes) and the score keys of every head
+ *                      (B*H*nb*nbp uint32, nbp = nb rounded up to 4);
  *   SPARK_CALL_ATTN    scratch of spark_attn_fwd (0: it needs none);
  *   SPARK_CALL_REBLOCK scratch of spark_reblock.
  * Returns 0 for an invalid shape or call id. */
@@ -117,7 +118,9 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
  *       kcap indices and records SPARK_ECAPACITY (kcap = nb never overflows).
  * Outputs: idx int32 [B, H, nb, kcap] (per row, ascending block indices in the first
  * cnt slots; later slots unspecified), cnt int32 [B, H, nb].
- * ws: spark_workspace_bytes(s, SPARK_CALL_SELECT) bytes (tau only; may be NULL for top-k). */
+ * The scores are computed by a tiled fp32 kernel into ws and each row is selected from
+ * there (per score: even and odd d terms in two fp32 chains, then scaled).
+ * ws: spark_workspace_bytes(s, SPARK_CALL_SELECT) bytes, 16-byte aligned (both modes). */
 int spark_score_select(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
                        double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
                        size_t ws_bytes, void* stream);
@@ -161,11 +164,12 @@ int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
  * memory of their own (the paper has no counterpart; this is a library convenience).
  * Some hosts own every byte of device memory up front - an engine that hands out one
  * arena at start-up, a plugin running inside another framework's allocator, a real-time
- * loop that must never reach the driver's allocator - and so cannot provide the tau-mode
- * moment scratch that spark_score_select asks for. This entry point uses a file-scope
- * device array of SPARK_NOALLOC_MAX_HEADS * 2 doubles (64 KiB, held by every GPU that
- * loads the library until the process exits) instead, and otherwise runs exactly the
- * spark_score_select path with the same arguments and outputs.
+ * loop that must never reach the driver's allocator - and so cannot provide the scratch
+ * that spark_score_select asks for. This entry point uses a file-scope device array of
+ * SPARK_NOALLOC_MAX_HEADS * 2 doubles (64 KiB, held by every GPU that loads the library
+ * until the process exits) for the tau moments instead, and keeps each CTA's score rows
+ * in shared memory rather than writing the score matrix out (a slower kernel with the
+ * same per-score arithmetic), with the same arguments and outputs.
  * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  * - B*H above SPARK_NOALLOC_MAX_HEADS returns SPARK_ESCRATCH before any launch.
  * - The first call on a device looks the array's device address up (cudaGetSymbolAddress,
