@@ -104,7 +104,7 @@ def load_peaks():
 # dram__bytes_read.sum + dram__bytes_write.sum of a 2-head capture of the same shape
 # (profiles/attn_tc_1152x640x243_h2_full.md), scaled by 12 to 24 heads. None once the
 # kernel has changed since it was measured.
-ATTN_TRAFFIC_BYTES = None
+ATTN_TRAFFIC_BYTES = 57.2e9
 
 
 class ClockSampler:
