@@ -337,54 +337,113 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
   int* piv = reinterpret_cast<int*>(misc + 8);
   const int tid = threadIdx.x;
 
-  // ---- tridiagonalisation
-  for (int k = 0; k < D - 2; ++k) {
-    const int m = D - k - 1;
-    for (int i = tid; i < m; i += kThreads) u[i] = C[(k + 1 + i) * D + k];
-    __syncthreads();
-    double ss = 0.0;
-    for (int i = tid; i < m; i += kThreads) ss += u[i] * u[i];
-    const double norm2 = block_sum_d(ss, red);
-    const double x0 = u[0];
-    const double tail = norm2 - x0 * x0;
-    __syncthreads();
-    if (!(tail > 1e-300 * (norm2 + 1e-300))) {  // column already reduced
-      if (tid == 0) {
-        bt[k] = 0.0;
-        e[k] = x0;
+  // ---- tridiagonalisation, with the matrix in registers: thread (ty, tx) of a 16 x 16
+  //      grid holds C[ty + 16 ra][tx + 16 rb] (ra, rb < D / 16). Per step k the column
+  //      below the diagonal becomes the Householder vector u (kept in column k for the
+  //      back-transformation), p = beta C u is reduced across the 16 threads of a row
+  //      group with shuffles, and the trailing block takes the rank-2 update
+  //      C -= u w^T + w u^T with w = p - (beta/2)(u.p) u.
+  {
+    constexpr int R = D / 16;
+    const int ty = tid >> 4, tx = tid & 15, lane = tid & 31, warp = tid >> 5;
+    double c[R][R];
+#pragma unroll
+    for (int ra = 0; ra < R; ++ra)
+#pragma unroll
+      for (int rb = 0; rb < R; ++rb) c[ra][rb] = C[(ty + 16 * ra) * D + tx + 16 * rb];
+    // k = 16 kb + kl: kb is unrolled so every register index is a compile-time constant
+#pragma unroll
+    for (int kb = 0; kb < R; ++kb) {
+      for (int kl = 0; kl < 16; ++kl) {
+        const int k = 16 * kb + kl;
+        if (k >= D - 2) break;
+        // column k below the diagonal into u (zero at and above the diagonal)
+        if (tx == kl) {
+#pragma unroll
+          for (int ra = 0; ra < R; ++ra) {
+            const int i = ty + 16 * ra;
+            if (i > k) u[i] = c[ra][kb];
+          }
+        }
+        if (tid <= k) u[tid] = 0.0;
+        __syncthreads();
+        if (warp == 0) {
+          double ss = 0.0;
+          for (int i = k + 1 + lane; i < D; i += 32) ss += u[i] * u[i];
+          ss = warp_sum_d(ss);
+          if (lane == 0) {
+            const double x0 = u[k + 1];
+            const double tail = ss - x0 * x0;
+            if (!(tail > 1e-300 * (ss + 1e-300))) {  // column already reduced
+              bt[k] = 0.0;
+              e[k] = x0;
+              misc[0] = 0.0;
+            } else {
+              const double alpha = -copysign(sqrt(ss), x0);
+              const double u0 = x0 - alpha;
+              const double beta = 2.0 / (tail + u0 * u0);
+              u[k + 1] = u0;
+              bt[k] = beta;
+              e[k] = alpha;
+              misc[0] = beta;
+            }
+          }
+        }
+        __syncthreads();
+        const double beta = misc[0];
+        if (beta == 0.0) continue;  // uniform across the CTA
+        double uj[R];
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) uj[rb] = u[tx + 16 * rb];
+#pragma unroll
+        for (int ra = 0; ra < R; ++ra) {
+          double sacc = 0.0;
+#pragma unroll
+          for (int rb = 0; rb < R; ++rb) sacc = fma(c[ra][rb], uj[rb], sacc);
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
+          if (tx == 0) w[ty + 16 * ra] = beta * sacc;  // p (rows at or above k are unused)
+        }
+        __syncthreads();
+        if (warp == 0) {
+          double dt = 0.0;
+          for (int i = k + 1 + lane; i < D; i += 32) dt += u[i] * w[i];
+          dt = warp_sum_d(dt);
+          if (lane == 0) misc[1] = 0.5 * beta * dt;
+        }
+        __syncthreads();
+        const double kc = misc[1];
+        double wj[R];
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) {
+          const int j = tx + 16 * rb;
+          wj[rb] = j > k ? w[j] - kc * uj[rb] : 0.0;
+        }
+#pragma unroll
+        for (int ra = 0; ra < R; ++ra) {
+          const int i = ty + 16 * ra;
+          const double ui = u[i];
+          const double wi = i > k ? w[i] - kc * ui : 0.0;
+#pragma unroll
+          for (int rb = 0; rb < R; ++rb) c[ra][rb] = fma(-ui, wj[rb], fma(-wi, uj[rb], c[ra][rb]));
+        }
+        // the Householder vector's first entry replaces C[k + 1][k] (row k + 1 lies in
+        // row group kb, or kb + 1 when kl = 15)
+        if (tx == kl && ty == ((k + 1) & 15)) {
+          const double u1 = u[k + 1];
+          if (kl < 15) {
+            c[kb][kb] = u1;
+          } else if (kb + 1 < R) {
+            c[(kb + 1) < R ? kb + 1 : kb][kb] = u1;
+          }
+        }
+        __syncthreads();  // u and w are rewritten by the next step
       }
-      __syncthreads();
-      continue;
     }
-    const double alpha = -copysign(sqrt(norm2), x0);
-    const double u0 = x0 - alpha;
-    const double beta = 2.0 / (tail + u0 * u0);
-    if (tid == 0) {
-      u[0] = u0;
-      bt[k] = beta;
-      e[k] = alpha;
-    }
-    __syncthreads();
-    for (int i = tid; i < m; i += kThreads) C[(k + 1 + i) * D + k] = u[i];
-    // w = beta * C' u over the trailing block (column reads; the block is symmetric)
-    {
-      const int i = tid >> 1, h = tid & 1;
-      double s = 0.0;
-      if (i < m)
-        for (int j = h; j < m; j += 2) s += C[(k + 1 + j) * D + (k + 1 + i)] * u[j];
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      if (i < m && h == 0) w[i] = beta * s;  // m <= 127 < kThreads / 2 rows
-    }
-    __syncthreads();
-    double dot = 0.0;
-    for (int i = tid; i < m; i += kThreads) dot += u[i] * w[i];
-    const double kc = 0.5 * beta * block_sum_d(dot, red);
-    for (int i = tid; i < m; i += kThreads) w[i] -= kc * u[i];
-    __syncthreads();
-    for (int q = tid; q < m * m; q += kThreads) {
-      const int i = q / m, j = q % m;
-      C[(k + 1 + i) * D + (k + 1 + j)] -= u[i] * w[j] + w[i] * u[j];
-    }
+#pragma unroll
+    for (int ra = 0; ra < R; ++ra)
+#pragma unroll
+      for (int rb = 0; rb < R; ++rb) C[(ty + 16 * ra) * D + tx + 16 * rb] = c[ra][rb];
     __syncthreads();
   }
   for (int i = tid; i < D; i += kThreads) a[i] = C[i * D + i];
