@@ -302,6 +302,18 @@ struct EigScratch {
   static constexpr int kBytes = kDoubles * 8 + D * 4;
 };
 
+// 1/x in fp64 by two Newton-Raphson steps r <- r (2 - x r) from the fp32 reciprocal
+// (relative error 2^-24 -> 2^-48 -> below fp64 rounding); magnitudes outside the fp32
+// range take the plain division.
+__device__ __forceinline__ double rcp_nr(double x) {
+  const double ax = fabs(x);
+  if (!(ax > 1e-36 && ax < 1e36)) return 1.0 / x;
+  double r = (double)__frcp_rn((float)x);
+  r = r * fma(-x, r, 2.0);
+  r = r * fma(-x, r, 2.0);
+  return r;
+}
+
 __device__ __forceinline__ int sturm_count(const double* a, const double* e2, int n, double x,
                                            double pivmin) {
   int c = 0;
@@ -309,7 +321,7 @@ __device__ __forceinline__ int sturm_count(const double* a, const double* e2, in
   if (q < 0.0) ++c;
   for (int i = 1; i < n; ++i) {
     const double den = fabs(q) < pivmin ? -pivmin : q;
-    q = (a[i] - x) - e2[i - 1] / den;
+    q = (a[i] - x) - e2[i - 1] * rcp_nr(den);
     if (q < 0.0) ++c;
   }
   return c;
@@ -357,44 +369,46 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
       for (int kl = 0; kl < 16; ++kl) {
         const int k = 16 * kb + kl;
         if (k >= D - 2) break;
-        // column k below the diagonal into u (zero at and above the diagonal)
+        // u and p alternate between two buffers so that one barrier before and one
+        // after the matrix-vector product suffice; every warp derives alpha, beta and
+        // u.p itself (identical arithmetic, identical results)
+        double* ub = (kl & 1) ? y : u;
+        double* pb = (kl & 1) ? dd : w;
+        // column k below the diagonal into ub (zero at and above the diagonal)
         if (tx == kl) {
 #pragma unroll
           for (int ra = 0; ra < R; ++ra) {
             const int i = ty + 16 * ra;
-            if (i > k) u[i] = c[ra][kb];
+            if (i > k) ub[i] = c[ra][kb];
           }
         }
-        if (tid <= k) u[tid] = 0.0;
+        if (tid <= k) ub[tid] = 0.0;
         __syncthreads();
-        if (warp == 0) {
-          double ss = 0.0;
-          for (int i = k + 1 + lane; i < D; i += 32) ss += u[i] * u[i];
-          ss = warp_sum_d(ss);
-          if (lane == 0) {
-            const double x0 = u[k + 1];
-            const double tail = ss - x0 * x0;
-            if (!(tail > 1e-300 * (ss + 1e-300))) {  // column already reduced
-              bt[k] = 0.0;
-              e[k] = x0;
-              misc[0] = 0.0;
-            } else {
-              const double alpha = -copysign(sqrt(ss), x0);
-              const double u0 = x0 - alpha;
-              const double beta = 2.0 / (tail + u0 * u0);
-              u[k + 1] = u0;
-              bt[k] = beta;
-              e[k] = alpha;
-              misc[0] = beta;
-            }
+        double ss = 0.0;
+        for (int i = k + 1 + lane; i < D; i += 32) ss += ub[i] * ub[i];
+        ss = warp_sum_d(ss);
+        const double x0 = ub[k + 1];
+        const double tail = ss - x0 * x0;
+        if (!(tail > 1e-300 * (ss + 1e-300))) {  // column already reduced (uniform)
+          if (tid == 0) {
+            bt[k] = 0.0;
+            e[k] = x0;
           }
+          continue;
         }
-        __syncthreads();
-        const double beta = misc[0];
-        if (beta == 0.0) continue;  // uniform across the CTA
+        const double alpha = -copysign(sqrt(ss), x0);
+        const double u0 = x0 - alpha;
+        const double beta = 2.0 / (tail + u0 * u0);
+        if (tid == 0) {
+          bt[k] = beta;
+          e[k] = alpha;
+        }
         double uj[R];
 #pragma unroll
-        for (int rb = 0; rb < R; ++rb) uj[rb] = u[tx + 16 * rb];
+        for (int rb = 0; rb < R; ++rb) {
+          const int j = tx + 16 * rb;
+          uj[rb] = j == k + 1 ? u0 : ub[j];
+        }
 #pragma unroll
         for (int ra = 0; ra < R; ++ra) {
           double sacc = 0.0;
@@ -402,52 +416,47 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
           for (int rb = 0; rb < R; ++rb) sacc = fma(c[ra][rb], uj[rb], sacc);
 #pragma unroll
           for (int off = 8; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
-          if (tx == 0) w[ty + 16 * ra] = beta * sacc;  // p (rows at or above k are unused)
+          if (tx == 0) pb[ty + 16 * ra] = beta * sacc;  // p (rows at or above k are unused)
         }
         __syncthreads();
-        if (warp == 0) {
-          double dt = 0.0;
-          for (int i = k + 1 + lane; i < D; i += 32) dt += u[i] * w[i];
-          dt = warp_sum_d(dt);
-          if (lane == 0) misc[1] = 0.5 * beta * dt;
-        }
-        __syncthreads();
-        const double kc = misc[1];
+        double dt = 0.0;
+        for (int i = k + 1 + lane; i < D; i += 32) dt += (i == k + 1 ? u0 : ub[i]) * pb[i];
+        const double kc = 0.5 * beta * warp_sum_d(dt);
         double wj[R];
 #pragma unroll
         for (int rb = 0; rb < R; ++rb) {
           const int j = tx + 16 * rb;
-          wj[rb] = j > k ? w[j] - kc * uj[rb] : 0.0;
+          wj[rb] = j > k ? pb[j] - kc * uj[rb] : 0.0;
         }
 #pragma unroll
         for (int ra = 0; ra < R; ++ra) {
           const int i = ty + 16 * ra;
-          const double ui = u[i];
-          const double wi = i > k ? w[i] - kc * ui : 0.0;
+          const double ui = i == k + 1 ? u0 : ub[i];
+          const double wi = i > k ? pb[i] - kc * ui : 0.0;
 #pragma unroll
           for (int rb = 0; rb < R; ++rb) c[ra][rb] = fma(-ui, wj[rb], fma(-wi, uj[rb], c[ra][rb]));
         }
         // the Householder vector's first entry replaces C[k + 1][k] (row k + 1 lies in
         // row group kb, or kb + 1 when kl = 15)
         if (tx == kl && ty == ((k + 1) & 15)) {
-          const double u1 = u[k + 1];
           if (kl < 15) {
-            c[kb][kb] = u1;
+            c[kb][kb] = u0;
           } else if (kb + 1 < R) {
-            c[(kb + 1) < R ? kb + 1 : kb][kb] = u1;
+            c[(kb + 1) < R ? kb + 1 : kb][kb] = u0;
           }
         }
-        __syncthreads();  // u and w are rewritten by the next step
       }
     }
+    __syncthreads();
+    // stored transposed: the Householder vector of step k is then row k of C, contiguous
 #pragma unroll
     for (int ra = 0; ra < R; ++ra)
 #pragma unroll
-      for (int rb = 0; rb < R; ++rb) C[(ty + 16 * ra) * D + tx + 16 * rb] = c[ra][rb];
+      for (int rb = 0; rb < R; ++rb) C[(tx + 16 * rb) * D + ty + 16 * ra] = c[ra][rb];
     __syncthreads();
   }
   for (int i = tid; i < D; i += kThreads) a[i] = C[i * D + i];
-  if (tid == 0) e[D - 2] = C[(D - 1) * D + (D - 2)];
+  if (tid == 0) e[D - 2] = C[(D - 2) * D + (D - 1)];
   __syncthreads();
   for (int i = tid; i < D - 1; i += kThreads) e2[i] = e[i] * e[i];
 
@@ -488,7 +497,7 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
   const double pivmin = misc[2];
   for (int round = 0; round < 12; ++round) {
     const double lo = misc[0], hi = misc[1];
-    if (hi - lo <= 4e-16 * fmax(fabs(lo), fabs(hi))) break;
+    if (hi - lo <= 1e-13 * fmax(fabs(lo), fabs(hi))) break;  // ample for the shift below
     const double x = lo + (hi - lo) * (double)(tid + 1) / (double)(kThreads + 1);
     const int c = sturm_count(a, e2, D, x, pivmin);
     double clo = (c <= D - 1) ? x : -1e300;  // at or below the top eigenvalue
@@ -528,12 +537,12 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
     for (int i = 0; i < D - 1; ++i) {
       if (fabs(dd[i]) >= fabs(dl[i])) {
         if (dd[i] == 0.0) dd[i] = tiny;
-        const double f = dl[i] / dd[i];
+        const double f = dl[i] * rcp_nr(dd[i]);
         dl[i] = f;
         dd[i + 1] -= f * du[i];
         piv[i] = 0;
       } else {
-        const double f = dd[i] / dl[i];
+        const double f = dd[i] * rcp_nr(dl[i]);
         dd[i] = dl[i];
         dl[i] = f;
         const double tmp = du[i];
@@ -547,6 +556,7 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
       }
     }
     if (dd[D - 1] == 0.0) dd[D - 1] = tiny;
+    for (int i = 0; i < D; ++i) dd[i] = rcp_nr(dd[i]);  // the solves multiply by 1 / pivot
     for (int i = 0; i < D; ++i) y[i] = 1.0 + 0.001 * i;
     for (int it = 0; it < 3; ++it) {
       for (int i = 0; i < D - 1; ++i) {
@@ -558,9 +568,9 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
           y[i + 1] = tmp;
         }
       }
-      y[D - 1] /= dd[D - 1];
-      y[D - 2] = (y[D - 2] - du[D - 2] * y[D - 1]) / dd[D - 2];
-      for (int i = D - 3; i >= 0; --i) y[i] = (y[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) / dd[i];
+      y[D - 1] *= dd[D - 1];
+      y[D - 2] = (y[D - 2] - du[D - 2] * y[D - 1]) * dd[D - 2];
+      for (int i = D - 3; i >= 0; --i) y[i] = (y[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) * dd[i];
       double nn = 0.0;
       for (int i = 0; i < D; ++i) nn += y[i] * y[i];
       const double inv = 1.0 / sqrt(nn);
@@ -576,9 +586,9 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
       if (b == 0.0) continue;
       const int m = D - k - 1;
       double s = 0.0;
-      for (int i = tid; i < m; i += 32) s += C[(k + 1 + i) * D + k] * y[k + 1 + i];
+      for (int i = tid; i < m; i += 32) s += C[k * D + k + 1 + i] * y[k + 1 + i];
       s = warp_sum_d(s) * b;
-      for (int i = tid; i < m; i += 32) y[k + 1 + i] -= s * C[(k + 1 + i) * D + k];
+      for (int i = tid; i < m; i += 32) y[k + 1 + i] -= s * C[k * D + k + 1 + i];
       __syncwarp();
     }
     double nn = 0.0;
