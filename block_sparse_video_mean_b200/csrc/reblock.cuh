@@ -135,6 +135,74 @@ __device__ void accumulate_moments(int n, LoadRow load_row, float* stage, double
   __syncthreads();
 }
 
+// As accumulate_moments, for fp32 rows already in global memory (`row_ptr(i)`, 16-byte
+// aligned, D floats): tiles are gathered with cp.async into two alternating stages, so the
+// next tile's gather overlaps this tile's products. `stage` holds 2 x kTile x (D + 4) floats.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+template <int D, class RowPtr>
+__device__ void accumulate_moments_rows(int n, RowPtr row_ptr, float* stage, double* S2, double* S1) {
+  constexpr int S = D / 16;
+  constexpr int LD = D + 4;  // padded staging row (16-byte multiple)
+  constexpr int C4 = D / 4;  // 16-byte chunks per row
+  const int tid = threadIdx.x;
+  const int ti = tid / 16, tj = tid % 16;
+  auto issue = [&](int t0, float* buf) {
+    const int nt = min(kTile, n - t0);
+    for (int e = tid; e < kTile * C4; e += kThreads) {
+      const int r = e / C4, c4 = e % C4;
+      float* dst = buf + r * LD + 4 * c4;
+      if (r < nt) cp_async16(dst, row_ptr(t0 + r) + 4 * c4);
+      else *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  const int ntiles = (n + kTile - 1) / kTile;
+  if (ntiles > 0) issue(0, stage);
+  cp_async_commit();
+  for (int tt = 0; tt < ntiles; ++tt) {
+    float* cur = stage + (tt & 1) * kTile * LD;
+    if (tt + 1 < ntiles) issue((tt + 1) * kTile, stage + ((tt + 1) & 1) * kTile * LD);
+    cp_async_commit();
+    cp_async_wait1();
+    __syncthreads();
+    float acc[S][S];
+#pragma unroll
+    for (int a = 0; a < S; ++a)
+#pragma unroll
+      for (int b = 0; b < S; ++b) acc[a][b] = 0.f;
+    for (int r = 0; r < kTile; ++r) {
+      const float* row = cur + r * LD;
+      float xa[S], xb[S];
+#pragma unroll
+      for (int a = 0; a < S; ++a) {
+        xa[a] = row[ti * S + a];
+        xb[a] = row[tj * S + a];
+      }
+#pragma unroll
+      for (int a = 0; a < S; ++a)
+#pragma unroll
+        for (int b = 0; b < S; ++b) acc[a][b] = fmaf(xa[a], xb[b], acc[a][b]);
+    }
+#pragma unroll
+    for (int a = 0; a < S; ++a)
+#pragma unroll
+      for (int b = 0; b < S; ++b) S2[(ti * S + a) * D + tj * S + b] += (double)acc[a][b];
+    if (S1 != nullptr && tid < D) {
+      float cs = 0.f;
+      for (int r = 0; r < kTile; ++r) cs += cur[r * LD + tid];
+      S1[tid] += (double)cs;
+    }
+    __syncthreads();  // this stage is refilled two tiles later
+  }
+}
+
 // Key second moment of one head: grid (chunks, B*H); fp64 atomics into macc[bh][D][D].
 template <int D>
 __global__ void __launch_bounds__(kThreads) kmoment_kernel(const uint16_t* __restrict__ K, int N, int nv,
@@ -218,58 +286,82 @@ __global__ void __launch_bounds__(kThreads) cholesky_kernel(const double* __rest
 }
 
 // x_i = L^T q_i / |L^T q_i| for the video rows of every head; also tok[i] = i and the
-// level-0 tree labels. grid (ceil(nv / 64), B*H).
+// level-0 tree labels. grid (ceil(nv / kWhTok), B*H). L stays in shared memory for the
+// CTA's kWhTok tokens, taken 64 at a time: thread (ty, tx) computes tokens 4 ty .. 4 ty + 3
+// x columns 4 tx .. 4 tx + 3 and 64 + 4 tx .. 64 + 4 tx + 3, summing k in increasing order.
+constexpr int kWhTok = 256;
 template <int D>
 __global__ void __launch_bounds__(kThreads)
     whiten_kernel(const uint16_t* __restrict__ Q, int N, int nv, const float* __restrict__ lmat,
                   float* __restrict__ X, int32_t* __restrict__ tok, int32_t* __restrict__ tree0,
                   size_t tree_head_stride) {
+  static_assert(D == 128 || D == 64, "head dim");
   extern __shared__ __align__(16) unsigned char smem[];
   float* Ls = reinterpret_cast<float*>(smem);  // D x D
-  float* qs = Ls + D * D;                      // 64 x (D + 4)
-  constexpr int LD = D + 4;
-  constexpr int CG = D / 4;                    // columns per thread
+  float* qs = Ls + D * D;                      // [D][64]: the tile's queries, transposed
+  constexpr int CW = D / 32;                   // columns per thread in each half
   const size_t bh = blockIdx.y;
-  const int t0 = blockIdx.x * 64;
   const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
   const float* L = lmat + bh * D * D;
   for (int e = tid; e < D * D / 4; e += kThreads)
     reinterpret_cast<float4*>(Ls)[e] = reinterpret_cast<const float4*>(L)[e];
-  for (int e = tid; e < 64 * D / 2; e += kThreads) {
-    const int r = e / (D / 2), c2 = e % (D / 2);
-    const int t = t0 + r;
-    uint32_t u = 0;
-    if (t < nv) u = *reinterpret_cast<const uint32_t*>(Q + (bh * N + t) * D + 2 * c2);
-    qs[r * LD + 2 * c2] = __uint_as_float(u << 16);
-    qs[r * LD + 2 * c2 + 1] = __uint_as_float(u & 0xffff0000u);
-  }
-  __syncthreads();
-  const int r = tid / 4, cg = tid % 4;  // token r of the tile, columns cg*CG ..
-  const int t = t0 + r;
-  float acc[CG];
+  for (int t0 = blockIdx.x * kWhTok; t0 < min(nv, (int)(blockIdx.x + 1) * kWhTok); t0 += 64) {
+    __syncthreads();  // qs reuse (and Ls on the first pass)
+    for (int e = tid; e < 64 * D / 2; e += kThreads) {
+      const int r = e / (D / 2), c2 = e % (D / 2);
+      const int t = t0 + r;
+      uint32_t u = 0;
+      if (t < nv) u = *reinterpret_cast<const uint32_t*>(Q + (bh * N + t) * D + 2 * c2);
+      qs[(2 * c2) * 64 + r] = __uint_as_float(u << 16);
+      qs[(2 * c2 + 1) * 64 + r] = __uint_as_float(u & 0xffff0000u);
+    }
+    __syncthreads();
+    float acc[4][2 * CW];
 #pragma unroll
-  for (int c = 0; c < CG; ++c) acc[c] = 0.f;
-  for (int k = 0; k < D; ++k) {
-    const float qk = qs[r * LD + k];
-    const float* lr = Ls + k * D + cg * CG;
+    for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int c = 0; c < CG; ++c) acc[c] = fmaf(qk, lr[c], acc[c]);
-  }
-  float ss = 0.f;
+      for (int c = 0; c < 2 * CW; ++c) acc[r][c] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+      const float4 q4 = *reinterpret_cast<const float4*>(qs + k * 64 + 4 * ty);
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      float lv[2 * CW];
 #pragma unroll
-  for (int c = 0; c < CG; ++c) ss = fmaf(acc[c], acc[c], ss);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-  const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
-  if (t < nv) {
-    float* xr = X + (bh * nv + t) * D + cg * CG;
+      for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-    for (int c = 0; c < CG; c += 4)
-      *reinterpret_cast<float4*>(xr + c) =
-          make_float4(acc[c] * inv, acc[c + 1] * inv, acc[c + 2] * inv, acc[c + 3] * inv);
-    if (cg == 0) {
-      tok[bh * nv + t] = t;
-      if (tree0 != nullptr) tree0[bh * tree_head_stride + t] = 0;
+        for (int c = 0; c < CW; c += 2) {
+          const float2 l2 = *reinterpret_cast<const float2*>(Ls + k * D + hh * (D / 2) + CW * tx + c);
+          lv[hh * CW + c] = l2.x;
+          lv[hh * CW + c + 1] = l2.y;
+        }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 2 * CW; ++c) acc[r][c] = fmaf(qv[r], lv[c], acc[r][c]);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2 * CW; ++c) ss = fmaf(acc[r][c], acc[r][c], ss);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+      const int t = t0 + 4 * ty + r;
+      if (t < nv) {
+        float* xr = X + (bh * nv + t) * D;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int c = 0; c < CW; c += 2)
+            *reinterpret_cast<float2*>(xr + hh * (D / 2) + CW * tx + c) =
+                make_float2(acc[r][hh * CW + c] * inv, acc[r][hh * CW + c + 1] * inv);
+        if (tx == 0) {
+          tok[bh * nv + t] = t;
+          if (tree0 != nullptr) tree0[bh * tree_head_stride + t] = 0;
+        }
+      }
     }
   }
 }
@@ -281,11 +373,8 @@ __device__ void node_covariance(const float* __restrict__ Xh, const int32_t* __r
                                 int n, float* stage, double* C, double* mu) {
   for (int i = threadIdx.x; i < D * D; i += kThreads) C[i] = 0.0;
   for (int i = threadIdx.x; i < D; i += kThreads) mu[i] = 0.0;
-  auto load = [&](int i, float* dst, int c4) {
-    const int t = tseg[i];
-    reinterpret_cast<float4*>(dst)[c4] = reinterpret_cast<const float4*>(Xh + (size_t)t * D)[c4];
-  };
-  accumulate_moments<D>(n, load, stage, C, mu);
+  auto rowp = [&](int i) { return Xh + (size_t)tseg[i] * D; };
+  accumulate_moments_rows<D>(n, rowp, stage, C, mu);
   const double inv = 1.0 / n;
   for (int i = threadIdx.x; i < D; i += kThreads) mu[i] *= inv;
   __syncthreads();
@@ -745,7 +834,7 @@ template <int D>
 struct SplitSmem {
   static constexpr int kC = D * D * 8;
   static constexpr int kVec = 2 * D * 8;
-  static constexpr int kStage = kTile * (D + 4) * 4;
+  static constexpr int kStage = 2 * kTile * (D + 4) * 4;
   static constexpr int kBytes = kC + kVec + EigScratch<D>::kBytes + kStage + (int)sizeof(SplitScratch) + 64;
 };
 
@@ -788,11 +877,8 @@ __global__ void __launch_bounds__(kThreads) node_moments_kernel(LevelArgs a, int
   for (int i = threadIdx.x; i < D * D + D; i += kThreads) S2[i] = 0.0;
   const float* Xh = a.X + bh * (size_t)a.nv * D;
   const int32_t* tseg = a.tin + bh * (size_t)a.nv + st * kBlock + t0;
-  auto load = [&](int i, float* dst, int c4) {
-    const int t = tseg[i];
-    reinterpret_cast<float4*>(dst)[c4] = reinterpret_cast<const float4*>(Xh + (size_t)t * D)[c4];
-  };
-  accumulate_moments<D>(n, load, stage, S2, S1);
+  auto rowp = [&](int i) { return Xh + (size_t)tseg[i] * D; };
+  accumulate_moments_rows<D>(n, rowp, stage, S2, S1);
   double* dst = nacc + ((size_t)c * gridDim.y + bh) * (D * D + D);
   for (int i = threadIdx.x; i < D * D + D; i += kThreads) atomicAdd(dst + i, S2[i]);
 }
@@ -1028,9 +1114,10 @@ int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, con
     kmoment_kernel<D><<<dim3((nv + kChunkTok - 1) / kChunkTok, bh), kThreads, smem_km, cs>>>(K, N, nv, macc);
     cudaFuncSetAttribute(cholesky_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, D * D * 8);
     cholesky_kernel<D><<<bh, kThreads, D * D * 8, cs>>>(macc, nv, lmat);
-    const int smem_wh = D * D * 4 + 64 * (D + 4) * 4;
+    const int smem_wh = D * D * 4 + 64 * D * 4;
     cudaFuncSetAttribute(whiten_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_wh);
-    whiten_kernel<D><<<dim3((nv + 63) / 64, bh), kThreads, smem_wh, cs>>>(Q, N, nv, lmat, X, tok0, tree, tree_stride);
+    whiten_kernel<D><<<dim3((nv + kWhTok - 1) / kWhTok, bh), kThreads, smem_wh, cs>>>(Q, N, nv, lmat, X, tok0, tree,
+                                                                                    tree_stride);
     SPARK_LAUNCH_CHECK();
     note_launches(3);
 
@@ -1044,7 +1131,7 @@ int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, con
     const int smem_split = SplitSmem<D>::kBytes;
     cudaFuncSetAttribute(node_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
     cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
-    const int smem_nm = (D * D + D) * 8 + kTile * (D + 4) * 4;
+    const int smem_nm = (D * D + D) * 8 + 2 * kTile * (D + 4) * 4;
     cudaFuncSetAttribute(node_moments_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_nm);
     for (int l = 0; l < P.first_small; ++l) {
       a.level = l;
