@@ -181,9 +181,11 @@ __device__ void accumulate_moments_rows(int n, RowPtr row_ptr, float* stage, dou
       const float* row = cur + r * LD;
       float xa[S], xb[S];
 #pragma unroll
-      for (int a = 0; a < S; ++a) {
-        xa[a] = row[ti * S + a];
-        xb[a] = row[tj * S + a];
+      for (int a = 0; a < S; a += 4) {
+        const float4 va = *reinterpret_cast<const float4*>(row + ti * S + a);
+        const float4 vb = *reinterpret_cast<const float4*>(row + tj * S + a);
+        xa[a] = va.x; xa[a + 1] = va.y; xa[a + 2] = va.z; xa[a + 3] = va.w;
+        xb[a] = vb.x; xb[a + 1] = vb.y; xb[a + 2] = vb.z; xb[a + 3] = vb.w;
       }
 #pragma unroll
       for (int a = 0; a < S; ++a)
@@ -746,19 +748,31 @@ __device__ void split_node(const double* v, const float* __restrict__ Xh, const 
                            int32_t* tout, float* proj, int n, int m, int label,
                            int32_t* tree_next, SplitScratch* sc) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int PL = D / 32;  // components per lane
+  // projections: 8 lanes per token, 4 tokens per warp at a time (PL = D / 8 components
+  // per lane, as float4 loads), so each warp keeps several row gathers in flight
+  constexpr int PL = D / 8;
+  const int sub = lane >> 3, sl = lane & 7;
   double vl[PL];
 #pragma unroll
-  for (int j = 0; j < PL; ++j) vl[j] = v[lane * PL + j];
+  for (int j = 0; j < PL; ++j) vl[j] = v[sl * PL + j];
   double psum = 0.0;
-  for (int i = warp; i < n; i += kThreads / 32) {
-    const int t = tin[i];
-    const float* xr = Xh + (size_t)t * D + lane * PL;
+  for (int i0 = 4 * warp; i0 < n; i0 += 4 * (kThreads / 32)) {
+    const int i = i0 + sub;
     double d = 0.0;
+    if (i < n) {
+      const float4* xr = reinterpret_cast<const float4*>(Xh + (size_t)tin[i] * D + sl * PL);
 #pragma unroll
-    for (int j = 0; j < PL; ++j) d = fma((double)xr[j], vl[j], d);
-    d = warp_sum_d(d);
-    if (lane == 0) {
+      for (int j = 0; j < PL / 4; ++j) {
+        const float4 x4 = xr[j];
+        d = fma((double)x4.x, vl[4 * j], d);
+        d = fma((double)x4.y, vl[4 * j + 1], d);
+        d = fma((double)x4.z, vl[4 * j + 2], d);
+        d = fma((double)x4.w, vl[4 * j + 3], d);
+      }
+    }
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (sl == 0 && i < n) {
       proj[i] = (float)d;
       psum += d;
     }
