@@ -494,17 +494,19 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
           bt[k] = beta;
           e[k] = alpha;
         }
+        // row and column groups below kb hold only indices <= k: the trailing block starts
+        // at group kb (a compile-time constant of this unrolled iteration)
         double uj[R];
 #pragma unroll
-        for (int rb = 0; rb < R; ++rb) {
+        for (int rb = kb; rb < R; ++rb) {
           const int j = tx + 16 * rb;
           uj[rb] = j == k + 1 ? u0 : ub[j];
         }
 #pragma unroll
-        for (int ra = 0; ra < R; ++ra) {
+        for (int ra = kb; ra < R; ++ra) {
           double sacc = 0.0;
 #pragma unroll
-          for (int rb = 0; rb < R; ++rb) sacc = fma(c[ra][rb], uj[rb], sacc);
+          for (int rb = kb; rb < R; ++rb) sacc = fma(c[ra][rb], uj[rb], sacc);
 #pragma unroll
           for (int off = 8; off > 0; off >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, off);
           if (tx == 0) pb[ty + 16 * ra] = beta * sacc;  // p (rows at or above k are unused)
@@ -515,17 +517,17 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
         const double kc = 0.5 * beta * warp_sum_d(dt);
         double wj[R];
 #pragma unroll
-        for (int rb = 0; rb < R; ++rb) {
+        for (int rb = kb; rb < R; ++rb) {
           const int j = tx + 16 * rb;
           wj[rb] = j > k ? pb[j] - kc * uj[rb] : 0.0;
         }
 #pragma unroll
-        for (int ra = 0; ra < R; ++ra) {
+        for (int ra = kb; ra < R; ++ra) {
           const int i = ty + 16 * ra;
           const double ui = i == k + 1 ? u0 : ub[i];
           const double wi = i > k ? pb[i] - kc * ui : 0.0;
 #pragma unroll
-          for (int rb = 0; rb < R; ++rb) c[ra][rb] = fma(-ui, wj[rb], fma(-wi, uj[rb], c[ra][rb]));
+          for (int rb = kb; rb < R; ++rb) c[ra][rb] = fma(-ui, wj[rb], fma(-wi, uj[rb], c[ra][rb]));
         }
         // the Householder vector's first entry replaces C[k + 1][k] (row k + 1 lies in
         // row group kb, or kb + 1 when kl = 15)
@@ -588,7 +590,7 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
   const double pivmin = misc[2];
   for (int round = 0; round < 12; ++round) {
     const double lo = misc[0], hi = misc[1];
-    if (hi - lo <= 1e-13 * fmax(fabs(lo), fabs(hi))) break;  // ample for the shift below
+    if (hi - lo <= 1e-11 * fmax(fabs(lo), fabs(hi))) break;  // ample for the shift below
     const double x = lo + (hi - lo) * (double)(tid + 1) / (double)(kThreads + 1);
     const int c = sturm_count(a, e2, D, x, pivmin);
     double clo = (c <= D - 1) ? x : -1e300;  // at or below the top eigenvalue
@@ -649,7 +651,7 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
     if (dd[D - 1] == 0.0) dd[D - 1] = tiny;
     for (int i = 0; i < D; ++i) dd[i] = rcp_nr(dd[i]);  // the solves multiply by 1 / pivot
     for (int i = 0; i < D; ++i) y[i] = 1.0 + 0.001 * i;
-    for (int it = 0; it < 3; ++it) {
+    for (int it = 0; it < 2; ++it) {  // each solve shrinks other components by (lambda1-theta)/gap
       for (int i = 0; i < D - 1; ++i) {
         if (piv[i] == 0) {
           y[i + 1] -= dl[i] * y[i];
@@ -670,23 +672,36 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
   }
   __syncthreads();
 
-  // ---- back-transform v = H_0 ... H_{D-3} y (one warp)
+  // ---- back-transform v = H_0 ... H_{D-3} y (one warp; lane l keeps y[l + 32 j] in
+  //      registers, the Householder vector of step k is row k of C)
   if (tid < 32) {
+    constexpr int YJ = D / 32;
+    double yr[YJ];
+#pragma unroll
+    for (int j = 0; j < YJ; ++j) yr[j] = y[tid + 32 * j];
     for (int k = D - 3; k >= 0; --k) {
       const double b = bt[k];
       if (b == 0.0) continue;
-      const int m = D - k - 1;
+      const double* hk = C + k * D;
+      double hv[YJ];
       double s = 0.0;
-      for (int i = tid; i < m; i += 32) s += C[k * D + k + 1 + i] * y[k + 1 + i];
+#pragma unroll
+      for (int j = 0; j < YJ; ++j) {
+        const int e = tid + 32 * j;
+        hv[j] = e > k ? hk[e] : 0.0;
+        s = fma(hv[j], yr[j], s);
+      }
       s = warp_sum_d(s) * b;
-      for (int i = tid; i < m; i += 32) y[k + 1 + i] -= s * C[k * D + k + 1 + i];
-      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < YJ; ++j) yr[j] = fma(-s, hv[j], yr[j]);
     }
     double nn = 0.0;
-    for (int i = tid; i < D; i += 32) nn += y[i] * y[i];
+#pragma unroll
+    for (int j = 0; j < YJ; ++j) nn = fma(yr[j], yr[j], nn);
     nn = warp_sum_d(nn);
     const double inv = 1.0 / sqrt(nn);
-    for (int i = tid; i < D; i += 32) v[i] = y[i] * inv;
+#pragma unroll
+    for (int j = 0; j < YJ; ++j) v[tid + 32 * j] = yr[j] * inv;
   }
   __syncthreads();
 }
