@@ -418,3 +418,26 @@ def test_whitening_is_mahalanobis_cosine_via_reblock():
     low = set(np.argsort(p)[:64].tolist())
     left = set(rb.splits[(0, 0)].left.tolist())
     assert left == low or left == set(range(128)) - low
+
+
+# --------------------------------------------------------------------------- branch fidelity
+# [Spark-H3] "What Spark-Attn changes": the compressed branch stands in for the blocks the
+# exact branch drops, and Spark-Reweight replaces the plain mean-pooled entry because
+# mean pooling gives exp(E[x]) where the softmax needs E[exp(x)]. On seeded synthetic
+# heads the oracle must order the three forwards by their distance to dense attention:
+# no compressed branch > mean-pooled branch > reweighted branch.
+@pytest.mark.parametrize("nv,ns,d,ratio,amp,seed", [
+    (64 * 48, 32, 64, 0.1, 0.5, 0),
+    (64 * 48, 32, 64, 0.2, 0.5, 1),
+    (64 * 48, 32, 64, 0.1, 1.0, 3),
+])
+def test_compressed_branch_fidelity_ordering(nv, ns, d, ratio, amp, seed):
+    Q, K, V = make_qkv(1, 1, nv, ns, d, seed=seed, amp=amp)
+    q, k, v = (orc.to_f64(t[0, 0]) for t in (Q, K, V))
+    dense, _, _ = orc.forward_head(q, k, v, ns, "topk", 1.0, False)
+    err = {}
+    for name, comp, pm in (("none", False, "reweight"), ("mean", True, "mean"),
+                           ("reweight", True, "reweight")):
+        o, _, _ = orc.forward_head(q, k, v, ns, "topk", ratio, comp, pool_mode=pm)
+        err[name] = np.linalg.norm(o[:nv] - dense[:nv]) / np.linalg.norm(dense[:nv])
+    assert err["reweight"] < err["mean"] < err["none"], err
