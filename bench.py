@@ -47,6 +47,7 @@ class Workload:
     param: float = 0.1
     compressed: bool = True
     reblock: bool = False
+    reblock_kv: bool = False
     B: int = 1
     d: int = 128
 
@@ -68,6 +69,9 @@ WORKLOADS = {w.name: w for w in [
     Workload("1344x768x240-reblock", "1344x768 240-frame clip: B=1 H=24 d=128, 61x84x48=245952 video "
              "tokens + 512 sink rows, Spark-Reblock partition, top-k 10%, exact + compressed; "
              "the step includes the reblock", 24, 245952, 512, reblock=True),
+    Workload("1344x768x240-reblock-kv", "as 1344x768x240-reblock with the keys on a partition of their "
+             "own (whitened by the queries' second moment) instead of reusing the queries'",
+             24, 245952, 512, reblock=True, reblock_kv=True),
 ]}
 DEFAULT = "1152x640x243"
 
@@ -199,7 +203,7 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     h = args.heads or w.H
     N = w.nv + w.ns
     Q, K, V = make_qkv(w.B, h, w.nv, w.ns, w.d, seed=args.seed + rank, device=dev)
-    cfg = spark.ForwardConfig(w.mode, w.param, w.compressed, reblock=w.reblock)
+    cfg = spark.ForwardConfig(w.mode, w.param, w.compressed, reblock=w.reblock, reblock_kv=w.reblock_kv)
     plan = spark.SparkAttention(w.B, h, N, w.d, w.ns, cfg, dev)
     nb = plan.nb
     stream = torch.cuda.current_stream(dev)

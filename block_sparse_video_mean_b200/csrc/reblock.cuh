@@ -1050,21 +1050,24 @@ __global__ void __launch_bounds__(kThreads) perm_kernel(const int32_t* __restric
 }
 
 // Qp/Kp/Vp rows p < nv come from rows perm[p]; dense rows are copied. 16 bytes per thread.
+// Q rows follow perm, K and V rows follow perm_kv (the same array under q_reuse_k).
 template <int D>
 __global__ void __launch_bounds__(kThreads) gather_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
                                                           const uint16_t* __restrict__ V, const int32_t* __restrict__ perm,
-                                                          int N, int nv, uint16_t* __restrict__ Qp,
-                                                          uint16_t* __restrict__ Kp, uint16_t* __restrict__ Vp) {
+                                                          const int32_t* __restrict__ perm_kv, int N, int nv,
+                                                          uint16_t* __restrict__ Qp, uint16_t* __restrict__ Kp,
+                                                          uint16_t* __restrict__ Vp) {
   constexpr int CH = D / 8;
   const size_t bh = blockIdx.y;
   const long long e = (long long)blockIdx.x * kThreads + threadIdx.x;
   if (e >= (long long)N * CH) return;
   const int p = (int)(e / CH), c = (int)(e % CH);
-  const int src = p < nv ? perm[bh * (size_t)nv + p] : p;
-  const size_t so = (bh * N + src) * D + c * 8, dof = (bh * N + p) * D + c * 8;
-  *reinterpret_cast<uint4*>(Qp + dof) = ldg_nc_v4(Q + so);
-  *reinterpret_cast<uint4*>(Kp + dof) = ldg_nc_v4(K + so);
-  *reinterpret_cast<uint4*>(Vp + dof) = ldg_nc_v4(V + so);
+  const int sq = p < nv ? perm[bh * (size_t)nv + p] : p;
+  const int sk = p < nv ? perm_kv[bh * (size_t)nv + p] : p;
+  const size_t dof = (bh * N + p) * D + c * 8;
+  *reinterpret_cast<uint4*>(Qp + dof) = ldg_nc_v4(Q + (bh * N + sq) * D + c * 8);
+  *reinterpret_cast<uint4*>(Kp + dof) = ldg_nc_v4(K + (bh * N + sk) * D + c * 8);
+  *reinterpret_cast<uint4*>(Vp + dof) = ldg_nc_v4(V + (bh * N + sk) * D + c * 8);
 }
 
 // ------------------------------------------------------------------ host side
@@ -1116,11 +1119,14 @@ inline size_t reblock_workspace_bytes(int bh, int nb, int d) {
   return rb::make_plan(bh, nb, d).total;
 }
 
+// Partition of the video rows of A (whitened by the second moment of the video rows of
+// Bm) into 64-row leaves: perm (and tree, when not null).
 template <int D>
-int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
-                int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
-                cudaStream_t cs) {
+int partition_run(int bh, int N, int nb, const uint16_t* A, const uint16_t* Bm, int32_t* perm,
+                  int32_t* tree, void* ws, cudaStream_t cs) {
   using namespace rb;
+  const uint16_t* Q = A;  // the rows being partitioned
+  const uint16_t* K = Bm; // the rows whose second moment whitens them
   const int nv = nb * kBlock;
   if (nb > 0) {
     const Plan P = make_plan(bh, nb, D);
@@ -1187,19 +1193,36 @@ int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, con
     SPARK_LAUNCH_CHECK();
     note_launches(3);
   }
+  return SPARK_OK;
+}
+
+// q_reuse_k when perm_k is null (K and V follow the query partition); otherwise the keys
+// get their own partition (whitened by the queries' second moment) in perm_k.
+template <int D>
+int reblock_run(int bh, int N, int nb, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                int32_t* perm, int32_t* perm_k, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp,
+                int32_t* tree, void* ws, cudaStream_t cs) {
+  using namespace rb;
+  const int nv = nb * kBlock;
+  int st = partition_run<D>(bh, N, nb, Q, K, perm, tree, ws, cs);
+  if (st != SPARK_OK) return st;
+  if (perm_k != nullptr) {
+    st = partition_run<D>(bh, N, nb, K, Q, perm_k, nullptr, ws, cs);
+    if (st != SPARK_OK) return st;
+  }
   const long long chunks = (long long)N * (D / 8);
   gather_kernel<D><<<dim3((unsigned)((chunks + kThreads - 1) / kThreads), bh), kThreads, 0, cs>>>(
-      Q, K, V, perm, N, nv, Qp, Kp, Vp);
+      Q, K, V, perm, perm_k != nullptr ? perm_k : perm, N, nv, Qp, Kp, Vp);
   SPARK_LAUNCH_CHECK();
   note_launches(1);
   return SPARK_OK;
 }
 
 inline int reblock_launch(int bh, int N, int nb, int d, const uint16_t* Q, const uint16_t* K,
-                          const uint16_t* V, int32_t* perm, uint16_t* Qp, uint16_t* Kp,
-                          uint16_t* Vp, int32_t* tree, void* ws, cudaStream_t stream) {
-  return d == 128 ? reblock_run<128>(bh, N, nb, Q, K, V, perm, Qp, Kp, Vp, tree, ws, stream)
-                  : reblock_run<64>(bh, N, nb, Q, K, V, perm, Qp, Kp, Vp, tree, ws, stream);
+                          const uint16_t* V, int32_t* perm, int32_t* perm_k, uint16_t* Qp,
+                          uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws, cudaStream_t stream) {
+  return d == 128 ? reblock_run<128>(bh, N, nb, Q, K, V, perm, perm_k, Qp, Kp, Vp, tree, ws, stream)
+                  : reblock_run<64>(bh, N, nb, Q, K, V, perm, perm_k, Qp, Kp, Vp, tree, ws, stream);
 }
 
 }  // namespace spark

@@ -401,9 +401,13 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   return s->d == 128 ? launch_attn_tc<128>(tp, K, V, pack, cs) : launch_attn_tc<64>(tp, K, V, pack, cs);
 }
 
-int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
-                  int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
-                  size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int reblock_impl(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                 int32_t* perm, int32_t* perm_k, bool independent, uint16_t* Qp, uint16_t* Kp,
+                 uint16_t* Vp, int32_t* tree, void* ws, size_t ws_bytes, void* stream) {
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   if (empty(s)) return SPARK_OK;
@@ -412,11 +416,27 @@ int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
       !aligned16(Vp))
     return SPARK_EINVAL;
   const int nb = (int)num_blocks(s);
-  if (nb > 0 && !perm) return SPARK_EINVAL;
+  if (nb > 0 && (!perm || (independent && !perm_k))) return SPARK_EINVAL;
   if (ws_bytes < spark_workspace_bytes(s, SPARK_CALL_REBLOCK)) return SPARK_EINVAL;
   if (spark_workspace_bytes(s, SPARK_CALL_REBLOCK) > 0 && (!ws || !aligned16(ws))) return SPARK_EINVAL;
-  return reblock_launch(s->B * s->H, s->N, nb, s->d, Q, K, V, perm, Qp, Kp, Vp, tree, ws,
-                        as_stream(stream));
+  return reblock_launch(s->B * s->H, s->N, nb, s->d, Q, K, V, perm, independent ? perm_k : nullptr, Qp, Kp,
+                        Vp, tree, ws, as_stream(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                  int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
+                  size_t ws_bytes, void* stream) {
+  return reblock_impl(s, Q, K, V, perm, nullptr, false, Qp, Kp, Vp, tree, ws, ws_bytes, stream);
+}
+
+int spark_reblock_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                     int32_t* perm_q, int32_t* perm_k, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp,
+                     void* ws, size_t ws_bytes, void* stream) {
+  return reblock_impl(s, Q, K, V, perm_q, perm_k, true, Qp, Kp, Vp, nullptr, ws, ws_bytes, stream);
 }
 
 int spark_device_error(int32_t* host_word, void* stream) {

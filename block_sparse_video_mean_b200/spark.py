@@ -28,7 +28,7 @@ BLOCK = 64
 
 EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
            "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
-           "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches")
+           "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches", "spark_reblock_kv")
 NOALLOC_MAX_HEADS = 4096
 
 
@@ -74,6 +74,8 @@ def load() -> ctypes.CDLL:
     lib.spark_attn_fwd.restype = I
     lib.spark_reblock.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
     lib.spark_reblock.restype = I
+    lib.spark_reblock_kv.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
+    lib.spark_reblock_kv.restype = I
     lib.spark_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
     lib.spark_device_error.restype = I
     lib.spark_strerror.argtypes = [I]
@@ -244,6 +246,27 @@ def reblock(Q, K, V, n_sink, tree=False, out=None, ws=None):
     return out
 
 
+def reblock_kv(Q, K, V, n_sink, out=None, ws=None):
+    """spark_reblock_kv (keys get their own partition): returns dict(perm, perm_k, Qp, Kp, Vp)."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        _need(t, n)
+    shape = _shape_of(Q, n_sink, None)
+    B, H, N, d = Q.shape
+    nb = num_blocks(shape)
+    dev = Q.device
+    if out is None:
+        out = dict(perm=torch.empty((B, H, nb * BLOCK), dtype=torch.int32, device=dev),
+                   perm_k=torch.empty((B, H, nb * BLOCK), dtype=torch.int32, device=dev),
+                   Qp=torch.empty_like(Q), Kp=torch.empty_like(K), Vp=torch.empty_like(V))
+    if ws is None:
+        ws = torch.empty(max(workspace_bytes(shape, CALL_REBLOCK), 16), dtype=torch.uint8, device=dev)
+    _check(load().spark_reblock_kv(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(out["perm"]),
+                                   _ptr(out["perm_k"]), _ptr(out["Qp"]), _ptr(out["Kp"]), _ptr(out["Vp"]),
+                                   _ptr(ws), ws.numel(), _stream(dev)),
+           "spark_reblock_kv")
+    return out
+
+
 # --------------------------------------------------------------------------- whole forward
 
 @dataclass
@@ -253,6 +276,7 @@ class ForwardConfig:
     compressed: bool = True     # Spark-Reweight compressed branch on/off
     pool_mode: str = "reweight"  # "reweight" or "mean"
     reblock: bool = False       # Spark-Reblock partition first (q_reuse_k)
+    reblock_kv: bool = False    # with reblock: keys get their own partition
     scale: float | None = None
     kcap: int | None = None     # slots per selection row (default: k, or nb for tau)
 
@@ -292,6 +316,8 @@ class SparkAttention:
                            Kp=torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
                            Vp=torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
                            tree=None)
+            if cfg.reblock_kv:
+                self.rb["perm_k"] = torch.empty((B, H, nb * BLOCK), dtype=torch.int32, device=dev)
             self.rb_ws = torch.empty(max(workspace_bytes(self.shape, CALL_REBLOCK), 16),
                                      dtype=torch.uint8, device=dev)
             self.levels = levels
@@ -309,7 +335,10 @@ class SparkAttention:
         perm = None
         mark(0)
         if self.rb is not None:
-            reblock(Q, K, V, self.n_sink, out=self.rb, ws=self.rb_ws)
+            if self.cfg.reblock_kv:
+                reblock_kv(Q, K, V, self.n_sink, out=self.rb, ws=self.rb_ws)
+            else:
+                reblock(Q, K, V, self.n_sink, out=self.rb, ws=self.rb_ws)
             Q, K, V, perm = self.rb["Qp"], self.rb["Kp"], self.rb["Vp"], self.rb["perm"]
         mark(1)
         pool_kv(Q, K, V, self.n_sink, self.pool_mode, cfg.scale, out=self.pool)

@@ -160,6 +160,18 @@ int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
                   int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
                   size_t ws_bytes, void* stream);
 
+/* Spark-Reblock with a partition of its own for the keys (the alternative to
+ * reblock_layout=q_reuse_k named in "Workflows"; the Spark-Reblock bullet whitens each side
+ * by the opposite side's second moment). perm_q is exactly what spark_reblock writes into
+ * perm; perm_k int32 [B, H, nb*64] partitions the video keys the same way with the roles of
+ * Q and K swapped (x_j = L^T k_j / |L^T k_j| with L L^T = mean over video queries of
+ * q q^T). Qp receives Q in the perm_q order, Kp and Vp receive K and V in the perm_k order
+ * (dense rows unchanged). Pass perm_q to spark_attn_fwd to get O back in the original
+ * query order. Same workspace as spark_reblock; about twice its time. No tree output. */
+int spark_reblock_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                     int32_t* perm_q, int32_t* perm_k, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp,
+                     void* ws, size_t ws_bytes, void* stream);
+
 /* spark_score_select without a scratch argument, for callers that cannot allocate device
  * memory of their own (the paper has no counterpart; this is a library convenience).
  * Some hosts own every byte of device memory up front - an engine that hands out one

@@ -378,13 +378,17 @@ def apply_perm(x, perm, n_sink, block=BLOCK):
 
 def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale=None,
                  block=BLOCK, reblock=False, qblocks=None, sel_override=None,
-                 pool_mode="reweight", perm_override=None):
+                 pool_mode="reweight", perm_override=None, reblock_kv=False,
+                 perm_k_override=None):
     """The whole forward of one head, in the original token order.
 
     Returns (O [N, d], LSE [N], info) where info holds the selection lists, the pooled
     summaries and, when ``reblock``, the Reblock result. ``sel_override`` replaces the
     oracle's own selection (used when a near-tie lets the GPU legitimately pick another
     block). ``qblocks`` restricts the video query blocks computed (others are NaN).
+    ``reblock_kv``: the keys get a partition of their own (the same bisection on the
+    keys, whitened by the queries' second moment) instead of reusing the queries'
+    (the alternative to q_reuse_k in [Spark-H3] "Workflows"); K and V follow it.
     """
     d = q.shape[1]
     scale = default_scale(d, scale)
@@ -395,7 +399,16 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
         else:
             rb = reblock_head(q, k, n_sink, block)
         info["reblock"] = rb
-        qp, kp, vp = (apply_perm(t, rb.perm, n_sink, block) for t in (q, k, v))
+        qp = apply_perm(q, rb.perm, n_sink, block)
+        if reblock_kv:
+            if perm_k_override is not None:
+                rbk = ReblockResult(np.asarray(perm_k_override, dtype=np.int64), None, {})
+            else:
+                rbk = reblock_head(k, q, n_sink, block)  # keys partitioned, whitened by queries
+            info["reblock_k"] = rbk
+            kp, vp = (apply_perm(t, rbk.perm, n_sink, block) for t in (k, v))
+        else:
+            kp, vp = (apply_perm(t, rb.perm, n_sink, block) for t in (k, v))
     else:
         qp, kp, vp = q, k, v
     pooled = pool_head(qp, kp, vp, n_sink, scale, block, pool_mode)

@@ -115,3 +115,52 @@ def test_reblock_full_size_sampled(spark):
         rows = np.concatenate([perm[i * 64:(i + 1) * 64] for i in blocks])
         check_output(O[0, h].float().cpu().numpy()[rows], ref[rows], f"head {h}")
         check_lse(Lse[0, h].cpu().numpy()[rows], lref[rows], f"head {h}")
+
+
+# ---------------------------------------------------------------- keys on their own partition
+@pytest.mark.parametrize("d,nb,ns,H", [(64, 5, 3, 2), (128, 13, 40, 2), (128, 70, 64, 1)])
+def test_reblock_kv_small(spark, d, nb, ns, H):
+    """perm_q is the q_reuse_k partition, perm_k the same construction with Q and K swapped
+    (node replay against the oracle through the swapped call's tree); Qp follows perm_q,
+    Kp and Vp follow perm_k."""
+    nv = 64 * nb
+    Q, K, V = make_qkv(1, H, nv, ns, d, seed=100 + nb)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    out = spark.reblock_kv(Qd, Kd, Vd, ns)
+    ref_q = spark.reblock(Qd, Kd, Vd, ns)
+    ref_k = spark.reblock(Kd, Qd, Vd, ns, tree=True)  # keys partitioned, whitened by queries
+    torch.cuda.synchronize()
+    assert spark.device_error() == 0
+    L = orc.n_levels(nb)
+    for h in range(H):
+        q, k, v = (orc.to_f64(t[0, h]) for t in (Q, K, V))
+        pq = out["perm"][0, h].cpu().numpy()
+        pk = out["perm_k"][0, h].cpu().numpy()
+        assert np.array_equal(pq, ref_q["perm"][0, h].cpu().numpy())
+        assert np.array_equal(pk, ref_k["perm"][0, h].cpu().numpy())
+        check_partition(pk, nv)
+        x = orc.whiten(k[:nv], orc.key_second_moment(q[:nv]))
+        replay_reblock_tree(x, ref_k["tree"][0, h].cpu().numpy(), L)
+        for name, T, pp in (("Qp", Q, pq), ("Kp", K, pk), ("Vp", V, pk)):
+            got = out[name][0, h].cpu()
+            exp = torch.cat([T[0, h][torch.from_numpy(pp).long()], T[0, h][nv:]])
+            assert torch.equal(got, exp), name
+
+
+def test_reblock_kv_forward_in_original_order(spark):
+    nb, ns, d = 30, 20, 128
+    Q, K, V = make_qkv(1, 2, 64 * nb, ns, d, seed=12)
+    cfg = spark.ForwardConfig("topk", 0.2, True, reblock=True, reblock_kv=True)
+    plan = spark.SparkAttention(1, 2, Q.shape[2], d, ns, cfg, DEV)
+    O, Lse = plan.run(Q.to(DEV), K.to(DEV), V.to(DEV))
+    torch.cuda.synchronize()
+    assert spark.device_error() == 0
+    for h in range(2):
+        q, k, v = (orc.to_f64(t[0, h]) for t in (Q, K, V))
+        pq = plan.rb["perm"][0, h].cpu().numpy()
+        pk = plan.rb["perm_k"][0, h].cpu().numpy()
+        sel = gpu_rows(plan.idx[0, h].cpu().numpy(), plan.cnt[0, h].cpu().numpy())
+        ref, lref, _ = orc.forward_head(q, k, v, ns, "topk", 0.2, True, reblock=True, reblock_kv=True,
+                                        perm_override=pq, perm_k_override=pk, sel_override=sel)
+        check_output(O[0, h].float().cpu().numpy(), ref, f"head {h}")
+        check_lse(Lse[0, h].cpu().numpy(), lref, f"head {h}")

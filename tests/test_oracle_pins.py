@@ -441,3 +441,30 @@ def test_compressed_branch_fidelity_ordering(nv, ns, d, ratio, amp, seed):
         o, _, _ = orc.forward_head(q, k, v, ns, "topk", ratio, comp, pool_mode=pm)
         err[name] = np.linalg.norm(o[:nv] - dense[:nv]) / np.linalg.norm(dense[:nv])
     assert err["reweight"] < err["mean"] < err["none"], err
+
+
+# --------------------------------------------------------------------------- keys' own partition
+def test_reblock_kv_full_density_is_dense_attention():
+    """With the keys on a partition of their own (and the queries on theirs), density 1.0
+    without the compressed branch is still dense softmax attention in the original order:
+    K and V must follow one permutation and O must be scattered back by the queries'."""
+    q, k, v = head(64 * 10, 24, 32, seed=31)
+    scale = 1 / math.sqrt(32)
+    O, L, info = orc.forward_head(q, k, v, 24, "topk", 1.0, compressed=False, reblock=True,
+                                  reblock_kv=True)
+    assert not np.array_equal(info["reblock"].perm, info["reblock_k"].perm)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, scale), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(L, lse64(q, k, scale), atol=1e-12, rtol=0)
+
+
+def test_reblock_kv_partition_is_the_swapped_partition_and_invariant():
+    """The keys' partition is the queries' construction with the roles swapped: leaves of 64
+    keys, unchanged when Q is scaled and when Q and K are rotated together."""
+    q, k, v = head(64 * 12, 0, 32, seed=22)
+    _, _, info = orc.forward_head(q, k, v, 0, "topk", 0.5, reblock=True, reblock_kv=True)
+    pk = info["reblock_k"].perm
+    assert sorted(pk.tolist()) == list(range(64 * 12))
+    base = _partition_sets(pk)
+    assert _partition_sets(orc.reblock_head(k, 3.1 * q, 0).perm) == base
+    R = random_orthogonal(32, 6).numpy()
+    assert _partition_sets(orc.reblock_head(k @ R, q @ R, 0).perm) == base
