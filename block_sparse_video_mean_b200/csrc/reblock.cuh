@@ -448,7 +448,7 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
   //      C -= u w^T + w u^T with w = p - (beta/2)(u.p) u.
   {
     constexpr int R = D / 16;
-    const int ty = tid >> 4, tx = tid & 15, lane = tid & 31, warp = tid >> 5;
+    const int ty = tid >> 4, tx = tid & 15, lane = tid & 31;
     double c[R][R];
 #pragma unroll
     for (int ra = 0; ra < R; ++ra)
