@@ -52,6 +52,13 @@ Readings where the pages are silent (each the plainest one the rest supports):
   >= 0, orders its tokens by (x . v, token index) and sends the first floor(m/2)*64 to
   the left child; leaves are ordered by their smallest token index and hold their
   tokens in ascending order. Keys reuse the query partition (q_reuse_k).
+* the 128-query x 64-key route ([H3-Opt] section "Manual Sparse Sage recovery": the
+  sparse fallback backends consume a 128Q x 64KV route): a query tile is two consecutive video blocks
+  (the last tile holds one block when nb is odd); its pooled query is the mean of the
+  tile's queries, it is scored against the 64-token key blocks and keeps
+  k = topk_count(ratio, nb) of them (tau: mu and sigma over all tile x block scores);
+  every query of the tile attends to the tile's selection. Keys, the anchor and the
+  compressed branch do not change.
 """
 from __future__ import annotations
 
@@ -84,7 +91,7 @@ def n_blocks(n_rows: int, n_sink: int, block: int = BLOCK) -> int:
 
 @dataclass
 class Pooled:
-    qbar: np.ndarray    # [nb, d] mean query of each block
+    qbar: np.ndarray    # [nt, d] mean query of each query tile (a block unless q_tile = 128)
     kbar: np.ndarray    # [nb, d] mean key of each block
     vtil: np.ndarray    # [nb, d] value summary of each block
     beta: np.ndarray    # [nb]    log-mass bias of each block
@@ -92,7 +99,17 @@ class Pooled:
     lse: np.ndarray     # [nb]    logsumexp of the anchor scores inside each block
 
 
-def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight") -> Pooled:
+def n_tiles(nb: int, q_tile: int = BLOCK, block: int = BLOCK) -> int:
+    """Query tiles of the route: ceil(nb * block / q_tile) (the last may be shorter)."""
+    return -(-nb * block // q_tile)
+
+
+def tile_rows(t: int, nv: int, q_tile: int = BLOCK) -> np.ndarray:
+    """Video rows of query tile t."""
+    return np.arange(t * q_tile, min((t + 1) * q_tile, nv))
+
+
+def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight", q_tile=BLOCK) -> Pooled:
     """Mean pooling, anchor and Spark-Reweight summaries of one head.
 
     [Spark-H3] "What Spark-Attn changes", Spark-Reweight bullet and the figure caption:
@@ -100,6 +117,8 @@ def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight") -> Pool
     the value summary is the softmax-weighted mean under those scores, and the log-mass
     bias makes exp(a . kbar_b * scale + beta_b) equal the block's total mass
     sum_j exp(s_j). ``mode="mean"`` gives the plain mean-pool branch instead.
+    ``q_tile`` = 128 pools the queries over the tiles of the 128-query route (qbar has
+    one row per tile); keys and the compressed branch keep 64-token blocks.
     """
     d = q.shape[1]
     scale = default_scale(d, scale)
@@ -108,7 +127,11 @@ def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight") -> Pool
     qb = q[:nv].reshape(nb, block, d)
     kb = k[:nv].reshape(nb, block, d)
     vb = v[:nv].reshape(nb, block, d)
-    qbar = qb.mean(axis=1)
+    if q_tile == block:
+        qbar = qb.mean(axis=1)
+    else:
+        qbar = np.stack([q[tile_rows(t, nv, q_tile)].mean(axis=0)
+                         for t in range(n_tiles(nb, q_tile, block))]) if nb else np.zeros((0, d))
     kbar = kb.mean(axis=1)
     anchor = q[:nv].mean(axis=0) if nv else np.zeros(d)
     s = (kb @ anchor) * scale                                   # [nb, block]
@@ -170,10 +193,9 @@ def select_tau_row(s_row, thr) -> np.ndarray:
 
 def select_head(qbar, kbar, scale, mode, param, rows=None):
     """Selected block lists of one head: a list of ascending int arrays, one per row."""
-    nb = qbar.shape[0]
-    rows = np.arange(nb) if rows is None else np.asarray(rows)
+    rows = np.arange(qbar.shape[0]) if rows is None else np.asarray(rows)
     if mode == "topk":
-        k = topk_count(param, nb)
+        k = topk_count(param, kbar.shape[0])
         S = block_scores(qbar, kbar, scale, rows)
         return [select_topk_row(S[r], k) for r in range(len(rows))]
     if mode == "tau":
@@ -196,8 +218,9 @@ def _softmax_out(logits, vals):
     return (p @ vals) / l, (m + np.log(l))[:, 0]
 
 
-def attn_video_block(q, k, v, n_sink, i, sel, pooled: Pooled | None, scale=None, block=BLOCK):
-    """Output rows of video query block i (in the order of q).
+def attn_video_block(q, k, v, n_sink, i, sel, pooled: Pooled | None, scale=None, block=BLOCK,
+                     q_tile=BLOCK):
+    """Output rows of video query tile i (block i unless ``q_tile`` = 128), in the order of q.
 
     [Spark-H3] "What Spark-Attn changes": the exact branch attends to the keys of the
     selected blocks, the compressed branch covers every other video block with one
@@ -208,7 +231,7 @@ def attn_video_block(q, k, v, n_sink, i, sel, pooled: Pooled | None, scale=None,
     scale = default_scale(d, scale)
     nb = n_blocks(q.shape[0], n_sink, block)
     nv = nb * block
-    qi = q[i * block:(i + 1) * block]
+    qi = q[tile_rows(i, nv, q_tile)]
     sel = np.asarray(sel, dtype=np.int64)
     key_rows = np.concatenate([np.arange(b * block, (b + 1) * block) for b in sel]
                               + [np.arange(nv, q.shape[0])]).astype(np.int64)
@@ -228,21 +251,22 @@ def attn_dense_rows(q, k, v, rows, scale=None):
 
 
 def attention_head(q, k, v, n_sink, sel_lists, pooled=None, scale=None, block=BLOCK,
-                   qblocks=None, dense_rows=True):
+                   qblocks=None, dense_rows=True, q_tile=BLOCK):
     """O [N, d] and LSE [N] of one head; rows not computed are NaN.
 
-    ``sel_lists[i]`` is the selected block list of video query block i (all blocks when
-    ``qblocks`` is None, else the blocks listed in ``qblocks``, in that order).
+    ``sel_lists[i]`` is the selected block list of video query tile i (all tiles when
+    ``qblocks`` is None, else the tiles listed in ``qblocks``, in that order).
     """
     N, d = q.shape
     nb = n_blocks(N, n_sink, block)
     O = np.full((N, d), np.nan)
     L = np.full(N, np.nan)
-    blocks = range(nb) if qblocks is None else qblocks
+    blocks = range(n_tiles(nb, q_tile, block)) if qblocks is None else qblocks
     for t, i in enumerate(blocks):
-        o, l = attn_video_block(q, k, v, n_sink, i, sel_lists[t], pooled, scale, block)
-        O[i * block:(i + 1) * block] = o
-        L[i * block:(i + 1) * block] = l
+        o, l = attn_video_block(q, k, v, n_sink, i, sel_lists[t], pooled, scale, block, q_tile)
+        rows = tile_rows(i, nb * block, q_tile)
+        O[rows] = o
+        L[rows] = l
     if dense_rows and N > nb * block:
         rows = np.arange(nb * block, N)
         o, l = attn_dense_rows(q, k, v, rows, scale)
@@ -379,7 +403,7 @@ def apply_perm(x, perm, n_sink, block=BLOCK):
 def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale=None,
                  block=BLOCK, reblock=False, qblocks=None, sel_override=None,
                  pool_mode="reweight", perm_override=None, reblock_kv=False,
-                 perm_k_override=None):
+                 perm_k_override=None, q_tile=BLOCK):
     """The whole forward of one head, in the original token order.
 
     Returns (O [N, d], LSE [N], info) where info holds the selection lists, the pooled
@@ -389,7 +413,10 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
     ``reblock_kv``: the keys get a partition of their own (the same bisection on the
     keys, whitened by the queries' second moment) instead of reusing the queries'
     (the alternative to q_reuse_k in [Spark-H3] "Workflows"); K and V follow it.
+    ``q_tile`` = 128: the 128-query route (``qblocks`` then lists query tiles).
     """
+    if q_tile not in (BLOCK, 2 * BLOCK) or block != BLOCK:
+        raise ValueError("q_tile must be 64 or 128 with 64-token blocks")
     d = q.shape[1]
     scale = default_scale(d, scale)
     info = {}
@@ -411,17 +438,17 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
             kp, vp = (apply_perm(t, rb.perm, n_sink, block) for t in (k, v))
     else:
         qp, kp, vp = q, k, v
-    pooled = pool_head(qp, kp, vp, n_sink, scale, block, pool_mode)
+    pooled = pool_head(qp, kp, vp, n_sink, scale, block, pool_mode, q_tile)
     info["pooled"] = pooled
-    nb = pooled.qbar.shape[0]
-    rows = np.arange(nb) if qblocks is None else np.asarray(qblocks)
+    nb = pooled.kbar.shape[0]
+    rows = np.arange(pooled.qbar.shape[0]) if qblocks is None else np.asarray(qblocks)
     if sel_override is not None:
         sel = sel_override
     else:
         sel = select_head(pooled.qbar, pooled.kbar, scale, mode, param, rows)
     info["sel"] = sel
     O, L = attention_head(qp, kp, vp, n_sink, sel, pooled if compressed else None, scale,
-                          block, qblocks=rows)
+                          block, qblocks=rows, q_tile=q_tile)
     if reblock:
         nv = nb * block
         O2, L2 = O.copy(), L.copy()

@@ -367,9 +367,9 @@ def test_planted_missing_scale_is_caught(monkeypatch):
 def test_planted_unweighted_summary_is_caught(monkeypatch):
     real = orc.pool_head
 
-    def bad(q, k, v, n_sink, scale=None, block=64, mode="reweight"):
-        P = real(q, k, v, n_sink, scale, block, mode)
-        nb = P.qbar.shape[0]
+    def bad(q, k, v, n_sink, scale=None, block=64, mode="reweight", q_tile=64):
+        P = real(q, k, v, n_sink, scale, block, mode, q_tile)
+        nb = P.kbar.shape[0]
         P.vtil = v[: nb * block].reshape(nb, block, -1).mean(1)
         return P
     monkeypatch.setattr(orc, "pool_head", bad)
@@ -468,3 +468,77 @@ def test_reblock_kv_partition_is_the_swapped_partition_and_invariant():
     assert _partition_sets(orc.reblock_head(k, 3.1 * q, 0).perm) == base
     R = random_orthogonal(32, 6).numpy()
     assert _partition_sets(orc.reblock_head(k @ R, q @ R, 0).perm) == base
+
+
+# ----------------------------------------------------------------- 128-query x 64-key route
+
+@pytest.mark.parametrize("nv,ns,d", [(448, 16, 64), (512 + 21, 7, 32)])
+def test_q128_full_density_no_compression_is_dense_attention(nv, ns, d):
+    """On the 128-query route (odd nb: the last tile holds one block; a ragged tail and
+    sinks follow), keep ratio 1.0 without compression is dense attention for every row."""
+    q, k, v = head(nv, ns, d, seed=11)
+    scale = 1 / math.sqrt(d)
+    O, L, info = orc.forward_head(q, k, v, ns, "topk", 1.0, compressed=False, q_tile=128)
+    assert len(info["sel"]) == orc.n_tiles(nv // 64, 128)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, scale), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(L, lse64(q, k, scale), atol=1e-12, rtol=0)
+
+
+def test_q128_tile_scores_are_means_of_block_scores():
+    """Pooling is linear: a tile's score against key block j is the mean of its blocks'
+    scores (the last tile of an odd nb is one block)."""
+    nv, ns, d = 7 * 64, 8, 64
+    q, k, v = head(nv, ns, d, seed=12)
+    scale = 1 / math.sqrt(d)
+    P64 = orc.pool_head(q, k, v, ns, scale)
+    P128 = orc.pool_head(q, k, v, ns, scale, q_tile=128)
+    S64 = orc.block_scores(P64.qbar, P64.kbar, scale)
+    S128 = orc.block_scores(P128.qbar, P128.kbar, scale)
+    assert S128.shape == (4, 7)
+    want = np.stack([S64[0:2].mean(0), S64[2:4].mean(0), S64[4:6].mean(0), S64[6]])
+    np.testing.assert_allclose(S128, want, atol=1e-13, rtol=0)
+    np.testing.assert_array_equal(P128.kbar, P64.kbar)
+    np.testing.assert_array_equal(P128.anchor, P64.anchor)
+
+
+@pytest.mark.parametrize("mode,param,nb", [("topk", 0.2, 7), ("topk", 0.5, 6), ("tau", 0.5, 8)])
+def test_q128_route_equals_block_route_when_block_pairs_repeat(mode, param, nb):
+    """When the second block of every tile repeats the first one's queries, a tile pools to
+    the same query as each of its blocks, selects the same key blocks and gives every row
+    the output of the 64-query route (for tau, with nb even, the score moments agree too)."""
+    ns, d = 12, 64
+    q, k, v = head(nb * 64, ns, d, seed=13)
+    for b in range(1, nb, 2):
+        q[b * 64:(b + 1) * 64] = q[(b - 1) * 64:b * 64]
+    O64, L64, i64 = orc.forward_head(q, k, v, ns, mode, param, compressed=True)
+    O128, L128, i128 = orc.forward_head(q, k, v, ns, mode, param, compressed=True, q_tile=128)
+    for t, sel in enumerate(i128["sel"]):
+        np.testing.assert_array_equal(sel, i64["sel"][2 * t])
+    np.testing.assert_allclose(O128, O64, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(L128, L64, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("mode,param", [("topk", 0.25), ("tau", 0.5)])
+def test_q128_constant_key_blocks_make_compression_exact(mode, param):
+    """The constant-key-block special case on the 128-query route: the pooled entries
+    carry each unselected block exactly, so the forward is dense attention."""
+    nv, ns, d = 5 * 64, 20, 64
+    q, k, v = head(nv, ns, d, seed=14)
+    kb = k[:nv].reshape(-1, 64, d)
+    kb[:] = kb[:, :1, :]
+    k[:nv] = kb.reshape(nv, d)
+    O, L, info = orc.forward_head(q, k, v, ns, mode, param, compressed=True, q_tile=128)
+    scale = 1 / math.sqrt(d)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, scale), atol=1e-10, rtol=0)
+    np.testing.assert_allclose(L, lse64(q, k, scale), atol=1e-10, rtol=0)
+
+
+def test_planted_end_aligned_last_tile_is_caught(monkeypatch):
+    """A last tile aligned to the end of the video rows (overlapping the tile before it,
+    instead of holding one block) breaks the linearity pin."""
+    def end_aligned(t, nv, q_tile=64):
+        hi = min((t + 1) * q_tile, nv)
+        return np.arange(max(hi - q_tile, 0), hi)
+    monkeypatch.setattr(orc, "tile_rows", end_aligned)
+    with pytest.raises(AssertionError):
+        test_q128_tile_scores_are_means_of_block_scores()
