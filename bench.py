@@ -50,6 +50,7 @@ class Workload:
     reblock_kv: bool = False
     B: int = 1
     d: int = 128
+    q_tile: int = 64
 
 
 WORKLOADS = {w.name: w for w in [
@@ -72,22 +73,32 @@ WORKLOADS = {w.name: w for w in [
     Workload("1344x768x240-reblock-kv", "as 1344x768x240-reblock with the keys on a partition of their "
              "own (whitened by the queries' second moment) instead of reusing the queries'",
              24, 245952, 512, reblock=True, reblock_kv=True),
+    Workload("1152x640x243-q128", "as 1152x640x243 on the 128-query x 64-key route: a query tile is two "
+             "consecutive blocks pooled together and sharing one selection (M = 128 tensor-core tiles)",
+             24, 175680, 512, q_tile=128),
+    Workload("1152x640x243-q128-tau1.5", "as 1152x640x243-q128 with tau=1.5", 24, 175680, 512,
+             mode="tau", param=1.5, q_tile=128),
+    Workload("1152x640x243-q128-dense", "as 1152x640x243-q128 at 100% density, compressed branch off",
+             24, 175680, 512, param=1.0, compressed=False, q_tile=128),
+    Workload("1344x768x240-reblock-q128", "as 1344x768x240-reblock on the 128-query route (a tile pairs "
+             "two consecutive leaves)", 24, 245952, 512, reblock=True, q_tile=128),
 ]}
 DEFAULT = "1152x640x243"
 
 
-def flop_counts(w: Workload, nb: int, kept_blocks: int, h=None):
+def flop_counts(w: Workload, nb: int, kept_qrows: int, h=None):
     """Algorithmic FLOPs of one forward (4*d per query-key pair: QK^T and PV).
 
-    kept_blocks = total selected (query block, key block) pairs over all heads."""
+    kept_qrows = selected (video query row, key block) pairs over all heads: the sum over
+    query tiles of (kept blocks x rows of the tile)."""
     h = w.H if h is None else h
     nv = nb * 64
     n = nv + w.ns
     d, b = w.d, w.B
-    exact = kept_blocks * 4 * 64 * 64 * d
+    exact = kept_qrows * 64 * 4 * d
     sink_keys = b * h * nv * w.ns * 4 * d          # video queries x dense keys
     sink_queries = b * h * w.ns * n * 4 * d        # dense queries x all keys
-    compressed = (b * h * nb * nb - kept_blocks) * 64 * 4 * d if w.compressed else 0
+    compressed = (b * h * nv * nb - kept_qrows) * 4 * d if w.compressed else 0
     dense_equiv = 4 * b * h * n * n * d
     return dict(exact=exact, sink=sink_keys + sink_queries, compressed=compressed,
                 selected=exact + sink_keys + sink_queries,
@@ -173,17 +184,17 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
-def phase_bytes(w: Workload, h: int, nb: int, kept_blocks: int, kcap: int):
+def phase_bytes(w: Workload, h: int, nb: int, nt: int, kept_blocks: int, kcap: int):
     """Algorithmic HBM bytes of the bandwidth-bound calls (each input read once, each
-    output written once)."""
+    output written once); nt query tiles (nb, or ceil(nb / 2) on the 128-query route)."""
     bh = w.B * h
     nv = nb * 64
     n = nv + w.ns
     row = w.d * 2
     nbp = (nb + 63) // 64 * 64
-    pool = (3 * bh * nv * row + 3 * bh * nb * w.d * 4 + bh * nb * 4 + 2 * bh * nb * w.d * 2
+    pool = (3 * bh * nv * row + (nt + 2 * nb) * bh * w.d * 4 + bh * nb * 4 + 2 * bh * nb * w.d * 2
             + bh * nbp * 4 + bh * w.d * 4)
-    select = 2 * bh * nb * w.d * 4 + kept_blocks * 4 + bh * nb * 4
+    select = (nt + nb) * bh * w.d * 4 + kept_blocks * 4 + bh * nt * 4
     gather = 6 * bh * n * row + bh * nv * 4          # permute Q,K,V (read + write) + perm
     return dict(pool=pool, select=select, reblock_gather=gather)
 
@@ -203,9 +214,10 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     h = args.heads or w.H
     N = w.nv + w.ns
     Q, K, V = make_qkv(w.B, h, w.nv, w.ns, w.d, seed=args.seed + rank, device=dev)
-    cfg = spark.ForwardConfig(w.mode, w.param, w.compressed, reblock=w.reblock, reblock_kv=w.reblock_kv)
+    cfg = spark.ForwardConfig(w.mode, w.param, w.compressed, reblock=w.reblock, reblock_kv=w.reblock_kv,
+                              q_tile=w.q_tile)
     plan = spark.SparkAttention(w.B, h, N, w.d, w.ns, cfg, dev)
-    nb = plan.nb
+    nb, nt = plan.nb, plan.nt
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -215,8 +227,12 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     if err != 0:
         raise RuntimeError(f"device error {err} ({spark.strerror(err)})")
     kept = int(plan.cnt.to(torch.int64).sum().item()) if nb > 0 else 0
-    fl = flop_counts(w, nb, kept, h)
-    by = phase_bytes(w, h, nb, kept, plan.kcap)
+    rows = torch.full((nt,), w.q_tile, dtype=torch.int64, device=dev)
+    if nt:
+        rows[-1] = nb * 64 - (nt - 1) * w.q_tile   # a one-block last tile on the 128-query route
+    kept_qrows = int((plan.cnt.to(torch.int64) * rows).sum().item()) if nb > 0 else 0
+    fl = flop_counts(w, nb, kept_qrows, h)
+    by = phase_bytes(w, h, nb, nt, kept, plan.kcap)
 
     ev = []
     if world > 1:
@@ -298,7 +314,7 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
                  "frac_hbm": round(by["pool"] / (phase_ms["pool"] * 1e-3) / 1e9 / hbm, 3)},
         "select": {"ms": round(phase_ms["select"], 3), "bytes": by["select"],
                    "GB/s": gbs(by["select"], phase_ms["select"]),
-                   "score_flops": 2 * w.B * h * nb * nb * w.d},
+                   "score_flops": 2 * w.B * h * nt * nb * w.d},
         "attn": {"ms": round(attn_ms, 3), "selected_flops": fl["selected"],
                  "compressed_flops": fl["compressed"]},
     }
@@ -322,7 +338,8 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
         "config": {"workload": w.name, "desc": w.desc, "global_batch": world * w.B, "heads": h,
                    "seq_len": N, "head_dim": w.d, "select": f"{w.mode} {w.param}",
                    "compressed": w.compressed, "reblock": w.reblock, "video_blocks": nb,
-                   "kept_blocks_mean_per_query_block": round(kept / max(w.B * h * nb, 1), 2),
+                   "query_tile": w.q_tile,
+                   "kept_blocks_mean_per_query_tile": round(kept / max(w.B * h * nt, 1), 2),
                    "parallelism": f"independent problem per GPU x{world}",
                    "l2": f"inputs {3 * Q.numel() * 2 / 1e9:.2f} GB "
                          + ("> 126 MB L2; no flush needed" if 3 * Q.numel() * 2 > 126e6
@@ -331,7 +348,8 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
         "phases": phases,
         # the attention kernel runs inside back-to-back steps of a seconds-long timed region,
         # under the power cap: the sustained figure is its denominator
-        "roofline": {"bound": "tensor", "kernel": f"attn_tc_kernel<{w.d}>",
+        "roofline": {"bound": "tensor",
+                     "kernel": f"attn_tc128_kernel<{w.d}>" if w.q_tile == 128 else f"attn_tc_kernel<{w.d}>",
                      "achieved": round(achieved, 2), "peak": bf16_sust or bf16_peak, "unit": "TFLOP/s",
                      "frac": round(achieved / (bf16_sust or bf16_peak), 4),
                      "peak_source": f"{peak_src} bf16 sustained (burst {bf16_peak})",
@@ -366,15 +384,18 @@ def cpu_baseline(w: Workload, Qc, Kc, Vc, n_blocks, seed=0):
     q, k, v = (orc.to_f64(t[0, 0]) for t in (Qc, Kc, Vc))
     n = q.shape[0]
     scale = 1.0 / math.sqrt(w.d)
-    P = orc.pool_head(q, k, v, w.ns, scale)
-    nb = P.qbar.shape[0]
+    P = orc.pool_head(q, k, v, w.ns, scale, 64, "reweight", w.q_tile)
+    nb, nt = P.kbar.shape[0], P.qbar.shape[0]
     rng = np.random.default_rng(seed)
-    blocks = rng.choice(nb, min(n_blocks, nb), replace=False)
+    # the same number of query rows on either route
+    blocks = rng.choice(nt, min(max(n_blocks * 64 // w.q_tile, 1), nt), replace=False)
     sel = orc.select_head(P.qbar, P.kbar, scale, w.mode, w.param, blocks)
+    rows = 0
     for t, i in enumerate(blocks):
-        orc.attn_video_block(q, k, v, w.ns, i, sel[t], P if w.compressed else None, scale)
+        o, _ = orc.attn_video_block(q, k, v, w.ns, i, sel[t], P if w.compressed else None, scale, 64,
+                                    w.q_tile)
+        rows += o.shape[0]
     dt = time.perf_counter() - t_start
-    rows = len(blocks) * 64
     flops = 4.0 * rows * n * w.d
     threads = None
     try:
@@ -385,7 +406,8 @@ def cpu_baseline(w: Workload, Qc, Kc, Vc, n_blocks, seed=0):
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s dense-equivalent",
             "cores": threads or os.cpu_count(), "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"1 of {w.H} heads: pooling of all {nb} blocks, {w.mode} {w.param} selection "
-                      f"of {len(blocks)} random query blocks and their attention ({rows} query rows)"}
+                      f"of {len(blocks)} random {w.q_tile}-query tiles and their attention "
+                      f"({rows} query rows)"}
 
 
 def run_reference(args, w: Workload, rank, world):

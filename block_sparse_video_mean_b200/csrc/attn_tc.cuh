@@ -65,6 +65,7 @@ struct TcParams {
   uint16_t* O;
   float* lse;
   int N, nb, nbp, kcap, BH, n_dq, pooled, n_items;
+  int nt;  // video query tiles per head (the 128-query route; nb for 64-query tiles)
   float scale_log2;
 };
 

@@ -23,31 +23,37 @@ struct RowLayout {
   static constexpr int NR = kBlock / RPP;  // rows per lane
 };
 
-// q_pool[bh, i, :] = mean of the 64 queries of block i.
-template <int D>
+// q_pool[bh, i, :] = mean of the queries of query tile i: QT = 64 rows (a block) or 128
+// (two blocks; the last tile holds one block when nb is odd).
+template <int D, int QT>
 __global__ void __launch_bounds__(kPoolWarps * 32) pool_q_kernel(const uint16_t* __restrict__ Q,
                                                                  float* __restrict__ q_pool, int N,
-                                                                 int nb) {
+                                                                 int nt, int nv) {
   using L = RowLayout<D>;
+  constexpr int NR = QT / L::RPP;  // rows per lane
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bi = blockIdx.x * kPoolWarps + warp;
-  if (bi >= nb) return;
+  if (bi >= nt) return;
   const size_t bh = blockIdx.y;
   const int c = lane % L::CPR, r0 = lane / L::CPR;
-  const uint16_t* base = Q + (bh * N + (size_t)bi * kBlock) * D + c * 8;
+  const int nrows = min(QT, nv - bi * QT);  // a multiple of 64, so of RPP
+  const int nr = nrows / L::RPP;             // rows this lane reads (warp-uniform)
+  const uint16_t* base = Q + (bh * N + (size_t)bi * QT) * D + c * 8;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  constexpr int NBATCH = L::NR < 8 ? L::NR : 8;  // 8 loads in flight per lane
+  constexpr int NBATCH = NR < 8 ? NR : 8;  // 8 loads in flight per lane
 #pragma unroll
-  for (int i0 = 0; i0 < L::NR; i0 += NBATCH) {
-    uint4 u[NBATCH];
+  for (int i0 = 0; i0 < NR; i0 += NBATCH) {
+    if (i0 < nr) {
+      uint4 u[NBATCH];
 #pragma unroll
-    for (int i = 0; i < NBATCH; ++i) u[i] = ldg_nc_v4(base + (size_t)(r0 + L::RPP * (i0 + i)) * D);
+      for (int i = 0; i < NBATCH; ++i) u[i] = ldg_nc_v4(base + (size_t)(r0 + L::RPP * (i0 + i)) * D);
 #pragma unroll
-    for (int i = 0; i < NBATCH; ++i) {
-      float f[8];
-      bf16x8_to_f32(u[i], f);
+      for (int i = 0; i < NBATCH; ++i) {
+        float f[8];
+        bf16x8_to_f32(u[i], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+      }
     }
   }
 #pragma unroll
@@ -55,33 +61,34 @@ __global__ void __launch_bounds__(kPoolWarps * 32) pool_q_kernel(const uint16_t*
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
   if (r0 == 0) {
-    float4* dst = reinterpret_cast<float4*>(q_pool + (bh * nb + bi) * D + c * 8);
-    const float inv = 1.0f / kBlock;
+    float4* dst = reinterpret_cast<float4*>(q_pool + (bh * nt + bi) * D + c * 8);
+    const float inv = 1.0f / nrows;
     dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
     dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
   }
 }
 
-// anchor[bh, :] = mean over blocks of q_pool (equal-size blocks: the mean video query).
-// Fixed-order reduction (deterministic): thread group g sums blocks g, g+G, ... then the
+// anchor[bh, :] = the mean video query: the mean of the nt rows of q_pool, the last one
+// weighted by last_w (1, or 0.5 for a one-block last tile of the 128-query route).
+// Fixed-order reduction (deterministic): thread group g sums tiles g, g+G, ... then the
 // groups are added in order.
 template <int D>
 __global__ void __launch_bounds__(256) anchor_kernel(const float* __restrict__ q_pool,
-                                                     float* __restrict__ anchor, int nb) {
+                                                     float* __restrict__ anchor, int nt, float last_w) {
   constexpr int G = 256 / D;
   __shared__ float part[G][D];
   const int c = threadIdx.x % D, g = threadIdx.x / D;
   const size_t bh = blockIdx.x;
-  const float* src = q_pool + bh * (size_t)nb * D;
+  const float* src = q_pool + bh * (size_t)nt * D;
   float acc = 0.f;
-  for (int b = g; b < nb; b += G) acc += src[(size_t)b * D + c];
+  for (int b = g; b < nt; b += G) acc += src[(size_t)b * D + c] * (b == nt - 1 ? last_w : 1.0f);
   part[g][c] = acc;
   __syncthreads();
   if (g == 0) {
     float t = 0.f;
 #pragma unroll
     for (int i = 0; i < G; ++i) t += part[i][c];
-    anchor[bh * D + c] = nb > 0 ? t / nb : 0.f;
+    anchor[bh * D + c] = nt > 0 ? t / ((float)(nt - 1) + last_w) : 0.f;
   }
 }
 

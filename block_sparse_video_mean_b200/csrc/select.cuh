@@ -26,8 +26,8 @@ constexpr int kSelKT = kSelJT + 1;  // padded row stride of the transposed tile 
 // acc = tr(Mq Mk) = sum_{i,j} (qbar_i . kbar_j)^2.
 template <int D>
 __global__ void __launch_bounds__(256) moments_kernel(const float* __restrict__ q_pool,
-                                                      const float* __restrict__ k_pool, int nb,
-                                                      double* __restrict__ acc) {
+                                                      const float* __restrict__ k_pool, int nq,
+                                                      int nb, double* __restrict__ acc) {
   constexpr int T = 32;
   constexpr int TPD = D / T;
   const int tr = blockIdx.x / TPD, tc = blockIdx.x % TPD;
@@ -37,18 +37,19 @@ __global__ void __launch_bounds__(256) moments_kernel(const float* __restrict__ 
   const int tid = threadIdx.x;
   const int r = tid / 8, c0 = (tid % 8) * 4;  // each thread: row r, columns c0..c0+3
   double mq[4] = {0, 0, 0, 0}, mk[4] = {0, 0, 0, 0};
-  const float* qp = q_pool + bh * (size_t)nb * D;
+  const float* qp = q_pool + bh * (size_t)nq * D;
   const float* kp = k_pool + bh * (size_t)nb * D;
-  for (int b0 = 0; b0 < nb; b0 += T) {
-    // stage 32 blocks x 32 columns of each operand (rows tr*T.., cols tc*T..)
+  const int nmax = nq > nb ? nq : nb;
+  for (int b0 = 0; b0 < nmax; b0 += T) {
+    // stage 32 rows x 32 columns of each operand (rows tr*T.., cols tc*T..)
     for (int e = tid; e < T * T; e += 256) {
       const int bb = e / T, cc = e % T;
-      const bool ok = b0 + bb < nb;
+      const bool okq = b0 + bb < nq, okk = b0 + bb < nb;
       const size_t o = (size_t)(b0 + bb) * D;
-      qa[bb][cc] = ok ? qp[o + tr * T + cc] : 0.f;
-      qb[bb][cc] = ok ? qp[o + tc * T + cc] : 0.f;
-      ka[bb][cc] = ok ? kp[o + tr * T + cc] : 0.f;
-      kb[bb][cc] = ok ? kp[o + tc * T + cc] : 0.f;
+      qa[bb][cc] = okq ? qp[o + tr * T + cc] : 0.f;
+      qb[bb][cc] = okq ? qp[o + tc * T + cc] : 0.f;
+      ka[bb][cc] = okk ? kp[o + tr * T + cc] : 0.f;
+      kb[bb][cc] = okk ? kp[o + tc * T + cc] : 0.f;
     }
     __syncthreads();
 #pragma unroll 4
@@ -76,24 +77,23 @@ __global__ void __launch_bounds__(256) moments_kernel(const float* __restrict__ 
   }
 }
 
-// thr[bh] = mu + tau * sigma with mu = scale * (sum qbar) . (sum kbar) / nb^2 and
-// sigma^2 = scale^2 * tr(Mq Mk) / nb^2 - mu^2 (population moments of all nb^2 scores).
+// thr[bh] = mu + tau * sigma with mu = scale * (sum qbar) . (sum kbar) / (nq nb) and
+// sigma^2 = scale^2 * tr(Mq Mk) / (nq nb) - mu^2 (population moments of all nq x nb
+// scores; nq query rows: blocks, or tiles of the 128-query route).
 template <int D>
 __global__ void __launch_bounds__(D) tau_threshold_kernel(const float* __restrict__ q_pool,
-                                                          const float* __restrict__ k_pool, int nb,
-                                                          const double* __restrict__ acc,
+                                                          const float* __restrict__ k_pool, int nq,
+                                                          int nb, const double* __restrict__ acc,
                                                           double scale, double tau,
                                                           double* __restrict__ thr) {
   __shared__ double red[D / 32];
   const size_t bh = blockIdx.x;
   const int c = threadIdx.x;
-  const float* qp = q_pool + bh * (size_t)nb * D;
+  const float* qp = q_pool + bh * (size_t)nq * D;
   const float* kp = k_pool + bh * (size_t)nb * D;
   double sq = 0.0, sk = 0.0;
-  for (int b = 0; b < nb; ++b) {
-    sq += qp[(size_t)b * D + c];
-    sk += kp[(size_t)b * D + c];
-  }
+  for (int b = 0; b < nq; ++b) sq += qp[(size_t)b * D + c];
+  for (int b = 0; b < nb; ++b) sk += kp[(size_t)b * D + c];
   double p = sq * sk;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(D) tau_threshold_kernel(const float* __restric
   if (c == 0) {
     double dot = 0.0;
     for (int w = 0; w < D / 32; ++w) dot += red[w];
-    const double n2 = (double)nb * (double)nb;
+    const double n2 = (double)nq * (double)nb;
     const double mu = scale * dot / n2;
     const double es2 = scale * scale * acc[bh] / n2;
     const double var = es2 - mu * mu;
@@ -117,7 +117,7 @@ struct SelectParams {
   int32_t* idx;
   int32_t* cnt;
   const double* thr;  // [B*H] (tau mode)
-  int nb, kcap, k, mode, rt;
+  int nq, nb, kcap, k, mode, rt;  // nq score rows (query blocks or tiles), nb key blocks
   float scale;
 };
 
@@ -226,8 +226,8 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t bh = blockIdx.y;
   const int row0 = blockIdx.x * RT;
-  const int nrows = min(RT, nb - row0);
-  const float* qp = p.q_pool + bh * (size_t)nb * D;
+  const int nrows = min(RT, p.nq - row0);
+  const float* qp = p.q_pool + bh * (size_t)p.nq * D;
   const float* kp = p.k_pool + bh * (size_t)nb * D;
 
   for (int e = tid; e < RT * D; e += kSelThreads) {
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(SelectParams 
   // ---- selection: warp w handles rows w, w + 8, ...
   uint32_t* h = hist + warp * 256;
   for (int r = warp; r < nrows; r += kSelThreads / 32)
-    select_row_warp(p, keys + (size_t)r * nbp, bh, bh * (size_t)nb + row0 + r, h, lane);
+    select_row_warp(p, keys + (size_t)r * nbp, bh, bh * (size_t)p.nq + row0 + r, h, lane);
 }
 
 // ---------------------------------------------------------------- scores, tiled
@@ -274,8 +274,8 @@ constexpr int kScI = 64, kScJ = 128, kScDC = 32;
 
 template <int D>
 __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict__ q_pool,
-                                                         const float* __restrict__ k_pool, int nb,
-                                                         int nbp, float scale,
+                                                         const float* __restrict__ k_pool, int nq,
+                                                         int nb, int nbp, float scale,
                                                          uint32_t* __restrict__ skeys) {
   __shared__ __align__(16) float qs[kScDC][kScI];
   __shared__ __align__(16) float ks[kScDC][kScJ];
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
   const int ty = tid >> 4, tx = tid & 15;
   const size_t bh = blockIdx.z;
   const int i0 = blockIdx.y * kScI, j0 = blockIdx.x * kScJ;
-  const float* qp = q_pool + bh * (size_t)nb * D;
+  const float* qp = q_pool + bh * (size_t)nq * D;
   const float* kp = k_pool + bh * (size_t)nb * D;
   float acc0[4][8], acc1[4][8];
 #pragma unroll
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
     for (int e = tid; e < kScI * kScDC / 4; e += 256) {
       const int rr = e / (kScDC / 4), cc = (e % (kScDC / 4)) * 4;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i0 + rr < nb) v = *reinterpret_cast<const float4*>(qp + (size_t)(i0 + rr) * D + d0 + cc);
+      if (i0 + rr < nq) v = *reinterpret_cast<const float4*>(qp + (size_t)(i0 + rr) * D + d0 + cc);
       qs[cc][rr] = v.x;
       qs[cc + 1][rr] = v.y;
       qs[cc + 2][rr] = v.z;
@@ -335,8 +335,8 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int i = i0 + 4 * ty + r;
-    if (i >= nb) continue;
-    uint32_t* dst = skeys + (bh * (size_t)nb + i) * nbp;
+    if (i >= nq) continue;
+    uint32_t* dst = skeys + (bh * (size_t)nq + i) * nbp;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int j = j0 + 64 * half + 4 * tx;
@@ -365,12 +365,12 @@ __global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t bh = blockIdx.y;
   const int i = blockIdx.x * 8 + warp;
-  if (i >= p.nb) return;
+  if (i >= p.nq) return;
   uint32_t* kr = rows + (size_t)warp * nbp;
-  const uint4* src = reinterpret_cast<const uint4*>(skeys + (bh * (size_t)p.nb + i) * nbp);
+  const uint4* src = reinterpret_cast<const uint4*>(skeys + (bh * (size_t)p.nq + i) * nbp);
   for (int e = lane; e < nbp / 4; e += 32) reinterpret_cast<uint4*>(kr)[e] = src[e];
   __syncwarp();
-  select_row_warp(p, kr, bh, bh * (size_t)p.nb + i, hist + warp * 256, lane);
+  select_row_warp(p, kr, bh, bh * (size_t)p.nq + i, hist + warp * 256, lane);
 }
 
 }  // namespace spark

@@ -12,6 +12,7 @@
 #include "pool.cuh"
 #include "select.cuh"
 #include "attn_tc.cuh"
+#include "attn_tc128.cuh"
 #include "reblock.cuh"
 
 using namespace spark;
@@ -27,6 +28,13 @@ inline int64_t num_blocks(const spark_shape* s) {
   return nv > 0 ? nv / kBlock : 0;
 }
 
+// Query tile of the route (64 or 128 rows) and the number of video query tiles.
+inline int q_tile_of(const spark_shape* s) { return s->q_tile == 0 ? kBlock : s->q_tile; }
+inline int64_t num_qtiles(const spark_shape* s) {
+  const int64_t nb = num_blocks(s);
+  return q_tile_of(s) == kBlock ? nb : (nb + 1) / 2;
+}
+
 inline float eff_scale(const spark_shape* s) {
   return s->scale > 0.f ? s->scale : 1.0f / std::sqrt((float)s->d);
 }
@@ -37,6 +45,7 @@ int check_shape(const spark_shape* s) {
   if (s->B < 0 || s->H < 0 || s->N < 0 || s->n_sink < 0 || s->n_sink > s->N) return SPARK_EINVAL;
   if (!(std::isfinite(s->scale))) return SPARK_EINVAL;
   if (s->block != kBlock) return SPARK_EUNSUPPORTED;
+  if (s->q_tile != 0 && s->q_tile != kBlock && s->q_tile != 2 * kBlock) return SPARK_EUNSUPPORTED;
   if (s->d != 64 && s->d != 128) return SPARK_EUNSUPPORTED;
   const int64_t bh = (int64_t)s->B * s->H;
   if (bh > 65535) return SPARK_EUNSUPPORTED;                       // grid.y of the pooling kernels
@@ -104,10 +113,9 @@ int num_sms() {
   return n;
 }
 
-template <int D>
+template <int D, bool Q128>
 int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, const void* pack,
                    cudaStream_t cs) {
-  using C = TcCfg<D>;
   TcMaps maps;
   const uint64_t rows = (uint64_t)tp.BH * tp.N;
   if (!bf16_tile_map(&maps.k, K, rows, D) || !bf16_tile_map(&maps.v, V, rows, D)) return SPARK_ECUDA;
@@ -120,15 +128,16 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
     maps.kp = maps.k;
     maps.vp = maps.v;
   }
-  const size_t smem = tc_smem_bytes<D>(tp.nb);
+  const size_t smem = Q128 ? tc128_smem_bytes<D>(tp.nb) : tc_smem_bytes<D>(tp.nb);
   if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
   const int sms = num_sms();
   if (sms <= 0) return SPARK_ECUDA;
-  const int grid = (int)std::min<int64_t>(sms, ((int64_t)tp.n_items + 1) / 2);
-  if (cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
+  // one CTA per SM; the 64-query kernel runs two items at a time per CTA
+  const int grid = (int)std::min<int64_t>(sms, Q128 ? (int64_t)tp.n_items : ((int64_t)tp.n_items + 1) / 2);
+  auto kern = Q128 ? attn_tc128_kernel<D> : attn_tc_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SPARK_ECUDA;
-  attn_tc_kernel<D><<<grid, C::kThreads, smem, cs>>>(maps, tp);
+  kern<<<grid, 384, smem, cs>>>(maps, tp);
   SPARK_LAUNCH_CHECK();
   note_launches(1);
   return SPARK_OK;
@@ -166,6 +175,11 @@ int32_t spark_num_blocks(const spark_shape* s) {
   return (int32_t)num_blocks(s);
 }
 
+int32_t spark_num_query_tiles(const spark_shape* s) {
+  if (check_shape(s) != SPARK_OK) return 0;
+  return (int32_t)num_qtiles(s);
+}
+
 int32_t spark_topk_count(double ratio, int32_t nb) {
   if (!(ratio > 0.0 && ratio <= 1.0)) return -1;
   if (nb <= 0) return 0;
@@ -183,7 +197,7 @@ size_t spark_workspace_bytes(const spark_shape* s, int call_id) {
     case SPARK_CALL_POOL:
       return pack_bias_offset(bh, nb, s->d) + bh * padded_blocks(nb) * sizeof(float);
     case SPARK_CALL_SELECT:
-      return select_scores_offset(bh) + bh * nb * select_row_stride(nb) * sizeof(uint32_t);
+      return select_scores_offset(bh) + bh * (size_t)num_qtiles(s) * select_row_stride(nb) * sizeof(uint32_t);
     case SPARK_CALL_ATTN:
       return 0;
     case SPARK_CALL_REBLOCK:
@@ -220,14 +234,21 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
   const int nbp = (int)padded_blocks(nb);
   const float scale = eff_scale(s);
   dim3 grid((nb + kPoolWarps - 1) / kPoolWarps, bh);
+  const int nt = (int)num_qtiles(s);
+  dim3 gq((nt + kPoolWarps - 1) / kPoolWarps, bh);
+  const bool q128 = q_tile_of(s) == 2 * kBlock;
+  const float last_w = (q128 && (nb & 1)) ? 0.5f : 1.0f;
+  const int nv = nb * kBlock;
   if (s->d == 128) {
-    pool_q_kernel<128><<<grid, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nb);
-    anchor_kernel<128><<<bh, 256, 0, cs>>>(q_pool, anchor, nb);
+    if (q128) pool_q_kernel<128, 128><<<gq, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nt, nv);
+    else pool_q_kernel<128, 64><<<gq, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nt, nv);
+    anchor_kernel<128><<<bh, 256, 0, cs>>>(q_pool, anchor, nt, last_w);
     pool_kv_kernel<128><<<grid, kPoolWarps * 32, 0, cs>>>(K, V, anchor, k_pool, v_summ, beta, k16,
                                                           v16, bl2, nbp, s->N, nb, scale, pool_mode);
   } else {
-    pool_q_kernel<64><<<grid, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nb);
-    anchor_kernel<64><<<bh, 256, 0, cs>>>(q_pool, anchor, nb);
+    if (q128) pool_q_kernel<64, 128><<<gq, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nt, nv);
+    else pool_q_kernel<64, 64><<<gq, kPoolWarps * 32, 0, cs>>>(Q, q_pool, s->N, nt, nv);
+    anchor_kernel<64><<<bh, 256, 0, cs>>>(q_pool, anchor, nt, last_w);
     pool_kv_kernel<64><<<grid, kPoolWarps * 32, 0, cs>>>(K, V, anchor, k_pool, v_summ, beta, k16,
                                                          v16, bl2, nbp, s->N, nb, scale, pool_mode);
   }
@@ -249,6 +270,7 @@ int score_select_impl(const spark_shape* s, const float* q_pool, const float* k_
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   const int nb = (int)num_blocks(s);
+  const int nq = (int)num_qtiles(s);
   const int bh = s->B * s->H;
   int k = 0;
   if (mode == SPARK_SELECT_TOPK_RATIO) {
@@ -279,11 +301,11 @@ int score_select_impl(const spark_shape* s, const float* q_pool, const float* k_
     thr = acc + bh;
     if (cudaMemsetAsync(acc, 0, (size_t)bh * sizeof(double), cs) != cudaSuccess) return SPARK_ECUDA;
     if (s->d == 128) {
-      moments_kernel<128><<<dim3(16, bh), 256, 0, cs>>>(q_pool, k_pool, nb, acc);
-      tau_threshold_kernel<128><<<bh, 128, 0, cs>>>(q_pool, k_pool, nb, acc, scale, param, thr);
+      moments_kernel<128><<<dim3(16, bh), 256, 0, cs>>>(q_pool, k_pool, nq, nb, acc);
+      tau_threshold_kernel<128><<<bh, 128, 0, cs>>>(q_pool, k_pool, nq, nb, acc, scale, param, thr);
     } else {
-      moments_kernel<64><<<dim3(4, bh), 256, 0, cs>>>(q_pool, k_pool, nb, acc);
-      tau_threshold_kernel<64><<<bh, 64, 0, cs>>>(q_pool, k_pool, nb, acc, scale, param, thr);
+      moments_kernel<64><<<dim3(4, bh), 256, 0, cs>>>(q_pool, k_pool, nq, nb, acc);
+      tau_threshold_kernel<64><<<bh, 64, 0, cs>>>(q_pool, k_pool, nq, nb, acc, scale, param, thr);
     }
     SPARK_LAUNCH_CHECK();
     note_launches(2);
@@ -294,6 +316,7 @@ int score_select_impl(const spark_shape* s, const float* q_pool, const float* k_
   sp.idx = idx;
   sp.cnt = cnt;
   sp.thr = thr;
+  sp.nq = nq;
   sp.nb = nb;
   sp.kcap = kcap;
   sp.k = k;
@@ -303,20 +326,20 @@ int score_select_impl(const spark_shape* s, const float* q_pool, const float* k_
   if (!fused) {
     const int nbp = (int)select_row_stride(nb);
     uint32_t* skeys = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + select_scores_offset(bh));
-    dim3 gs((nb + kScJ - 1) / kScJ, (nb + kScI - 1) / kScI, bh);
+    dim3 gs((nb + kScJ - 1) / kScJ, (nq + kScI - 1) / kScI, bh);
     if (s->d == 128)
-      score_tile_kernel<128><<<gs, 256, 0, cs>>>(q_pool, k_pool, nb, nbp, scale, skeys);
+      score_tile_kernel<128><<<gs, 256, 0, cs>>>(q_pool, k_pool, nq, nb, nbp, scale, skeys);
     else
-      score_tile_kernel<64><<<gs, 256, 0, cs>>>(q_pool, k_pool, nb, nbp, scale, skeys);
+      score_tile_kernel<64><<<gs, 256, 0, cs>>>(q_pool, k_pool, nq, nb, nbp, scale, skeys);
     const size_t smem_sel = (size_t)8 * nbp * 4 + 8 * 256 * 4;
     if (smem_sel > 227 * 1024) return SPARK_EUNSUPPORTED;
     cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_sel);
-    select_rows_kernel<<<dim3((nb + 7) / 8, bh), 256, smem_sel, cs>>>(sp, skeys, nbp);
+    select_rows_kernel<<<dim3((nq + 7) / 8, bh), 256, smem_sel, cs>>>(sp, skeys, nbp);
     SPARK_LAUNCH_CHECK();
     note_launches(2);
     return SPARK_OK;
   }
-  dim3 grid((nb + rt - 1) / rt, bh);
+  dim3 grid((nq + rt - 1) / rt, bh);
   if (s->d == 128) {
     cudaFuncSetAttribute(score_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     score_select_kernel<128><<<grid, kSelThreads, smem, cs>>>(sp);
@@ -371,8 +394,10 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
     if (pool_pack && !aligned16(pool_pack)) return SPARK_EINVAL;
   }
   const int nv = nb * kBlock;
-  const int n_dq = (s->N - nv + kBlock - 1) / kBlock;
-  const int64_t items = (int64_t)bh * (n_dq + nb);
+  const int qt = q_tile_of(s);
+  const int nt = (int)num_qtiles(s);
+  const int n_dq = (s->N - nv + qt - 1) / qt;
+  const int64_t items = (int64_t)bh * (n_dq + nt);
   if (items > 0x7fffffff) return SPARK_EUNSUPPORTED;
   if ((int64_t)bh * s->N >= ((int64_t)1 << 31)) return SPARK_EUNSUPPORTED;  // TMA row coordinates
   TcParams tp;
@@ -393,12 +418,15 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   tp.kcap = kcap;
   tp.BH = bh;
   tp.n_dq = n_dq;
+  tp.nt = nt;
   tp.pooled = (nb > 0 && pool_pack != nullptr) ? 1 : 0;
   tp.n_items = (int)items;
   tp.scale_log2 = eff_scale(s) * kLog2e;
   cudaStream_t cs = as_stream(stream);
   const void* pack = tp.pooled ? pool_pack : nullptr;
-  return s->d == 128 ? launch_attn_tc<128>(tp, K, V, pack, cs) : launch_attn_tc<64>(tp, K, V, pack, cs);
+  if (qt == 2 * kBlock)
+    return s->d == 128 ? launch_attn_tc<128, true>(tp, K, V, pack, cs) : launch_attn_tc<64, true>(tp, K, V, pack, cs);
+  return s->d == 128 ? launch_attn_tc<128, false>(tp, K, V, pack, cs) : launch_attn_tc<64, false>(tp, K, V, pack, cs);
 }
 
 }  // extern "C"

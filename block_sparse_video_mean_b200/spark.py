@@ -28,7 +28,8 @@ BLOCK = 64
 
 EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
            "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
-           "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches", "spark_reblock_kv")
+           "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches", "spark_reblock_kv",
+           "spark_num_query_tiles")
 NOALLOC_MAX_HEADS = 4096
 
 
@@ -41,7 +42,7 @@ class SparkError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("block", ctypes.c_int32),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("q_tile", ctypes.c_int32)]
 
 
 _lib = None
@@ -60,6 +61,8 @@ def load() -> ctypes.CDLL:
     SP = ctypes.POINTER(Shape)
     lib.spark_num_blocks.argtypes = [SP]
     lib.spark_num_blocks.restype = ctypes.c_int32
+    lib.spark_num_query_tiles.argtypes = [SP]
+    lib.spark_num_query_tiles.restype = ctypes.c_int32
     lib.spark_workspace_bytes.argtypes = [SP, I]
     lib.spark_workspace_bytes.restype = Z
     lib.spark_topk_count.argtypes = [D, ctypes.c_int32]
@@ -103,12 +106,17 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def make_shape(B, H, N, d, n_sink, scale=None) -> Shape:
-    return Shape(B, H, N, d, n_sink, BLOCK, float(scale) if scale else 0.0)
+def make_shape(B, H, N, d, n_sink, scale=None, q_tile=BLOCK) -> Shape:
+    return Shape(B, H, N, d, n_sink, BLOCK, float(scale) if scale else 0.0, int(q_tile))
 
 
 def num_blocks(shape: Shape) -> int:
     return int(load().spark_num_blocks(ctypes.byref(shape)))
+
+
+def num_query_tiles(shape: Shape) -> int:
+    """Video query tiles per head: nb, or ceil(nb / 2) on the 128-query route."""
+    return int(load().spark_num_query_tiles(ctypes.byref(shape)))
 
 
 def topk_count(ratio: float, nb: int) -> int:
@@ -130,9 +138,9 @@ def device_error(device=None) -> int:
     return int(word.value)
 
 
-def _shape_of(Q, n_sink, scale):
+def _shape_of(Q, n_sink, scale, q_tile=BLOCK):
     B, H, N, d = Q.shape
-    return make_shape(B, H, N, d, n_sink, scale)
+    return make_shape(B, H, N, d, n_sink, scale, q_tile)
 
 
 def _need(t, name):
@@ -142,17 +150,18 @@ def _need(t, name):
 
 # --------------------------------------------------------------------------- the four calls
 
-def pool_kv(Q, K, V, n_sink, pool_mode=POOL_REWEIGHT, scale=None, out=None):
-    """spark_pool_kv: returns dict(q_pool, k_pool, v_summ, beta, anchor, pack)."""
+def pool_kv(Q, K, V, n_sink, pool_mode=POOL_REWEIGHT, scale=None, out=None, q_tile=BLOCK):
+    """spark_pool_kv: returns dict(q_pool [B,H,nt,d], k_pool, v_summ, beta, anchor, pack)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, n)
-    shape = _shape_of(Q, n_sink, scale)
+    shape = _shape_of(Q, n_sink, scale, q_tile)
     B, H, N, d = Q.shape
     nb = num_blocks(shape)
+    nt = num_query_tiles(shape)
     dev = Q.device
     if out is None:
         out = dict(
-            q_pool=torch.empty((B, H, nb, d), dtype=torch.float32, device=dev),
+            q_pool=torch.empty((B, H, nt, d), dtype=torch.float32, device=dev),
             k_pool=torch.empty((B, H, nb, d), dtype=torch.float32, device=dev),
             v_summ=torch.empty((B, H, nb, d), dtype=torch.float32, device=dev),
             beta=torch.empty((B, H, nb), dtype=torch.float32, device=dev),
@@ -166,16 +175,18 @@ def pool_kv(Q, K, V, n_sink, pool_mode=POOL_REWEIGHT, scale=None, out=None):
     return out
 
 
-def score_select(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, out=None, ws=None):
-    """spark_score_select: returns (idx [B,H,nb,kcap] int32, cnt [B,H,nb] int32)."""
-    B, H, nb, d = q_pool.shape
-    shape = make_shape(B, H, N, d, n_sink, scale)
+def score_select(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, out=None, ws=None,
+                 q_tile=BLOCK):
+    """spark_score_select: returns (idx [B,H,nt,kcap] int32, cnt [B,H,nt] int32)."""
+    B, H, nt, d = q_pool.shape
+    nb = k_pool.shape[2]
+    shape = make_shape(B, H, N, d, n_sink, scale, q_tile)
     dev = q_pool.device
     if kcap is None:
         kcap = topk_count(param, nb) if mode == SELECT_TOPK_RATIO else max(nb, 1)
     if out is None:
-        out = (torch.empty((B, H, nb, max(kcap, 1)), dtype=torch.int32, device=dev),
-               torch.empty((B, H, nb), dtype=torch.int32, device=dev))
+        out = (torch.empty((B, H, nt, max(kcap, 1)), dtype=torch.int32, device=dev),
+               torch.empty((B, H, nt), dtype=torch.int32, device=dev))
     if ws is None:
         ws = torch.empty(max(workspace_bytes(shape, CALL_SELECT), 16), dtype=torch.uint8, device=dev)
     idx, cnt = out
@@ -186,17 +197,19 @@ def score_select(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, 
     return idx, cnt
 
 
-def score_select_noalloc(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, out=None):
+def score_select_noalloc(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scale=None, out=None,
+                         q_tile=BLOCK):
     """spark_score_select_noalloc: the selection without a scratch argument (the library
     uses its own fixed device array); returns (idx, cnt) like score_select."""
-    B, H, nb, d = q_pool.shape
-    shape = make_shape(B, H, N, d, n_sink, scale)
+    B, H, nt, d = q_pool.shape
+    nb = k_pool.shape[2]
+    shape = make_shape(B, H, N, d, n_sink, scale, q_tile)
     dev = q_pool.device
     if kcap is None:
         kcap = topk_count(param, nb) if mode == SELECT_TOPK_RATIO else max(nb, 1)
     if out is None:
-        out = (torch.empty((B, H, nb, max(kcap, 1)), dtype=torch.int32, device=dev),
-               torch.empty((B, H, nb), dtype=torch.int32, device=dev))
+        out = (torch.empty((B, H, nt, max(kcap, 1)), dtype=torch.int32, device=dev),
+               torch.empty((B, H, nt), dtype=torch.int32, device=dev))
     idx, cnt = out
     _check(load().spark_score_select_noalloc(ctypes.byref(shape), _ptr(q_pool), _ptr(k_pool),
                                              int(mode), float(param), int(kcap), _ptr(idx),
@@ -205,11 +218,11 @@ def score_select_noalloc(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scal
 
 
 def attn_fwd(Q, K, V, idx, cnt, n_sink, pack=None, beta=None, perm=None, scale=None,
-             out=None, lse=True):
+             out=None, lse=True, q_tile=BLOCK):
     """spark_attn_fwd: returns (O bf16 [B,H,N,d], LSE fp32 [B,H,N] or None)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, n)
-    shape = _shape_of(Q, n_sink, scale)
+    shape = _shape_of(Q, n_sink, scale, q_tile)
     B, H, N, d = Q.shape
     dev = Q.device
     if out is None:
@@ -279,6 +292,7 @@ class ForwardConfig:
     reblock_kv: bool = False    # with reblock: keys get their own partition
     scale: float | None = None
     kcap: int | None = None     # slots per selection row (default: k, or nb for tau)
+    q_tile: int = BLOCK         # query tile: 64, or 128 (the 128-query x 64-key route)
 
 
 class SparkAttention:
@@ -288,8 +302,9 @@ class SparkAttention:
     def __init__(self, B, H, N, d, n_sink, cfg: ForwardConfig, device="cuda"):
         self.cfg = cfg
         self.n_sink = n_sink
-        self.shape = make_shape(B, H, N, d, n_sink, cfg.scale)
+        self.shape = make_shape(B, H, N, d, n_sink, cfg.scale, cfg.q_tile)
         self.nb = nb = num_blocks(self.shape)
+        self.nt = nt = num_query_tiles(self.shape)
         dev = torch.device(device)
         self.mode = SELECT_TOPK_RATIO if cfg.mode == "topk" else SELECT_TAU
         if cfg.kcap is not None:
@@ -298,13 +313,13 @@ class SparkAttention:
             self.kcap = max(topk_count(cfg.param, nb) if self.mode == SELECT_TOPK_RATIO else nb, 1)
         self.pool_mode = POOL_REWEIGHT if cfg.pool_mode == "reweight" else POOL_MEAN
         f32 = dict(dtype=torch.float32, device=dev)
-        self.pool = dict(q_pool=torch.empty((B, H, nb, d), **f32), k_pool=torch.empty((B, H, nb, d), **f32),
+        self.pool = dict(q_pool=torch.empty((B, H, nt, d), **f32), k_pool=torch.empty((B, H, nb, d), **f32),
                          v_summ=torch.empty((B, H, nb, d), **f32), beta=torch.empty((B, H, nb), **f32),
                          anchor=torch.empty((B, H, d), **f32),
                          pack=torch.empty(max(workspace_bytes(self.shape, CALL_POOL), 16),
                                           dtype=torch.uint8, device=dev))
-        self.idx = torch.empty((B, H, nb, self.kcap), dtype=torch.int32, device=dev)
-        self.cnt = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+        self.idx = torch.empty((B, H, nt, self.kcap), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, H, nt), dtype=torch.int32, device=dev)
         self.sel_ws = torch.empty(max(workspace_bytes(self.shape, CALL_SELECT), 16), dtype=torch.uint8, device=dev)
         self.O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, H, N), **f32)
@@ -341,13 +356,14 @@ class SparkAttention:
                 reblock(Q, K, V, self.n_sink, out=self.rb, ws=self.rb_ws)
             Q, K, V, perm = self.rb["Qp"], self.rb["Kp"], self.rb["Vp"], self.rb["perm"]
         mark(1)
-        pool_kv(Q, K, V, self.n_sink, self.pool_mode, cfg.scale, out=self.pool)
+        pool_kv(Q, K, V, self.n_sink, self.pool_mode, cfg.scale, out=self.pool, q_tile=cfg.q_tile)
         mark(2)
         score_select(self.pool["q_pool"], self.pool["k_pool"], self.n_sink, Q.shape[2], self.mode,
-                     cfg.param, self.kcap, cfg.scale, out=(self.idx, self.cnt), ws=self.sel_ws)
+                     cfg.param, self.kcap, cfg.scale, out=(self.idx, self.cnt), ws=self.sel_ws,
+                     q_tile=cfg.q_tile)
         mark(3)
         attn_fwd(Q, K, V, self.idx, self.cnt, self.n_sink,
                  pack=self.pool["pack"] if cfg.compressed else None, beta=self.pool["beta"],
-                 perm=perm, scale=cfg.scale, out=(self.O, self.lse))
+                 perm=perm, scale=cfg.scale, out=(self.O, self.lse), q_tile=cfg.q_tile)
         mark(4)
         return self.O, self.lse

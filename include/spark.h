@@ -66,7 +66,18 @@ typedef struct spark_shape {
   int32_t n_sink;     /* sink/text rows at the end of each (b, h) */
   int32_t block;      /* video block size; must be 64 */
   float scale;        /* softmax scale; <= 0 selects 1/sqrt(d) */
+  int32_t q_tile;     /* query tile of the route: 64 (0 means 64) or 128 */
 } spark_shape;
+
+/* The query tile ("H3 Optimizations" README, section "Manual Sparse Sage recovery": the
+ * sparse backends consume a 128-query x 64-key route). With q_tile = 128 a query tile is
+ * two consecutive video blocks (the last one holds one block when nb is odd): q_pool has
+ * one row per tile (the mean of the tile's queries), the score and selection rows are the
+ * nt = ceil(nb / 2) tiles against the nb key blocks (k = spark_topk_count(ratio, nb); tau
+ * moments over all nt x nb scores), idx / cnt are [B, H, nt, kcap] / [B, H, nt], and every
+ * query of a tile attends to the tile's selection. Keys, the anchor, the compressed branch,
+ * the dense rows and Reblock do not change. With q_tile = 64, nt = nb. */
+int32_t spark_num_query_tiles(const spark_shape* s);
 
 /* Number of full video blocks nb = floor((N - n_sink) / 64) (0 when N <= n_sink). */
 int32_t spark_num_blocks(const spark_shape* s);
@@ -79,7 +90,7 @@ int32_t spark_num_blocks(const spark_shape* s);
  *                      2*B*H*nb*d*2 + B*H*nbp*4 bytes;
  *   SPARK_CALL_SELECT  scratch of spark_score_select: fp64 tau moments (2*B*H doubles,
  *                      padded to 256 bytes) and the score keys of every head
- *                      (B*H*nb*nbp uint32, nbp = nb rounded up to 4);
+ *                      (B*H*nt*nbp uint32, nbp = nb rounded up to 4);
  *   SPARK_CALL_ATTN    scratch of spark_attn_fwd (0: it needs none);
  *   SPARK_CALL_REBLOCK scratch of spark_reblock.
  * Returns 0 for an invalid shape or call id. */
@@ -91,8 +102,9 @@ int32_t spark_topk_count(double ratio, int32_t nb);
 
 /* Pooling, anchor and compressed-branch summaries ("What Spark-Attn changes",
  * Spark-Reweight bullet and the figure caption after it).
- * Per (b, h):  q_pool[i]  = mean of the 64 queries of video block i        fp32 [B,H,nb,d]
- *              anchor     = mean of all video queries (= mean of q_pool)   fp32 [B,H,d]
+ * Per (b, h):  q_pool[i]  = mean of the queries of query tile i           fp32 [B,H,nt,d]
+ *              anchor     = mean of all video queries (the row-weighted mean of q_pool)
+ *                                                                          fp32 [B,H,d]
  *              s_j        = anchor . k_j * scale for every video key j
  *              k_pool[i]  = mean of the 64 keys of block i                  fp32 [B,H,nb,d]
  *              v_summ[i]  = sum_j softmax_i(s)_j v_j (REWEIGHT) | mean v     fp32 [B,H,nb,d]
@@ -107,17 +119,18 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
                   float* anchor, void* pool_pack, size_t pool_pack_bytes, void* stream);
 
 /* Block scores and selection ("Block-sparse attention: one node, three backends").
- * S[i, j] = q_pool[i] . k_pool[j] * scale over video blocks, computed in fp32.
+ * S[i, j] = q_pool[i] . k_pool[j] * scale for query tile i (a block unless q_tile = 128)
+ * and video key block j, computed in fp32.
  *   mode SPARK_SELECT_TOPK_RATIO, param = ratio in (0, 1]: keeps the k =
  *       spark_topk_count(ratio, nb) largest scores of each row, ties to the lower j;
  *       requires kcap >= k.
  *   mode SPARK_SELECT_TAU, param = tau (finite): keeps S[i, j] > mu + tau * sigma,
- *       mu and sigma (population) over all nb^2 scores of the head, obtained in fp64
+ *       mu and sigma (population) over all nt*nb scores of the head, obtained in fp64
  *       from the d x d second moments of q_pool and k_pool. No per-row floor: a row
  *       may keep nothing. More than kcap kept blocks truncates the row to its first
  *       kcap indices and records SPARK_ECAPACITY (kcap = nb never overflows).
- * Outputs: idx int32 [B, H, nb, kcap] (per row, ascending block indices in the first
- * cnt slots; later slots unspecified), cnt int32 [B, H, nb].
+ * Outputs: idx int32 [B, H, nt, kcap] (per row, ascending block indices in the first
+ * cnt slots; later slots unspecified), cnt int32 [B, H, nt].
  * The scores are computed by a tiled fp32 kernel into ws and each row is selected from
  * there (per score: even and odd d terms in two fp32 chains, then scaled).
  * ws: spark_workspace_bytes(s, SPARK_CALL_SELECT) bytes, 16-byte aligned (both modes). */
@@ -127,7 +140,7 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
 
 /* Attention forward ("What Spark-Attn changes": exact + compressed branches merged in
  * one softmax; sink_conditioning: sink keys attended exactly; "Nodes": dense rows).
- * A video query of block i attends to the 64 keys of each selected block idx[i, :cnt[i]]
+ * A video query of tile i attends to the 64 keys of each selected block idx[i, :cnt[i]]
  * and to every dense key; when pool_pack is not NULL it also attends to one pooled
  * entry per unselected video block b, with logit q . k_pool[b] * scale + beta[b] and
  * value v_summ[b] (bf16 k_pool / v_summ and fp32 beta, all read from pool_pack; the
@@ -137,7 +150,9 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
  * perm (nullable) int32 [B, H, nb*64]: the inputs are in a reblocked order and output
  * row p of a video query is written to original row perm[p] (dense rows unchanged).
  * Outputs: O bf16 [B, H, N, d]; lse fp32 [B, H, N] natural-log (nullable).
- * Block indices outside [0, nb) are skipped and recorded as SPARK_EDEVICE_INDEX. */
+ * Block indices outside [0, nb) are skipped and recorded as SPARK_EDEVICE_INDEX.
+ * q_tile = 64 runs 64-query tiles on M = 64 tensor-core MMAs, q_tile = 128 runs 128-query
+ * tiles (dense rows too) on M = 128 MMAs. */
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
                    const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,

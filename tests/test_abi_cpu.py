@@ -55,6 +55,25 @@ def test_num_blocks_and_workspace(spark):
     assert spark.num_blocks(spark.make_shape(1, 1, 40, 64, 8)) == 0
 
 
+def test_query_tiles_of_the_128_query_route(spark):
+    s64 = spark.make_shape(1, 24, 175680 + 512, 128, 512)
+    s128 = spark.make_shape(1, 24, 175680 + 512, 128, 512, q_tile=128)
+    assert spark.num_query_tiles(s64) == 2745
+    assert spark.num_query_tiles(s128) == 1373          # the last tile holds one block
+    assert spark.num_query_tiles(spark.make_shape(1, 1, 64 * 4, 64, 0, q_tile=128)) == 2
+    # key-side buffers do not change; the score keys have one row per tile
+    assert spark.workspace_bytes(s128, spark.CALL_POOL) == spark.workspace_bytes(s64, spark.CALL_POOL)
+    off = (2 * 24 * 8 + 255) // 256 * 256
+    assert spark.workspace_bytes(s128, spark.CALL_SELECT) == off + 24 * 1373 * 2748 * 4
+    assert spark.workspace_bytes(s64, spark.CALL_SELECT) == off + 24 * 2745 * 2748 * 4
+    lib = spark.load()
+    bad_tile = spark.make_shape(1, 1, 128, 64, 0, q_tile=96)
+    dummy = ctypes.c_void_p(16)
+    assert lib.spark_attn_fwd(ctypes.byref(bad_tile), dummy, dummy, dummy, dummy, dummy, 1, None,
+                              None, None, dummy, None, None, 0, None) == -2
+    assert spark.num_query_tiles(bad_tile) == 0
+
+
 def test_bad_arguments_are_rejected_on_the_host(spark):
     lib = spark.load()
     P = ctypes.c_void_p
@@ -62,7 +81,7 @@ def test_bad_arguments_are_rejected_on_the_host(spark):
     bad_d = spark.make_shape(1, 1, 128, 96, 0)
     assert lib.spark_pool_kv(ctypes.byref(bad_d), dummy, dummy, dummy, 0, dummy, dummy, dummy,
                              dummy, dummy, dummy, 1 << 20, None) == -2
-    bad_block = spark.Shape(1, 1, 128, 64, 0, 32, 0.0)
+    bad_block = spark.Shape(1, 1, 128, 64, 0, 32, 0.0, 0)
     assert lib.spark_attn_fwd(ctypes.byref(bad_block), dummy, dummy, dummy, dummy, dummy, 1, None,
                               None, None, dummy, None, None, 0, None) == -2
     neg = spark.make_shape(1, 1, 128, 64, 200)

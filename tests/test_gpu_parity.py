@@ -39,12 +39,14 @@ def head_f64(Q, K, V, b, h):
 
 
 def compare_head(plan, O, L, Q, K, V, b, h, ns, cfg, qblocks=None, check_pool=True, dense=True):
-    """Compare one head (all or sampled query blocks) against the oracle."""
+    """Compare one head (all or sampled query tiles: blocks, or pairs of blocks on the
+    128-query route) against the oracle."""
     q, k, v = head_f64(Q, K, V, b, h)
     scale = cfg.scale or 1.0 / math.sqrt(q.shape[1])
-    P = orc.pool_head(q, k, v, ns, scale, 64, cfg.pool_mode)
-    nb = P.qbar.shape[0]
-    blocks = np.arange(nb) if qblocks is None else np.asarray(qblocks)
+    qt = cfg.q_tile
+    P = orc.pool_head(q, k, v, ns, scale, 64, cfg.pool_mode, qt)
+    nb = P.kbar.shape[0]
+    blocks = np.arange(P.qbar.shape[0]) if qblocks is None else np.asarray(qblocks)
     if check_pool and nb:
         gp = {n: plan.pool[n][b, h].cpu().double().numpy() for n in ("q_pool", "k_pool", "v_summ", "beta", "anchor")}
         np.testing.assert_allclose(gp["q_pool"], P.qbar, atol=2e-6, rtol=0)
@@ -64,8 +66,8 @@ def compare_head(plan, O, L, Q, K, V, b, h, ns, cfg, qblocks=None, check_pool=Tr
     Og = O[b, h].float().cpu().numpy()
     Lg = L[b, h].cpu().numpy()
     for i in blocks:
-        o, l = orc.attn_video_block(q, k, v, ns, i, sel[i], pooled, scale)
-        rows = slice(i * 64, (i + 1) * 64)
+        o, l = orc.attn_video_block(q, k, v, ns, i, sel[i], pooled, scale, 64, qt)
+        rows = orc.tile_rows(i, nb * 64, qt)
         check_output(Og[rows], o, f"head {b},{h} block {i}")
         check_lse(Lg[rows], l, f"head {b},{h} block {i}")
     N = q.shape[0]
