@@ -12,16 +12,19 @@
 // * TMEM (512 columns): S/P double buffer (2 x 128 columns), O (D columns), Q double
 //   buffer (2 x D/2 columns, bf16 pairs: the A operand of the S MMAs). Row r of the tile
 //   is TMEM lane r.
-// * Warp roles: warps 0-7 softmax (warp w reads lane quadrant w % 4; warps w and w + 4
-//   split the 128 keys of a tile and the D columns of O in halves), warp 8 fills the K
-//   ring, warp 10 the V ring (TMA), warp 9 issues the S MMAs (and owns TMEM), warp 11 the
-//   PV MMAs. With two issuers the tensor pipe gets S(t + 1) while PV(t) waits for its P.
+// * Warp roles: warps 0-7 softmax (warp w owns rows 32 (w % 4) + 16 (w / 4) .. + 15 of its
+//   lane quadrant; lanes 0-15 take keys 0-63 of those rows and lanes 16-31 keys 64-127,
+//   through the 16-lane x 2 TMEM access shape), warp 8 fills the K ring, warp 10 the V
+//   ring (TMA), warp 9 issues the S MMAs (and owns TMEM), warp 11 the PV MMAs. With two
+//   issuers the tensor pipe gets S(t + 1) while PV(t) waits for its P.
 // * Per tile of 128 keys: S = Q K^T (D/16 MMAs 128x128x16, Q from TMEM); each softmax
-//   thread takes 64 keys of one row; the two halves of a row exchange their maxima
-//   through shared memory under an mbarrier per warp pair; the running max is lazy (O is
-//   rescaled only when it grows by more than 2^8); P is written as bf16 over the thread's
-//   own S columns (64h .. 64h + 31), so no warp overwrites S that another warp still
-//   reads; O += P V (8 MMAs 128xDx16, the A columns of each key half taken from where
+//   thread takes 64 keys of one row and the two halves of a row meet in one warp shuffle;
+//   the running max is lazy (O is rescaled only when it grows by more than 2^8), so the
+//   exponentials are taken against the running max first, with the row max alongside, and
+//   redone (from the logits, still in registers) only on the rare tiles that raise it; the
+//   softmax warps are bound by their instruction stream, so scale, subtract and row sums
+//   use packed fp32 pairs; P is written as bf16 over the thread's own S columns (64h ..
+//   64h + 31); O += P V (8 MMAs 128xDx16, the A columns of each key half taken from where
 //   that half's P lives).
 // * Every mbarrier wait is bounded; a timeout records SPARK_ETIMEOUT, raises the CTA abort
 //   flag, the TMA roles drain their copies in flight and TMEM is released.
@@ -29,6 +32,24 @@
 #include "attn_tc.cuh"
 
 namespace spark {
+
+// Packed fp32 pairs: one fma.rn.f32x2 / add.rn.f32x2 does the work of two FMAs / ADDs.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
 
 template <int D>
 struct Tc128Cfg {
@@ -43,13 +64,12 @@ struct Tc128Cfg {
   static constexpr int kThreads = 384;
   static constexpr int kRingBytes = 2 * kStages * kTileBytes;
   static constexpr int kBarBytes = 1024;
-  static constexpr int kXchgBytes = (2 * 2 * 128 + 2 * 128) * 4;  // row maxima [2][2][128], sums [2][128]
 };
 
 template <int D>
 __host__ __device__ inline size_t tc128_smem_bytes(int nb) {
   using C = Tc128Cfg<D>;
-  return 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes + C::kXchgBytes +
+  return 1024 /*alignment slack*/ + C::kRingBytes + C::kBarBytes +
          (size_t)8 * 2 * tc_bitmap_words(nb) * 4;  // two bitmaps per softmax warp
 }
 
@@ -118,12 +138,9 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* ofree = qfull + 2;            // the epilogue has read O
   uint64_t* odone = ofree + 1;            // last PV of an item completed
   uint64_t* finbar = odone + 1;           // [issuer]: all its MMAs completed
-  uint64_t* pairbar = finbar + 2;         // [warp pair][max buffer 0, 1 | sums]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pairbar + 12);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* xmax = reinterpret_cast<float*>(ring + C::kRingBytes + C::kBarBytes);  // [2][2][128]
-  float* xsum = xmax + 2 * 2 * 128;                                              // [2][128]
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(xsum + 2 * 128);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -143,7 +160,6 @@ __global__ void __launch_bounds__(384, 1)
     tc::mbar_init(oready, 1);
     tc::mbar_init(ofree, 8);
     tc::mbar_init(odone, 1);
-    for (int i = 0; i < 12; ++i) tc::mbar_init(&pairbar[i], 64);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -321,13 +337,12 @@ __global__ void __launch_bounds__(384, 1)
   } else {
     tc::regs_inc<200>();
     // ================================================================ softmax
-    const int w = warp & 3;              // TMEM lane quadrant: rows 32w .. 32w + 31
-    const int h = warp >> 2;             // key half of a tile, column half of O and Q
-    const int r = 32 * w + lane;         // query row within the tile
-    const uint32_t lanes = (uint32_t)(32 * w) << 16;
+    const int row0 = 32 * (warp & 3) + 16 * (warp >> 2);  // the warp's 16 rows (one lane quadrant)
+    const int r = row0 + (lane & 15);    // query row within the tile
+    const int h = lane >> 4;             // key half of a tile, column half of O and Q
+    const uint32_t lanes = (uint32_t)row0 << 16;
     const int nbwp = tc_bitmap_words(p.nb);
     uint32_t* bm2 = bitmap + warp * 2 * nbwp;  // this warp's two selection bitmaps
-    uint64_t* pb = pairbar + 3 * w;            // this warp pair's exchange barriers
     bool ok = true;
 
     // ---- preparation of an item: the thread's half Q row into a TMEM Q buffer (then
@@ -348,7 +363,7 @@ __global__ void __launch_bounds__(384, 1)
         }
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tc::tmem_st_32x32b_x16(tbase + lanes + C::kColQ + qb * (D / 2) + h * (D / 4) + 16 * c, qv + 16 * c);
+          tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + qb * (D / 2) + 16 * c, qv + 16 * c);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
@@ -392,18 +407,14 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t o[D / 2];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c)
-        tc::tmem_ld_32x32b_x16(tbase + lanes + C::kColO + h * (D / 2) + 16 * c, o + 16 * c);
+        tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, o + 16 * c);
       tc::tmem_wait_ld();
       // O is in registers: the next item's first PV may overwrite it
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(ofree);
-      // the row's total: this half's sum and the partner warp's
-      xsum[h * 128 + r] = l_run;
-      tc::mbar_arrive(&pb[2]);
-      if (!tc::mbar_wait(&pb[2], ndone & 1, abort_flag)) return false;
       ++ndone;
-      const float l_tot = l_run + xsum[(1 - h) * 128 + r];
+      const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float inv = l_tot > 0.f ? 1.0f / l_tot : 0.f;
       int orow = I.q0 + r;
       bool write = r < I.nq;
@@ -491,8 +502,8 @@ __global__ void __launch_bounds__(384, 1)
         float x[64];
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          tc::tmem_ld_32x32b_x16(tbase + lanes + C::kColS + 128 * b + 64 * h + 16 * c,
-                                 reinterpret_cast<uint32_t*>(x) + 16 * c);
+          tc::tmem_ld_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * c,
+                                       reinterpret_cast<uint32_t*>(x) + 16 * c);
         tc::tmem_wait_ld();
         // ---- logits (base 2) and masks of this half
         if (kind != kHalfPooled) {
@@ -534,7 +545,29 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         const float xs = kind == kHalfPooled ? 1.0f : p.scale_log2;  // factor still to apply
-        // row max: this half's 64 keys, then the partner warp's half of the same row
+        // exponentials against the running max first (it rarely moves), the row max
+        // alongside; when a row's max grew by more than 2^8 the warp redoes them
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        auto exps = [&](float m_use) {
+          float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          const float2 s2 = make_float2(xs, xs), m2 = make_float2(-m_use, -m_use);
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int e = 32 * hc + 2 * j;
+              const float2 a2 = ffma2(make_float2(x[e], x[e + 1]), s2, m2);
+              const float p0 = ex2f(a2.x);
+              const float p1 = ex2f(a2.y);
+              l2[j & 1] = fadd2(l2[j & 1], make_float2(p0, p1));
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+            tc::tmem_st_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
+          }
+          ls[0] = l2[0].x; ls[1] = l2[0].y; ls[2] = l2[1].x; ls[3] = l2[1].y;
+        };
+        exps(m_run == -INFINITY ? 0.f : m_run);
         float mx;
         {
           float a0 = x[0], a1 = x[1], a2 = x[2], a3 = x[3];
@@ -547,52 +580,34 @@ __global__ void __launch_bounds__(384, 1)
           }
           mx = max3f(max3f(a0, a1, a2), a3, a3) * xs;
         }
-        xmax[(2 * b + h) * 128 + r] = mx;
-        tc::mbar_arrive(&pb[b]);
-        if (!tc::mbar_wait(&pb[b], (g >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        mx = fmaxf(mx, xmax[(2 * b + 1 - h) * 128 + r]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run, mx);
         const bool need = m_new > m_run + 8.0f;  // also true when m_run = -inf and m_new finite
-        const float alpha = need ? ex2f(m_run - m_new) : 1.0f;
-        if (__any_sync(0xffffffffu, need && t > 0)) {
-          // rescale this thread's half of its O row once the previous PV has landed
-          if (!tc::mbar_wait(oready, (g - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2f(m_run - m_new) : 1.0f;
+          if (t > 0) {
+            // rescale this thread's half of its O row once the previous PV has landed
+            if (!tc::mbar_wait(oready, (g - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc::tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t v[16];
+              tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+              tc::tmem_st_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
+            }
           }
-          tc::tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[16];
-            tc::tmem_ld_32x32b_x16(tbase + lanes + C::kColO + h * (D / 2) + 16 * c, v);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-            tc::tmem_st_32x32b_x16(tbase + lanes + C::kColO + h * (D / 2) + 16 * c, v);
+          if (need) {
+            l_run *= alpha;
+            m_run = m_new;
           }
-        }
-        if (need) {
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
-        // P over this half's own S columns (64h .. 64h + 31), 32 keys at a time
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int e = 32 * hc + 2 * j;
-            const float p0 = ex2f(fmaf(x[e], xs, -m_use));
-            const float p1 = ex2f(fmaf(x[e + 1], xs, -m_use));
-            ls[j & 3] += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
-          }
-          tc::tmem_st_32x32b_x16(tbase + lanes + C::kColS + 128 * b + 64 * h + 16 * hc, pk);
+          tc::tmem_wait_st();
+          exps(m_run == -INFINITY ? 0.f : m_run);
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tc::tmem_wait_st();

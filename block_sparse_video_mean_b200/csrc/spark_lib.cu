@@ -137,7 +137,7 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
   auto kern = Q128 ? attn_tc128_kernel<D> : attn_tc_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SPARK_ECUDA;
-  kern<<<grid, 384, smem, cs>>>(maps, tp);
+  kern<<<grid, Q128 ? Tc128Cfg<D>::kThreads : TcCfg<D>::kThreads, smem, cs>>>(maps, tp);
   SPARK_LAUNCH_CHECK();
   note_launches(1);
   return SPARK_OK;
