@@ -738,20 +738,24 @@ __global__ void __launch_bounds__(384, 1)
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
         // P over S (packed columns 32h .. 32h+31 of the buffer), 32 keys at a time
+        {
+          float2 l2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          const float2 s2 = make_float2(xs, xs), m2 = make_float2(-m_use, -m_use);
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t pk[16];
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int e = 32 * hc + 2 * j;
-            const float a0 = fmaf(x[e], xs, -m_use);
-            const float a1 = fmaf(x[e + 1], xs, -m_use);
-            const float p0 = ex2f(a0);
-            const float p1 = ex2f(a1);
-            ls[j & 3] += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
+            for (int j = 0; j < 16; ++j) {
+              const int e = 32 * hc + 2 * j;
+              const float2 a2 = tc::ffma2(make_float2(x[e], x[e + 1]), s2, m2);
+              const float p0 = ex2f(a2.x);
+              const float p1 = ex2f(a2.y);
+              l2[j & 1] = tc::fadd2(l2[j & 1], make_float2(p0, p1));
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+            tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
           }
-          tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
+          ls[0] = l2[0].x; ls[1] = l2[0].y; ls[2] = l2[1].x; ls[3] = l2[1].y;
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         SPARK_TC_ACC(17, t_ex);

@@ -33,24 +33,6 @@
 
 namespace spark {
 
-// Packed fp32 pairs: one fma.rn.f32x2 / add.rn.f32x2 does the work of two FMAs / ADDs.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
 template <int D>
 struct Tc128Cfg {
   static constexpr int kStages = 2;
@@ -557,10 +539,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int e = 32 * hc + 2 * j;
-              const float2 a2 = ffma2(make_float2(x[e], x[e + 1]), s2, m2);
+              const float2 a2 = tc::ffma2(make_float2(x[e], x[e + 1]), s2, m2);
               const float p0 = ex2f(a2.x);
               const float p1 = ex2f(a2.y);
-              l2[j & 1] = fadd2(l2[j & 1], make_float2(p0, p1));
+              l2[j & 1] = tc::fadd2(l2[j & 1], make_float2(p0, p1));
               pk[j] = pack_bf16x2(p0, p1);
             }
             tc::tmem_st_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
