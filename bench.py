@@ -115,11 +115,11 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-# DRAM bytes (read + write) of one attention launch at the default workload: the
-# dram__bytes_read.sum + dram__bytes_write.sum of a 2-head capture of the same shape
-# (profiles/attn_tc_1152x640x243_h2_full.md), scaled by 12 to 24 heads. None once the
-# kernel has changed since it was measured.
-ATTN_TRAFFIC_BYTES = 57.2e9
+# DRAM bytes (read + write) of one attention launch: the dram__bytes_read.sum +
+# dram__bytes_write.sum of a 2-head capture of the same shape, scaled by 12 to 24 heads
+# (profiles/attn_tc_1152x640x243_h2_full.md, profiles/attn_tc128_1152x640x243_h2_full.md).
+# A workload without a capture of its current kernel reports None.
+ATTN_TRAFFIC_BYTES = {"1152x640x243": 57.2e9, "1152x640x243-q128": 31.3e9}
 
 
 class ClockSampler:
@@ -304,7 +304,6 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     achieved = fl["attn_total"] / (attn_ms * 1e-3) / 1e12
     value = world * fl["dense_equiv"] / (ms_step * 1e-3) / 1e12
     clocks = clk.summary()
-    default = (w.name == DEFAULT and h == w.H)
 
     def gbs(nbytes, t_ms):
         return round(nbytes / (t_ms * 1e-3) / 1e9, 1) if t_ms > 0 else None
@@ -354,7 +353,7 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
                      "frac": round(achieved / (bf16_sust or bf16_peak), 4),
                      "peak_source": f"{peak_src} bf16 sustained (burst {bf16_peak})",
                      "algorithmic_flops_per_launch": fl["attn_total"],
-                     "traffic": ATTN_TRAFFIC_BYTES if default else None},
+                     "traffic": ATTN_TRAFFIC_BYTES.get(w.name) if not args.heads else None},
         "e2e": {"value": round(world * fl["dense_equiv"] / (e2e_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s dense-equivalent, host buffers, copies inside the timed region",
                 "ms_per_step": round(e2e_ms, 3),
