@@ -67,6 +67,48 @@ struct TcParams {
   int N, nb, nbp, kcap, BH, n_dq, pooled, n_items;
   int nt;  // video query tiles per head (the 128-query route; nb for 64-query tiles)
   float scale_log2;
+  int* item_ctr;  // per-launch counter of items handed out (zeroed before the launch)
+};
+
+// Items handed out at run time: the claiming warp takes the next item index from the
+// launch's counter and publishes it in a ring of shared-memory entries; every other role
+// of the CTA reads the same entries in the same order. Longer items (the dense ones come
+// first) and rows of varying length (tau) then spread over the CTAs as they free up.
+constexpr int kQueueLen = 16;
+struct TcQueue {
+  int* ids;         // [kQueueLen] item index, -1 after the last item
+  uint64_t* full;   // [kQueueLen] arrival: the claimer wrote the entry
+  uint64_t* empty;  // [kQueueLen] arrivals: every reader took the entry
+  // The claiming warp (all lanes): entry j gets the next item index (or -1).
+  __device__ __forceinline__ bool claim(uint32_t j, const TcParams& p, volatile int* abort_flag, int* id) {
+    const int e = j % kQueueLen;
+    const bool ok = j < (uint32_t)kQueueLen || tc::mbar_wait(&empty[e], ((j / kQueueLen) - 1) & 1, abort_flag);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    int v = 0;
+    if ((threadIdx.x & 31) == 0) {
+      v = atomicAdd(p.item_ctr, 1);
+      if (v >= p.n_items) v = -1;
+      ids[e] = v;
+      tc::mbar_arrive(&full[e]);
+    }
+    *id = __shfl_sync(0xffffffffu, v, 0);
+    return true;
+  }
+  // A reading warp (all lanes) or a single reading thread (one_thread): entry j.
+  __device__ __forceinline__ bool read(uint32_t j, volatile int* abort_flag, int* id, bool one_thread) {
+    const int e = j % kQueueLen;
+    bool ok = tc::mbar_wait(&full[e], (j / kQueueLen) & 1, abort_flag);
+    if (!one_thread) ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    *id = ids[e];
+    if (one_thread) {
+      tc::mbar_arrive(&empty[e]);
+    } else {
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) tc::mbar_arrive(&empty[e]);
+    }
+    return true;
+  }
 };
 
 template <int D>
@@ -545,10 +587,10 @@ __global__ void __launch_bounds__(384, 1)
       ++ndone;
       tc::tc_fence_after();
       uint32_t o[D / 2];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c)
-        tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, o + 16 * c);
-      tc::tmem_wait_ld();
+      if constexpr (D == 128)
+        tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColO, o);
+      else
+        tc::tmem_ld_16x32bx2_x32_sync<32>(tbase + lanes + C::kColO, o);
       // O is in registers: the next item's first PV may overwrite it
       tc::tc_fence_before();
       __syncwarp();
@@ -642,11 +684,7 @@ __global__ void __launch_bounds__(384, 1)
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h+63 of the S buffer)
         float x[64];
         SPARK_TC_T0(t_ld);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tc::tmem_ld_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * c,
-                                       reinterpret_cast<uint32_t*>(x) + 16 * c);
-        tc::tmem_wait_ld();
+        tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, reinterpret_cast<uint32_t*>(x));
         SPARK_TC_ACC(6, t_ld);
         SPARK_TC_T0(t_cp);
         // ---- logits (base 2) and masks of this half
@@ -722,8 +760,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t v[16];
-            tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
-            tc::tmem_wait_ld();
+            tc::tmem_ld_16x32bx2_x16_sync<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
             tc::tmem_st_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);

@@ -120,8 +120,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* ofree = qfull + 2;            // the epilogue has read O
   uint64_t* odone = ofree + 1;            // last PV of an item completed
   uint64_t* finbar = odone + 1;           // [issuer]: all its MMAs completed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 2);
+  TcQueue queue;                          // items handed out at run time (warp 8 claims)
+  queue.full = finbar + 2;
+  queue.empty = queue.full + kQueueLen;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(queue.empty + kQueueLen);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  queue.ids = const_cast<int*>(abort_flag) + 1;
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -142,6 +146,10 @@ __global__ void __launch_bounds__(384, 1)
     tc::mbar_init(oready, 1);
     tc::mbar_init(ofree, 8);
     tc::mbar_init(odone, 1);
+    for (int i = 0; i < kQueueLen; ++i) {
+      tc::mbar_init(&queue.full[i], 1);
+      tc::mbar_init(&queue.empty[i], 11);  // V producer, two issuers, 8 softmax warps
+    }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -175,11 +183,42 @@ __global__ void __launch_bounds__(384, 1)
     unsigned char* rbase = is_v ? vring : ring;
     const CUtensorMap* map_x = is_v ? &maps.v : &maps.k;
     const CUtensorMap* map_p = is_v ? &maps.vp : &maps.kp;
-    // The whole warp walks the tile sequence; the selected block indices are fetched 32
-    // halves at a time, one chunk ahead.
-    Tc128Walk walk = {(int)blockIdx.x, (int)gridDim.x, p.n_items};
+    // The whole warp walks the tile sequence (warp 8 claims the items, warp 10 reads
+    // them from the queue); the selected block indices are fetched 32 halves at a time,
+    // one chunk ahead.
+    uint32_t qj = 0;
+    bool ok = true;
+    auto take_nonempty = [&](TcItem* I) -> bool {
+      while (true) {
+        int id;
+        if (!(is_v ? queue.read(qj, abort_flag, &id, false) : queue.claim(qj, p, abort_flag, &id))) {
+          ok = false;
+          return false;
+        }
+        ++qj;
+        if (id < 0) return false;
+        *I = tc128_item(p, id);
+        if (I->ntiles > 0) return true;
+      }
+    };
+    // warp 8 keeps one non-empty item claimed ahead of the one it loads, so that every
+    // reader of the queue finds the next item already published when it starts an item
+    TcItem ahead_item;
+    bool have_ahead = false;
+    auto next_nonempty = [&](TcItem* I) -> bool {
+      if (is_v) return take_nonempty(I);
+      bool have_now;
+      if (qj == 0) {
+        have_now = take_nonempty(I);
+      } else {
+        have_now = have_ahead;
+        *I = ahead_item;
+      }
+      have_ahead = have_now && take_nonempty(&ahead_item);
+      return have_now && ok;
+    };
     TcItem cur;
-    bool have = walk.next_nonempty(p, &cur);
+    bool have = next_nonempty(&cur);
     int t = 0;
     int ic = 0, in = 0;  // idx of halves 32c + lane (current / next chunk)
     if (have && !cur.dense) {
@@ -187,7 +226,6 @@ __global__ void __launch_bounds__(384, 1)
       in = 32 + lane < cur.cnt ? p.idx[cur.row * (size_t)p.kcap + 32 + lane] : 0;
     }
     uint32_t q = 0;
-    bool ok = true;
     while (ok && have) {
       const int stage = q % C::kStages;
       if (q >= (uint32_t)C::kStages &&
@@ -229,7 +267,7 @@ __global__ void __launch_bounds__(384, 1)
       ++q;
       if (++t == cur.ntiles) {
         t = 0;
-        have = walk.next_nonempty(p, &cur);
+        have = next_nonempty(&cur);
         if (have && !cur.dense) {
           ic = lane < cur.cnt ? p.idx[cur.row * (size_t)p.kcap + lane] : 0;
           in = 32 + lane < cur.cnt ? p.idx[cur.row * (size_t)p.kcap + 32 + lane] : 0;
@@ -255,12 +293,25 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idPV = tc::make_idesc_bf16(128, D, 0, 1);
       const uint32_t ring_addr = tc::smem_addr(ring);
       const uint32_t vring_addr = tc::smem_addr(vring);
-      Tc128Walk walk = {(int)blockIdx.x, (int)gridDim.x, p.n_items};
+      uint32_t qj = 0;
+      bool ok = true;
+      auto next_nonempty = [&](TcItem* I) -> bool {
+        while (true) {
+          int id;
+          if (!queue.read(qj, abort_flag, &id, true)) {
+            ok = false;
+            return false;
+          }
+          ++qj;
+          if (id < 0) return false;
+          *I = tc128_item(p, id);
+          if (I->ntiles > 0) return true;
+        }
+      };
       TcItem cur;
-      bool have = walk.next_nonempty(p, &cur);
+      bool have = next_nonempty(&cur);
       uint32_t g = 0, nitem = 0;
       int t = 0;
-      bool ok = true;
       while (ok && have) {
         const uint32_t b = g & 1;
         const int stage = g % C::kStages;
@@ -308,7 +359,7 @@ __global__ void __launch_bounds__(384, 1)
         if (++t == cur.ntiles) {
           t = 0;
           ++nitem;
-          have = walk.next_nonempty(p, &cur);
+          have = next_nonempty(&cur);
         }
       }
       // every MMA of this issuer must be complete before TMEM is released
@@ -387,10 +438,10 @@ __global__ void __launch_bounds__(384, 1)
       if (!tc::mbar_wait(odone, ndone & 1, abort_flag)) return false;
       tc::tc_fence_after();
       uint32_t o[D / 2];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c)
-        tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, o + 16 * c);
-      tc::tmem_wait_ld();
+      if constexpr (D == 128)
+        tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColO, o);
+      else
+        tc::tmem_ld_16x32bx2_x32_sync<32>(tbase + lanes + C::kColO, o);
       // O is in registers: the next item's first PV may overwrite it
       tc::tc_fence_before();
       __syncwarp();
@@ -424,12 +475,18 @@ __global__ void __launch_bounds__(384, 1)
       return true;
     };
 
-    // Items in order; an item with nothing to attend to gets O = 0, LSE = -inf.
-    Tc128Walk walk = {(int)blockIdx.x, (int)gridDim.x, p.n_items};
+    // Items in the queue's order; an item with nothing to attend to gets O = 0, LSE = -inf.
+    uint32_t qj = 0;
     auto next_item = [&](TcItem* I) -> bool {
-      while (walk.it < walk.n) {
-        *I = tc128_item(p, walk.it);
-        walk.it += walk.stride;
+      while (true) {
+        int id;
+        if (!queue.read(qj, abort_flag, &id, false)) {
+          ok = false;
+          return false;
+        }
+        ++qj;
+        if (id < 0) return false;
+        *I = tc128_item(p, id);
         if (I->ntiles > 0) return true;
         if (r < I->nq) {
           int orow = I->q0 + r;
@@ -447,7 +504,6 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      return false;
     };
 
     uint32_t g = 0;  // tiles processed (all items)
@@ -457,13 +513,14 @@ __global__ void __launch_bounds__(384, 1)
     bool have_prev = false;
     float m_prev = -INFINITY, l_prev = 0.f;
     bool have = next_item(&I);
-    Tc128Walk ahead = walk;  // finds the next non-empty item one ahead
     if (have) prepare(I, 0);
     int cur_bad = bad_next;
     bad_next = 0;
     while (ok && have) {
+      // the next item (published before this item's first copies were issued)
       TcItem nxt;
-      const bool have_nxt = ahead.next_nonempty(p, &nxt);
+      const bool have_nxt = next_item(&nxt);
+      if (!ok) break;
       const uint32_t* bm = bm2 + (n & 1) * nbwp;
 
       float m_run = -INFINITY, l_run = 0.f;
@@ -482,11 +539,7 @@ __global__ void __launch_bounds__(384, 1)
         tc::tc_fence_after();
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h + 63 of the buffer)
         float x[64];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tc::tmem_ld_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * c,
-                                       reinterpret_cast<uint32_t*>(x) + 16 * c);
-        tc::tmem_wait_ld();
+        tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, reinterpret_cast<uint32_t*>(x));
         // ---- logits (base 2) and masks of this half
         if (kind != kHalfPooled) {
           int valid = kBlock;
@@ -577,8 +630,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t v[16];
-              tc::tmem_ld_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
-              tc::tmem_wait_ld();
+              tc::tmem_ld_16x32bx2_x16_sync<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
 #pragma unroll
               for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
               tc::tmem_st_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
@@ -613,7 +665,8 @@ __global__ void __launch_bounds__(384, 1)
       l_prev = l_run;
       cur_bad = bad_next;
       bad_next = 0;
-      have = next_item(&I);
+      I = nxt;
+      have = have_nxt;
       ++n;
     }
     if (ok && have_prev) epilogue(prev, m_prev, l_prev);

@@ -199,7 +199,7 @@ size_t spark_workspace_bytes(const spark_shape* s, int call_id) {
     case SPARK_CALL_SELECT:
       return select_scores_offset(bh) + bh * (size_t)num_qtiles(s) * select_row_stride(nb) * sizeof(uint32_t);
     case SPARK_CALL_ATTN:
-      return 0;
+      return 256;  // the per-launch counter of the dynamic item queue
     case SPARK_CALL_REBLOCK:
       return reblock_workspace_bytes(s->B * s->H, (int)nb, s->d);
     default:
@@ -380,11 +380,10 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
                    const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,
                    size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   if (empty(s)) return SPARK_OK;
+  if (!ws || ws_bytes < spark_workspace_bytes(s, SPARK_CALL_ATTN) || !aligned16(ws)) return SPARK_EINVAL;
   const int nb = (int)num_blocks(s);
   const int bh = s->B * s->H;
   if (!Q || !K || !V || !O) return SPARK_EINVAL;
@@ -422,7 +421,9 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   tp.pooled = (nb > 0 && pool_pack != nullptr) ? 1 : 0;
   tp.n_items = (int)items;
   tp.scale_log2 = eff_scale(s) * kLog2e;
+  tp.item_ctr = static_cast<int*>(ws);
   cudaStream_t cs = as_stream(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return SPARK_ECUDA;
   const void* pack = tp.pooled ? pool_pack : nullptr;
   if (qt == 2 * kBlock)
     return s->d == 128 ? launch_attn_tc<128, true>(tp, K, V, pack, cs) : launch_attn_tc<64, true>(tp, K, V, pack, cs);

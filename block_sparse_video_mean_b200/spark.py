@@ -218,13 +218,15 @@ def score_select_noalloc(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scal
 
 
 def attn_fwd(Q, K, V, idx, cnt, n_sink, pack=None, beta=None, perm=None, scale=None,
-             out=None, lse=True, q_tile=BLOCK):
+             out=None, lse=True, q_tile=BLOCK, ws=None):
     """spark_attn_fwd: returns (O bf16 [B,H,N,d], LSE fp32 [B,H,N] or None)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, n)
     shape = _shape_of(Q, n_sink, scale, q_tile)
     B, H, N, d = Q.shape
     dev = Q.device
+    if ws is None:
+        ws = torch.empty(max(workspace_bytes(shape, CALL_ATTN), 16), dtype=torch.uint8, device=dev)
     if out is None:
         out = (torch.empty_like(Q),
                torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse else None)
@@ -232,7 +234,7 @@ def attn_fwd(Q, K, V, idx, cnt, n_sink, pack=None, beta=None, perm=None, scale=N
     kcap = idx.shape[-1] if idx is not None else 1
     _check(load().spark_attn_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                                  _ptr(cnt), int(kcap), _ptr(pack), _ptr(beta), _ptr(perm), _ptr(O),
-                                 _ptr(L), None, 0, _stream(dev)), "spark_attn_fwd")
+                                 _ptr(L), _ptr(ws), ws.numel(), _stream(dev)), "spark_attn_fwd")
     return O, L
 
 
@@ -321,6 +323,7 @@ class SparkAttention:
         self.idx = torch.empty((B, H, nt, self.kcap), dtype=torch.int32, device=dev)
         self.cnt = torch.empty((B, H, nt), dtype=torch.int32, device=dev)
         self.sel_ws = torch.empty(max(workspace_bytes(self.shape, CALL_SELECT), 16), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(max(workspace_bytes(self.shape, CALL_ATTN), 16), dtype=torch.uint8, device=dev)
         self.O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, H, N), **f32)
         self.rb = None
@@ -364,6 +367,6 @@ class SparkAttention:
         mark(3)
         attn_fwd(Q, K, V, self.idx, self.cnt, self.n_sink,
                  pack=self.pool["pack"] if cfg.compressed else None, beta=self.pool["beta"],
-                 perm=perm, scale=cfg.scale, out=(self.O, self.lse), q_tile=cfg.q_tile)
+                 perm=perm, scale=cfg.scale, out=(self.O, self.lse), q_tile=cfg.q_tile, ws=self.attn_ws)
         mark(4)
         return self.O, self.lse

@@ -91,7 +91,8 @@ int32_t spark_num_blocks(const spark_shape* s);
  *   SPARK_CALL_SELECT  scratch of spark_score_select: fp64 tau moments (2*B*H doubles,
  *                      padded to 256 bytes) and the score keys of every head
  *                      (B*H*nt*nbp uint32, nbp = nb rounded up to 4);
- *   SPARK_CALL_ATTN    scratch of spark_attn_fwd (0: it needs none);
+ *   SPARK_CALL_ATTN    scratch of spark_attn_fwd: 256 bytes (the launch's counter of
+ *                      work items handed out to the CTAs; zeroed by the call);
  *   SPARK_CALL_REBLOCK scratch of spark_reblock.
  * Returns 0 for an invalid shape or call id. */
 size_t spark_workspace_bytes(const spark_shape* s, int call_id);
@@ -152,7 +153,10 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
  * Outputs: O bf16 [B, H, N, d]; lse fp32 [B, H, N] natural-log (nullable).
  * Block indices outside [0, nb) are skipped and recorded as SPARK_EDEVICE_INDEX.
  * q_tile = 64 runs 64-query tiles on M = 64 tensor-core MMAs, q_tile = 128 runs 128-query
- * tiles (dense rows too) on M = 128 MMAs. */
+ * tiles (dense rows too) on M = 128 MMAs; the 128-query kernel hands the tiles out to the
+ * CTAs at run time (longest first: the dense rows' tiles lead).
+ * ws: spark_workspace_bytes(s, SPARK_CALL_ATTN) bytes, 16-byte aligned, not shared with a
+ * launch in flight on another stream. */
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
                    const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,

@@ -49,7 +49,7 @@ def test_num_blocks_and_workspace(spark):
     assert spark.num_blocks(s) == 2745
     # bf16 k_pool and v_summ, then beta*log2(e) padded to 2752 = 43 x 64 entries per head
     assert spark.workspace_bytes(s, spark.CALL_POOL) == 2 * 24 * 2745 * 128 * 2 + 24 * 2752 * 4
-    assert spark.workspace_bytes(s, spark.CALL_ATTN) == 0
+    assert spark.workspace_bytes(s, spark.CALL_ATTN) == 256   # the item counter
     ragged = spark.make_shape(1, 1, 64 * 3 + 17 + 5, 64, 5)
     assert spark.num_blocks(ragged) == 3
     assert spark.num_blocks(spark.make_shape(1, 1, 40, 64, 8)) == 0
@@ -108,6 +108,11 @@ def test_bad_arguments_are_rejected_on_the_host(spark):
                                   None) == -1
     assert lib.spark_reblock(ctypes.byref(ok), dummy, dummy, dummy, None, dummy, dummy, dummy, None,
                              dummy, 1 << 30, None) == -1
+    # the attention call needs its item-counter workspace
+    assert lib.spark_attn_fwd(ctypes.byref(ok), dummy, dummy, dummy, dummy, dummy, 1, None, None,
+                              None, dummy, None, None, 0, None) == -1
+    assert lib.spark_attn_fwd(ctypes.byref(ok), dummy, dummy, dummy, dummy, dummy, 1, None, None,
+                              None, dummy, None, dummy, 64, None) == -1
 
 
 def test_empty_inputs_are_a_no_op(spark):
