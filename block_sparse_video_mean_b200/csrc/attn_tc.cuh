@@ -175,19 +175,6 @@ __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
   return r;
 }
 
-// Slot s of CTA c walks items 2c + s, 2c + s + 2G, ... and skips items without tiles.
-struct TcSlotWalk {
-  int it, stride, n;
-  __device__ __forceinline__ bool next_nonempty(const TcParams& p, TcItem* I) {
-    while (it < n) {
-      *I = tc_item(p, it);
-      it += stride;
-      if (I->ntiles > 0) return true;
-    }
-    return false;
-  }
-};
-
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -256,8 +243,15 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* ofree = qfull + 4;             // [slot]: the epilogue has read O
   uint64_t* odone = ofree + 2;             // [slot]: last PV of an item completed
   uint64_t* finbar = odone + 2;            // [slot]: all MMAs of that slot's issuer done
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(finbar + 2);
+  TcQueue queue[2];                        // [slot]: items handed out at run time (warp 8 claims)
+  queue[0].full = finbar + 2;
+  queue[0].empty = queue[0].full + kQueueLen;
+  queue[1].full = queue[0].empty + kQueueLen;
+  queue[1].empty = queue[1].full + kQueueLen;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(queue[1].empty + kQueueLen);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  queue[0].ids = const_cast<int*>(abort_flag) + 1;
+  queue[1].ids = queue[0].ids + kQueueLen;
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -281,6 +275,11 @@ __global__ void __launch_bounds__(384, 1)
     }
     tc::mbar_init(&finbar[0], 1);
     tc::mbar_init(&finbar[1], 1);
+    for (int q = 0; q < 2; ++q)
+      for (int i = 0; i < kQueueLen; ++i) {
+        tc::mbar_init(&queue[q].full[i], 1);
+        tc::mbar_init(&queue[q].empty[i], 7);  // V producer, two issuers, the slot's 4 softmax warps
+      }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -298,7 +297,6 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = *tmem_holder;
-  const int stride = 2 * gridDim.x;
   const int nv = p.nb * kBlock;
   const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
 
@@ -317,17 +315,47 @@ __global__ void __launch_bounds__(384, 1)
     unsigned char* rbase = is_v ? vring : ring;
     const CUtensorMap* map_x = is_v ? &maps.v : &maps.k;
     const CUtensorMap* map_p = is_v ? &maps.vp : &maps.kp;
-    // The whole warp walks the tile sequence; the selected block indices are fetched 32
-    // halves at a time, one chunk ahead, so no global load sits on the issue path.
-    TcSlotWalk walk[2] = {{2 * (int)blockIdx.x, stride, p.n_items},
-                          {2 * (int)blockIdx.x + 1, stride, p.n_items}};
+    // The whole warp walks the tile sequence (warp 8 claims each slot's items, warp 10
+    // reads them from the slot's queue); the selected block indices are fetched 32 halves
+    // at a time, one chunk ahead, so no global load sits on the issue path.
+    uint32_t qj[2] = {0, 0};
+    bool ok = true;
+    auto take_nonempty = [&](int s, TcItem* I) -> bool {
+      while (true) {
+        int id;
+        if (!(is_v ? queue[s].read(qj[s], abort_flag, &id, false) : queue[s].claim(qj[s], p, abort_flag, &id))) {
+          ok = false;
+          return false;
+        }
+        ++qj[s];
+        if (id < 0) return false;
+        *I = tc_item(p, id);
+        if (I->ntiles > 0) return true;
+      }
+    };
+    // warp 8 keeps one non-empty item per slot claimed ahead of the one it loads, so that
+    // every reader finds a slot's next item published when it starts an item
+    TcItem ahead_item[2] = {};
+    bool have_ahead[2] = {false, false};
+    auto next_nonempty = [&](int s, TcItem* I) -> bool {
+      if (is_v) return take_nonempty(s, I);
+      bool have_now;
+      if (qj[s] == 0) {
+        have_now = take_nonempty(s, I);
+      } else {
+        have_now = have_ahead[s];
+        *I = ahead_item[s];
+      }
+      have_ahead[s] = have_now && take_nonempty(s, &ahead_item[s]);
+      return have_now && ok;
+    };
     TcItem cur[2];
     bool have[2];
     int t[2] = {0, 0};
     int ic[2] = {0, 0}, in[2] = {0, 0};  // idx of halves 32c + lane (current / next chunk)
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
-      have[s] = walk[s].next_nonempty(p, &cur[s]);
+      have[s] = next_nonempty(s, &cur[s]);
       if (have[s] && !cur[s].dense) {
         const int h0 = lane, h1 = 32 + lane;
         ic[s] = h0 < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + h0] : 0;
@@ -335,7 +363,6 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     uint32_t q = 0;
-    bool ok = true;
     while (ok && (have[0] || have[1])) {
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
@@ -382,7 +409,7 @@ __global__ void __launch_bounds__(384, 1)
             ++q;
             if (++t[s] == cur[s].ntiles) {
               t[s] = 0;
-              have[s] = walk[s].next_nonempty(p, &cur[s]);
+              have[s] = next_nonempty(s, &cur[s]);
               if (have[s] && !cur[s].dense) {
                 const int h0 = lane, h1 = 32 + lane;
                 ic[s] = h0 < cur[s].cnt ? p.idx[cur[s].row * (size_t)p.kcap + h0] : 0;
@@ -413,13 +440,26 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idS = tc::make_idesc_bf16(64, 128, 0, 0);
       constexpr uint32_t idPV = tc::make_idesc_bf16(64, D, 0, 1);
       const uint32_t lanes = (uint32_t)(16 * s) << 16;
-      TcSlotWalk walk[2] = {{2 * (int)blockIdx.x, stride, p.n_items},
-                            {2 * (int)blockIdx.x + 1, stride, p.n_items}};
+      uint32_t qj[2] = {0, 0};
+      bool ok = true;
+      auto next_nonempty = [&](int o, TcItem* I) -> bool {
+        while (true) {
+          int id;
+          if (!queue[o].read(qj[o], abort_flag, &id, true)) {
+            ok = false;
+            return false;
+          }
+          ++qj[o];
+          if (id < 0) return false;
+          *I = tc_item(p, id);
+          if (I->ntiles > 0) return true;
+        }
+      };
       TcItem cur[2];
       bool have[2];
       int t[2] = {0, 0};
 #pragma unroll
-      for (int o = 0; o < 2; ++o) have[o] = walk[o].next_nonempty(p, &cur[o]);
+      for (int o = 0; o < 2; ++o) have[o] = next_nonempty(o, &cur[o]);
       uint32_t g = 0;      // tiles of this slot issued (all items)
       uint32_t nitem = 0;  // non-empty items of this slot started
       bool pend = false;   // PV of the previous tile still to issue
@@ -427,7 +467,6 @@ __global__ void __launch_bounds__(384, 1)
       bool pfirst = false, plast = false;
       const uint32_t ring_addr = tc::smem_addr(ring);
       const uint32_t vring_addr = tc::smem_addr(vring);
-      bool ok = true;
       auto issue_pv = [&]() -> bool {
         const uint32_t b = pg & 1;
         SPARK_TC_T0(t_pw);
@@ -498,7 +537,14 @@ __global__ void __launch_bounds__(384, 1)
               ++q;
               if (++t[o] == cur[o].ntiles) {
                 t[o] = 0;
-                have[o] = walk[o].next_nonempty(p, &cur[o]);
+                have[o] = next_nonempty(o, &cur[o]);
+                // this slot is done: its last PV goes out now, since the V stage it holds is
+                // needed by the other slot's tiles (this issuer keeps reading the other
+                // slot's items only to stay in step with the queue)
+                if (o == s && !have[o] && ok && pend) {
+                  ok = issue_pv();
+                  pend = false;
+                }
               }
             }
           }
@@ -623,12 +669,19 @@ __global__ void __launch_bounds__(384, 1)
       return true;
     };
 
-    // Items of this slot in order; an item with nothing to attend to gets O = 0, LSE = -inf.
-    TcSlotWalk walk = {2 * (int)blockIdx.x + s, stride, p.n_items};
+    // Items of this slot in the queue's order; an item with nothing to attend to gets
+    // O = 0, LSE = -inf.
+    uint32_t qj = 0;
     auto next_item = [&](TcItem* I) -> bool {
-      while (walk.it < walk.n) {
-        *I = tc_item(p, walk.it);
-        walk.it += walk.stride;
+      while (true) {
+        int id;
+        if (!queue[s].read(qj, abort_flag, &id, false)) {
+          ok = false;
+          return false;
+        }
+        ++qj;
+        if (id < 0) return false;
+        *I = tc_item(p, id);
         if (I->ntiles > 0) return true;
         if (r < I->nq) {
           int orow = I->q0 + r;
@@ -646,7 +699,6 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      return false;
     };
 
     uint32_t g = 0;  // tiles processed by this slot (all items)
@@ -656,13 +708,14 @@ __global__ void __launch_bounds__(384, 1)
     bool have_prev = false;
     float m_prev = -INFINITY, l_prev = 0.f;
     bool have = next_item(&I);
-    TcSlotWalk ahead = walk;  // finds the next non-empty item one ahead
     if (have) prepare(I, 0);
     int cur_bad = bad_next;
     bad_next = 0;
     while (ok && have) {
+      // the slot's next item (published before this item's first copies were issued)
       TcItem nxt;
-      const bool have_nxt = ahead.next_nonempty(p, &nxt);
+      const bool have_nxt = next_item(&nxt);
+      if (!ok) break;
       const uint32_t* bm = bm2 + (n & 1) * nbwp;
 
       float m_run = -INFINITY, l_run = 0.f;
@@ -820,7 +873,8 @@ __global__ void __launch_bounds__(384, 1)
       l_prev = l_run;
       cur_bad = bad_next;
       bad_next = 0;
-      have = next_item(&I);
+      I = nxt;
+      have = have_nxt;
       ++n;
     }
     if (ok && have_prev) epilogue(prev, m_prev, l_prev);

@@ -86,19 +86,6 @@ __device__ __forceinline__ TcItem tc128_item(const TcParams& p, int it) {
   return r;
 }
 
-// CTA c walks items c, c + G, c + 2G, ... and skips items without tiles.
-struct Tc128Walk {
-  int it, stride, n;
-  __device__ __forceinline__ bool next_nonempty(const TcParams& p, TcItem* I) {
-    while (it < n) {
-      *I = tc128_item(p, it);
-      it += stride;
-      if (I->ntiles > 0) return true;
-    }
-    return false;
-  }
-};
-
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     attn_tc128_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
@@ -203,7 +190,7 @@ __global__ void __launch_bounds__(384, 1)
     };
     // warp 8 keeps one non-empty item claimed ahead of the one it loads, so that every
     // reader of the queue finds the next item already published when it starts an item
-    TcItem ahead_item;
+    TcItem ahead_item = {};
     bool have_ahead = false;
     auto next_nonempty = [&](TcItem* I) -> bool {
       if (is_v) return take_nonempty(I);
