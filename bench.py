@@ -119,7 +119,7 @@ def load_peaks():
 # dram__bytes_write.sum of a 2-head capture of the same shape, scaled by 12 to 24 heads
 # (profiles/attn_tc_1152x640x243_h2_full.md, profiles/attn_tc128_1152x640x243_h2_full.md).
 # A workload without a capture of its current kernel reports None.
-ATTN_TRAFFIC_BYTES = {"1152x640x243": 57.2e9, "1152x640x243-q128": 31.3e9}
+ATTN_TRAFFIC_BYTES = {"1152x640x243": 37.6e9, "1152x640x243-q128": 25.5e9}
 
 
 class ClockSampler:
