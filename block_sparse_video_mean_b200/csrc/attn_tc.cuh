@@ -115,9 +115,9 @@ template <int D>
 struct TcCfg {
   // A tile is 128 keys: two 64-key halves (each a selected block, 64 dense rows or 64
   // pooled entries), so S = Q K^T is one N = 128 MMA per K step.
-  // Two 32 KB stages per ring: deeper rings measured slower (shared memory and L1 share
-  // the SM's 256 KB, and the softmax warps' loads and spills live in L1).
-  static constexpr int kStages = D == 128 ? 2 : 4;
+  // Three 32 KB stages per ring (202 KB of shared memory with the bitmaps): each K/V tile
+  // takes about 1.7 us from L2 under load, so the copies in flight set the delivery rate.
+  static constexpr int kStages = D == 128 ? 3 : 4;
   static constexpr int kPanels = D / 64;           // 128-byte swizzle panels per row
   static constexpr int kHalfBytes = 64 * 128;      // 64 rows x 128 B (one TMA box)
   static constexpr int kPanelBytes = 128 * 128;    // 128 rows x 128 B
