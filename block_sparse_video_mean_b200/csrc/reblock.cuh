@@ -405,15 +405,36 @@ __device__ __forceinline__ double rcp_nr(double x) {
   return r;
 }
 
+// Eigenvalues of the tridiagonal (a, e) below x, counted as sign changes of the Sturm
+// sequence p_0 = 1, p_1 = a_0 - x, p_{i+1} = (a_i - x) p_i - e_{i-1}^2 p_{i-1}. The ratio
+// p_{i+1} / p_i is pivot i of the LDL^T factorisation of T - xI, so this counts negative
+// pivots without a division: one FMA per step on the dependency chain. A pivot below pivmin
+// in magnitude becomes -pivmin, as in the division form; signs are read from the sign bits
+// (a term scaled down to zero keeps its sign). Every 4 steps the pair (p_i, p_{i-1}) is
+// multiplied by the exact power of two that brings the larger to [1, 2); the entries are a
+// covariance of whitened rows, O(1), so 4 steps can neither overflow nor lose the pair.
 __device__ __forceinline__ int sturm_count(const double* a, const double* e2, int n, double x,
                                            double pivmin) {
-  int c = 0;
-  double q = a[0] - x;
-  if (q < 0.0) ++c;
+  constexpr double kTrueMin = 4.9406564584124654e-324;
+  double pm = 1.0;      // p_{i-1}
+  double p = a[0] - x;  // p_i
+  if (fabs(p) < pivmin) p = -pivmin;
+  int c = signbit(p) ? 1 : 0;
   for (int i = 1; i < n; ++i) {
-    const double den = fabs(q) < pivmin ? -pivmin : q;
-    q = (a[i] - x) - e2[i - 1] * rcp_nr(den);
-    if (q < 0.0) ++c;
+    const double lim = fmax(pivmin * fabs(p), kTrueMin);
+    double pn = fma(a[i] - x, p, -e2[i - 1] * pm);
+    if (fabs(pn) < lim) pn = signbit(p) ? lim : -lim;
+    c += (signbit(pn) != signbit(p)) ? 1 : 0;
+    pm = p;
+    p = pn;
+    if ((i & 3) == 0) {
+      const double m = fmax(fabs(p), fabs(pm));
+      int ex = (int)((__double2hiint(m) >> 20) & 0x7ff) - 1023;
+      ex = min(max(ex, -1022), 1022);
+      const double s = __hiloint2double((1023 - ex) << 20, 0);  // 2^-ex
+      p *= s;
+      pm *= s;
+    }
   }
   return c;
 }
