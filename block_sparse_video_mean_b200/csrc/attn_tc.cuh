@@ -147,24 +147,28 @@ struct TcItem {
   size_t row;                                  // selection row (video items)
 };
 
+// Item `it`, head-major: each head's dense items (64 dense query rows each, the longest
+// items) and then its video query blocks (nb), so that the CTAs at work at any moment share
+// one or two heads' K/V in L2.
 __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
   TcItem r;
-  const int nd = p.BH * p.n_dq;
   const int nv = p.nb * kBlock;
   const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
-  if (it < nd) {
-    r.bh = it / p.n_dq;
+  const int per_h = p.n_dq + p.nb;
+  const int hb = it / per_h, jj = it - hb * per_h;
+  if (jj < p.n_dq) {
+    r.bh = hb;
     r.dense = 1;
-    r.q0 = nv + (it % p.n_dq) * kBlock;
+    r.q0 = nv + jj * kBlock;
     r.cnt = 0;
     r.row = 0;
     r.nhalf = (p.N + kBlock - 1) / kBlock;
   } else {
-    const int v = it - nd;
-    r.bh = v / p.nb;
+    const int v = jj - p.n_dq;
+    r.bh = hb;
     r.dense = 0;
-    r.q0 = (v % p.nb) * kBlock;
-    r.row = (size_t)r.bh * p.nb + (v % p.nb);
+    r.q0 = v * kBlock;
+    r.row = (size_t)r.bh * p.nb + v;
     int c = p.cnt[r.row];
     c = c < 0 ? 0 : (c > p.kcap ? p.kcap : c);
     r.cnt = c;

@@ -55,27 +55,29 @@ __host__ __device__ inline size_t tc128_smem_bytes(int nb) {
          (size_t)8 * 2 * tc_bitmap_words(nb) * 4;  // two bitmaps per softmax warp
 }
 
-// Item `it`: dense items first (128 dense query rows of one head each), then the video
-// query tiles (nt per head).
+// Item `it`, head-major: each head's dense items (128 dense query rows each, the longest
+// items) and then its video query tiles (nt), so that the CTAs at work at any moment share
+// one or two heads' K/V in L2.
 __device__ __forceinline__ TcItem tc128_item(const TcParams& p, int it) {
   TcItem r;
-  const int nd = p.BH * p.n_dq;
   const int nv = p.nb * kBlock;
   const int n_dk = (p.N - nv + kBlock - 1) / kBlock;
-  if (it < nd) {
-    r.bh = it / p.n_dq;
+  const int per_h = p.n_dq + p.nt;
+  const int hb = it / per_h, jj = it - hb * per_h;
+  if (jj < p.n_dq) {
+    r.bh = hb;
     r.dense = 1;
-    r.q0 = nv + (it % p.n_dq) * 128;
+    r.q0 = nv + jj * 128;
     r.cnt = 0;
     r.row = 0;
     r.nhalf = (p.N + kBlock - 1) / kBlock;
     r.nq = min(128, p.N - r.q0);
   } else {
-    const int v = it - nd;
-    r.bh = v / p.nt;
+    const int v = jj - p.n_dq;
+    r.bh = hb;
     r.dense = 0;
-    r.q0 = (v % p.nt) * 128;
-    r.row = (size_t)r.bh * p.nt + (v % p.nt);
+    r.q0 = v * 128;
+    r.row = (size_t)r.bh * p.nt + v;
     int c = p.cnt[r.row];
     c = c < 0 ? 0 : (c > p.kcap ? p.kcap : c);
     r.cnt = c;

@@ -501,3 +501,4 @@ const char* spark_strerror(int status) {
 }
 
 }  // extern "C"
+#include "host_fwd.cuh"

@@ -29,7 +29,7 @@ BLOCK = 64
 EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
            "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
            "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches", "spark_reblock_kv",
-           "spark_num_query_tiles")
+           "spark_num_query_tiles", "spark_forward_host", "spark_forward_host_workspace_bytes")
 NOALLOC_MAX_HEADS = 4096
 
 
@@ -43,6 +43,13 @@ class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("n_sink", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("scale", ctypes.c_float), ("q_tile", ctypes.c_int32)]
+
+
+class FwdConfig(ctypes.Structure):
+    _fields_ = [("param", ctypes.c_double), ("select_mode", ctypes.c_int32),
+                ("kcap", ctypes.c_int32), ("pool_mode", ctypes.c_int32),
+                ("compressed", ctypes.c_int32), ("reblock", ctypes.c_int32),
+                ("heads_per_group", ctypes.c_int32)]
 
 
 _lib = None
@@ -79,6 +86,11 @@ def load() -> ctypes.CDLL:
     lib.spark_reblock.restype = I
     lib.spark_reblock_kv.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
     lib.spark_reblock_kv.restype = I
+    FP = ctypes.POINTER(FwdConfig)
+    lib.spark_forward_host_workspace_bytes.argtypes = [SP, FP]
+    lib.spark_forward_host_workspace_bytes.restype = Z
+    lib.spark_forward_host.argtypes = [SP, FP, P, P, P, P, P, P, Z, P]
+    lib.spark_forward_host.restype = I
     lib.spark_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), P]
     lib.spark_device_error.restype = I
     lib.spark_strerror.argtypes = [I]
@@ -282,6 +294,38 @@ def reblock_kv(Q, K, V, n_sink, out=None, ws=None):
     return out
 
 
+def fwd_config(mode=SELECT_TOPK_RATIO, param=0.1, kcap=0, pool_mode=POOL_REWEIGHT, compressed=True,
+               reblock=0, heads_per_group=0) -> FwdConfig:
+    """spark_fwd_config of spark_forward_host (reblock: 0 none, 1 shared, 2 own key partition)."""
+    return FwdConfig(float(param), int(mode), int(kcap or 0), int(pool_mode), int(bool(compressed)),
+                     int(reblock), int(heads_per_group or 0))
+
+
+def forward_host_workspace_bytes(shape: Shape, cfg: FwdConfig) -> int:
+    return int(load().spark_forward_host_workspace_bytes(ctypes.byref(shape), ctypes.byref(cfg)))
+
+
+def forward_host(hQ, hK, hV, shape: Shape, cfg: FwdConfig, hO=None, hlse=None, ws=None, device=None):
+    """The whole forward from host tensors (bf16 [B, H, N, d], pinned for the copies to
+    overlap the compute) into host ``hO`` (and ``hlse``), pipelined over groups of heads by
+    spark_forward_host. Asynchronous on the current stream of ``device``; synchronise it
+    before reading ``hO``."""
+    lib = load()
+    dev = torch.device(device if device is not None else "cuda")
+    for t, name in ((hQ, "Q"), (hK, "K"), (hV, "V")):
+        if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    if hO is None:
+        hO = torch.empty(hQ.shape, dtype=torch.bfloat16).pin_memory()
+    need = forward_host_workspace_bytes(shape, cfg)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.spark_forward_host(ctypes.byref(shape), ctypes.byref(cfg), _ptr(hQ), _ptr(hK), _ptr(hV),
+                                  _ptr(hO), _ptr(hlse), _ptr(ws), ws.numel(), _stream(dev)),
+           "spark_forward_host")
+    return hO, hlse
+
+
 # --------------------------------------------------------------------------- whole forward
 
 @dataclass
@@ -370,3 +414,19 @@ class SparkAttention:
                  perm=perm, scale=cfg.scale, out=(self.O, self.lse), q_tile=cfg.q_tile, ws=self.attn_ws)
         mark(4)
         return self.O, self.lse
+
+    def host_config(self, heads_per_group=0) -> FwdConfig:
+        cfg = self.cfg
+        rb = 0 if not cfg.reblock else (2 if cfg.reblock_kv else 1)
+        return fwd_config(self.mode, cfg.param, self.kcap, self.pool_mode, cfg.compressed, rb,
+                          heads_per_group)
+
+    def run_host(self, hQ, hK, hV, hO=None, hlse=None, heads_per_group=0):
+        """One forward from host tensors into host ``hO`` (and ``hlse``): the copies of
+        each group of heads overlap the compute of its neighbours (spark_forward_host).
+        The device workspace is allocated on the first call and kept."""
+        hcfg = self.host_config(heads_per_group)
+        need = forward_host_workspace_bytes(self.shape, hcfg)
+        if getattr(self, "host_ws", None) is None or self.host_ws.numel() < need:
+            self.host_ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.O.device)
+        return forward_host(hQ, hK, hV, self.shape, hcfg, hO, hlse, self.host_ws, self.O.device)

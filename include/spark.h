@@ -20,9 +20,9 @@
  *   to every key and their keys are attended by every query. Dense rows are never
  *   pooled, scored, compressed or reblocked.
  * - block must be 64; d must be 64 or 128; scale <= 0 means 1/sqrt(d).
- * - Every pointer is a device pointer owned by the caller; the library allocates
- *   nothing, keeps no state beyond one device-side error word (and the fixed scratch
- *   array of spark_score_select_noalloc), and never
+ * - Every pointer is a device pointer owned by the caller (spark_forward_host also takes
+ *   host buffers); the library allocates no memory, keeps no state beyond one device-side
+ *   error word (and the fixed scratch array of spark_score_select_noalloc), and never
  *   synchronises except in spark_device_error. Calls are asynchronous on `stream`
  *   (a cudaStream_t, NULL = legacy default stream) and re-entrant.
  * - Return value: SPARK_OK, or a negative status for arguments rejected on the host
@@ -154,7 +154,7 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
  * Block indices outside [0, nb) are skipped and recorded as SPARK_EDEVICE_INDEX.
  * q_tile = 64 runs 64-query tiles on M = 64 tensor-core MMAs, q_tile = 128 runs 128-query
  * tiles (dense rows too) on M = 128 MMAs; the 128-query kernel hands the tiles out to the
- * CTAs at run time (longest first: the dense rows' tiles lead).
+ * CTAs at run time, head by head (each head's dense-row tiles, the longest, lead its tiles).
  * ws: spark_workspace_bytes(s, SPARK_CALL_ATTN) bytes, 16-byte aligned, not shared with a
  * launch in flight on another stream. */
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
@@ -190,6 +190,49 @@ int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
 int spark_reblock_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                      int32_t* perm_q, int32_t* perm_k, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* The whole forward from host memory, pipelined over groups of heads (the pages have no
+ * counterpart; a library convenience for callers whose Q/K/V start in host memory). Every
+ * step of the method is per (b, h), so the flattened B*H heads are cut into groups of
+ * heads_per_group (the last group may be smaller) and each group runs as a forward of its
+ * own shape [1, G, N, d]: its Q/K/V are copied host-to-device on one internal stream, the
+ * group is computed on `stream` (optional Reblock, spark_pool_kv, spark_score_select,
+ * spark_attn_fwd), and its O (and lse) are copied device-to-host on a second internal
+ * stream, so that the copies of neighbouring groups overlap the compute. Two staging slots
+ * alternate between groups.
+ * - hQ, hK, hV: host bf16 [B, H, N, d]; hO: host bf16 [B, H, N, d]; hlse: host fp32
+ *   [B, H, N] or NULL. Page-locked (pinned) host memory is needed for the copies to
+ *   overlap; pageable memory works but the copies then serialise with the compute.
+ *   Outputs are those of the device calls with the same configuration.
+ * - cfg: select_mode / param / kcap as in spark_score_select (kcap <= 0 picks k for top-k
+ *   and nb for tau); pool_mode as in spark_pool_kv; compressed != 0 turns the compressed
+ *   branch on; reblock 0 = none, 1 = spark_reblock (keys reuse the query partition),
+ *   2 = spark_reblock_kv; heads_per_group <= 0 picks ceil(B*H / 8).
+ * - ws: device buffer of spark_forward_host_workspace_bytes(s, cfg) bytes, 256-byte
+ *   aligned, holding both staging slots and every intermediate of one group.
+ * - Asynchronous: returns once everything is enqueued; `stream` waits for the last copy
+ *   back, so synchronising `stream` means hO / hlse are complete. The host buffers must
+ *   stay valid and unchanged until then. Unlike the other calls this one creates two
+ *   streams and seven events per call (released by the driver once their work completes).
+ * - Returns SPARK_EINVAL / SPARK_EUNSUPPORTED for rejected arguments (nothing enqueued),
+ *   SPARK_ECUDA if a copy or launch fails to enqueue, or the first error status of a
+ *   per-group call (groups before it are enqueued). */
+typedef struct spark_fwd_config {
+  double param;            /* top-k ratio in (0, 1] or tau */
+  int32_t select_mode;     /* SPARK_SELECT_TOPK_RATIO or SPARK_SELECT_TAU */
+  int32_t kcap;            /* selection slots per row; <= 0: k (top-k) or nb (tau) */
+  int32_t pool_mode;       /* SPARK_POOL_REWEIGHT or SPARK_POOL_MEAN */
+  int32_t compressed;      /* compressed branch on (!= 0) or off */
+  int32_t reblock;         /* 0 none, 1 spark_reblock, 2 spark_reblock_kv */
+  int32_t heads_per_group; /* heads per pipeline group; <= 0: ceil(B*H / 8) */
+} spark_fwd_config;
+
+/* Device workspace bytes of spark_forward_host; 0 for an invalid shape or config. */
+size_t spark_forward_host_workspace_bytes(const spark_shape* s, const spark_fwd_config* cfg);
+
+int spark_forward_host(const spark_shape* s, const spark_fwd_config* cfg, const uint16_t* hQ,
+                       const uint16_t* hK, const uint16_t* hV, uint16_t* hO, float* hlse,
+                       void* ws, size_t ws_bytes, void* stream);
 
 /* spark_score_select without a scratch argument, for callers that cannot allocate device
  * memory of their own (the paper has no counterpart; this is a library convenience).

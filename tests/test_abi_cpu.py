@@ -128,3 +128,56 @@ def test_empty_inputs_are_a_no_op(spark):
 def test_strerror(spark):
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert spark.strerror(code) and spark.strerror(code) != "unknown status"
+
+
+def test_host_forward_config_and_workspace(spark):
+    assert ctypes.sizeof(spark.FwdConfig) == 32
+    s = spark.make_shape(2, 3, 64 * 10 + 7 + 16, 64, 16)
+    nb, N, d = 10, 64 * 10 + 7 + 16, 64
+    cfg = spark.fwd_config(heads_per_group=2)
+    ws = spark.forward_host_workspace_bytes(s, cfg)
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    G = 2
+    g = spark.make_shape(1, G, N, d, 16)
+    slots = 2 * (4 * up(G * N * d * 2) + up(G * N * 4))
+    k = spark.topk_count(0.1, nb)
+    inter = (up(G * nb * d * 4) + 2 * up(G * nb * d * 4) + up(G * nb * 4) + up(G * d * 4)
+             + up(spark.workspace_bytes(g, spark.CALL_POOL)) + up(G * nb * k * 4) + up(G * nb * 4)
+             + up(spark.workspace_bytes(g, spark.CALL_SELECT)) + up(256))
+    assert ws == slots + inter
+    # reblock adds the permutation, the permuted copies and its own scratch
+    rb = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=2, reblock=1))
+    assert rb == ws + up(G * nb * 64 * 4) + 3 * up(G * N * d * 2) + up(spark.workspace_bytes(g, spark.CALL_REBLOCK))
+    # the automatic group is ceil(B*H / 8) heads; one group never exceeds B*H
+    auto = spark.forward_host_workspace_bytes(s, spark.fwd_config())
+    one = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=1))
+    assert auto == one
+    big = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=100))
+    assert big == spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=6))
+    # invalid configurations size to 0
+    for bad in (spark.fwd_config(mode=7), spark.fwd_config(pool_mode=3), spark.fwd_config(reblock=3),
+                spark.fwd_config(param=0.0), spark.fwd_config(param=float("nan"))):
+        assert spark.forward_host_workspace_bytes(s, bad) == 0
+
+
+def test_host_forward_rejects_bad_arguments_before_any_cuda_call(spark):
+    lib = spark.load()
+    s = spark.make_shape(1, 2, 64 * 4 + 8, 64, 8)
+    cfg = spark.fwd_config()
+    need = spark.forward_host_workspace_bytes(s, cfg)
+    host = (ctypes.c_uint16 * 16)()
+    h = ctypes.cast(host, ctypes.c_void_p)
+    ws = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
+    assert lib.spark_forward_host(ctypes.byref(s), ctypes.byref(cfg), None, h, h, h, None, ws, need, None) == -1
+    assert lib.spark_forward_host(ctypes.byref(s), ctypes.byref(cfg), h, h, h, h, None, None, need, None) == -1
+    assert lib.spark_forward_host(ctypes.byref(s), ctypes.byref(cfg), h, h, h, h, None, ws, need - 1, None) == -1
+    assert lib.spark_forward_host(ctypes.byref(s), ctypes.byref(cfg), h, h, h, h, None,
+                                  ctypes.c_void_p(4096 + 16), need, None) == -1   # not 256-aligned
+    assert lib.spark_forward_host(ctypes.byref(s), None, h, h, h, h, None, ws, need, None) == -1
+    bad_d = spark.make_shape(1, 2, 64 * 4 + 8, 96, 8)
+    assert lib.spark_forward_host(ctypes.byref(bad_d), ctypes.byref(cfg), h, h, h, h, None, ws, need, None) == -2
+    empty = spark.make_shape(0, 2, 64, 64, 0)
+    assert lib.spark_forward_host(ctypes.byref(empty), ctypes.byref(cfg), None, None, None, None, None,
+                                  None, 0, None) == 0
