@@ -352,8 +352,8 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
         "e2e": {"value": round(world * fl["dense_equiv"] / (e2e_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s dense-equivalent, host buffers, copies inside the timed region",
                 "ms_per_step": round(e2e_ms, 3),
-                "api": "SparkAttention.run_host (spark_forward_host: heads in groups of "
-                       f"{-(-plan.shape.B * plan.shape.H // 8)}, copies overlapping compute)",
+                "api": "SparkAttention.run_host (spark_forward_host: automatic head groups, "
+                       "copies overlapping compute)",
                 "h2d_bytes_per_step": 3 * Q.numel() * Q.element_size(),
                 "d2h_bytes_per_step": plan.O.numel() * plan.O.element_size()},
         "gpu_launches": launches,

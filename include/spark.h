@@ -207,7 +207,8 @@ int spark_reblock_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K,
  * - cfg: select_mode / param / kcap as in spark_score_select (kcap <= 0 picks k for top-k
  *   and nb for tau); pool_mode as in spark_pool_kv; compressed != 0 turns the compressed
  *   branch on; reblock 0 = none, 1 = spark_reblock (keys reuse the query partition),
- *   2 = spark_reblock_kv; heads_per_group <= 0 picks ceil(B*H / 8).
+ *   2 = spark_reblock_kv; heads_per_group <= 0 picks the fewest heads whose Q/K/V reach
+ *   32 MiB (ceil(2^25 / (6*N*d)), at most B*H): one head at a time for video-sized heads.
  * - ws: device buffer of spark_forward_host_workspace_bytes(s, cfg) bytes, 256-byte
  *   aligned, holding both staging slots and every intermediate of one group.
  * - Asynchronous: returns once everything is enqueued; `stream` waits for the last copy
@@ -224,7 +225,7 @@ typedef struct spark_fwd_config {
   int32_t pool_mode;       /* SPARK_POOL_REWEIGHT or SPARK_POOL_MEAN */
   int32_t compressed;      /* compressed branch on (!= 0) or off */
   int32_t reblock;         /* 0 none, 1 spark_reblock, 2 spark_reblock_kv */
-  int32_t heads_per_group; /* heads per pipeline group; <= 0: ceil(B*H / 8) */
+  int32_t heads_per_group; /* heads per pipeline group; <= 0: automatic (see above) */
 } spark_fwd_config;
 
 /* Device workspace bytes of spark_forward_host; 0 for an invalid shape or config. */

@@ -150,10 +150,16 @@ def test_host_forward_config_and_workspace(spark):
     # reblock adds the permutation, the permuted copies and its own scratch
     rb = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=2, reblock=1))
     assert rb == ws + up(G * nb * 64 * 4) + 3 * up(G * N * d * 2) + up(spark.workspace_bytes(g, spark.CALL_REBLOCK))
-    # the automatic group is ceil(B*H / 8) heads; one group never exceeds B*H
+    # automatic groups hold at least 32 MiB of Q/K/V (capped at B*H): all 6 small heads here,
+    # one head at a time at video size; one group never exceeds B*H
     auto = spark.forward_host_workspace_bytes(s, spark.fwd_config())
-    one = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=1))
-    assert auto == one
+    assert auto == spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=6))
+    video = spark.make_shape(1, 24, 175680 + 512, 128, 512)
+    assert (spark.forward_host_workspace_bytes(video, spark.fwd_config())
+            == spark.forward_host_workspace_bytes(video, spark.fwd_config(heads_per_group=1)))
+    mid = spark.make_shape(1, 24, 4096, 64, 0)   # 1.5 MiB of Q/K/V per head: 22 heads
+    assert (spark.forward_host_workspace_bytes(mid, spark.fwd_config())
+            == spark.forward_host_workspace_bytes(mid, spark.fwd_config(heads_per_group=22)))
     big = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=100))
     assert big == spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=6))
     # invalid configurations size to 0

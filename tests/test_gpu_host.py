@@ -36,7 +36,7 @@ def device_and_host(spark, Q, K, V, ns, cfg, heads_per_group):
 
 CASES = [
     # B, H, d, n_video, n_sink, mode, param, compressed, q_tile, heads_per_group
-    (2, 3, 64, 64 * 20 + 9, 16, "topk", 0.1, True, 64, 0),     # auto: ceil(6 / 8) = 1 head
+    (2, 3, 64, 64 * 20 + 9, 16, "topk", 0.1, True, 64, 0),     # auto: the 6 small heads in one group
     (2, 3, 128, 64 * 17, 40, "tau", 1.0, True, 64, 4),          # a ragged last group of 2
     (1, 5, 128, 64 * 33 + 17, 64, "topk", 0.2, True, 128, 2),   # 128-query route
     (1, 4, 64, 64 * 12, 0, "topk", 0.3, False, 64, 3),          # no sinks, no compression
