@@ -115,11 +115,11 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-# DRAM bytes (read + write) of one attention launch: the dram__bytes_read.sum +
-# dram__bytes_write.sum of a 2-head capture of the same shape, scaled by 12 to 24 heads
-# (profiles/attn_tc_1152x640x243_h2_full.md, profiles/attn_tc128_1152x640x243_h2_full.md).
+# DRAM bytes (read + write) of one attention launch: dram__bytes_read.sum +
+# dram__bytes_write.sum from one full-size (24-head) capture of the current kernels
+# (profiles/attn_tc_1152x640x243_launches.md, profiles/attn_tc128_1152x640x243_launches.md).
 # A workload without a capture of its current kernel reports None.
-ATTN_TRAFFIC_BYTES = {"1152x640x243": 37.6e9, "1152x640x243-q128": 25.5e9}
+ATTN_TRAFFIC_BYTES = {"1152x640x243": 106.27e9, "1152x640x243-q128": 30.10e9}
 
 
 class ClockSampler:
