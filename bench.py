@@ -201,6 +201,18 @@ def phase_bytes(w: Workload, h: int, nb: int, nt: int, kept_blocks: int, kcap: i
 
 # --------------------------------------------------------------------------- GPU arm
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of ``x`` over all ranks of the default process group: every rank must
+    call it at the same point (world 1 returns ``x`` without a collective)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_gpu(args, w: Workload, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -258,10 +270,7 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     ms = t0.elapsed_time(t1)
     phase_ms = {name: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev)
                 for i, name in enumerate(("reblock", "pool", "select", "attn"))}
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
 
     # end to end from pinned host buffers through the public host call: each group of heads
@@ -285,12 +294,7 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_ms /= e2e_steps
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
 
     if rank != 0:
         return None
