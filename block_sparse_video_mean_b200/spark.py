@@ -320,9 +320,11 @@ def forward_host(hQ, hK, hV, shape: Shape, cfg: FwdConfig, hO=None, hlse=None, w
     need = forward_host_workspace_bytes(shape, cfg)
     if ws is None:
         ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    _check(lib.spark_forward_host(ctypes.byref(shape), ctypes.byref(cfg), _ptr(hQ), _ptr(hK), _ptr(hV),
-                                  _ptr(hO), _ptr(hlse), _ptr(ws), ws.numel(), _stream(dev)),
-           "spark_forward_host")
+    with torch.cuda.device(ws.device):   # the library's internal streams go on this device
+        _check(lib.spark_forward_host(ctypes.byref(shape), ctypes.byref(cfg), _ptr(hQ), _ptr(hK),
+                                      _ptr(hV), _ptr(hO), _ptr(hlse), _ptr(ws), ws.numel(),
+                                      _stream(ws.device)),
+               "spark_forward_host")
     return hO, hlse
 
 

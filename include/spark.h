@@ -210,7 +210,9 @@ int spark_reblock_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K,
  *   2 = spark_reblock_kv; heads_per_group <= 0 picks the fewest heads whose Q/K/V reach
  *   32 MiB (ceil(2^25 / (6*N*d)), at most B*H): one head at a time for video-sized heads.
  * - ws: device buffer of spark_forward_host_workspace_bytes(s, cfg) bytes, 256-byte
- *   aligned, holding both staging slots and every intermediate of one group.
+ *   aligned, holding both staging slots and every intermediate of one group. The current
+ *   device must be the one that holds ws and `stream` (the internal streams are created
+ *   there).
  * - Asynchronous: returns once everything is enqueued; `stream` waits for the last copy
  *   back, so synchronising `stream` means hO / hlse are complete. The host buffers must
  *   stay valid and unchanged until then. Unlike the other calls this one creates two
