@@ -13,6 +13,7 @@
 // writes the kept indices in ascending order with ballots (ties: lower index first).
 #pragma once
 #include "spark_common.cuh"
+#include "tc_util.cuh"
 
 namespace spark {
 
@@ -285,11 +286,13 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
   const int i0 = blockIdx.y * kScI, j0 = blockIdx.x * kScJ;
   const float* qp = q_pool + bh * (size_t)nq * D;
   const float* kp = k_pool + bh * (size_t)nb * D;
-  float acc0[4][8], acc1[4][8];
+  // accumulators in column pairs for the packed fp32 FMA (fma.rn.f32x2): each lane runs
+  // exactly the fmaf chain of its own score
+  float2 acc0[4][4], acc1[4][4];
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc0[r][u] = acc1[r][u] = 0.f;
+    for (int u = 0; u < 4; ++u) acc0[r][u] = acc1[r][u] = make_float2(0.f, 0.f);
   for (int d0 = 0; d0 < D; d0 += kScDC) {
     __syncthreads();
     // stage q rows i0.. (64 x 32) and k rows j0.. (128 x 32), transposed to [d][row]
@@ -321,14 +324,16 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
       const float4 kb0 = *reinterpret_cast<const float4*>(&ks[c + 1][4 * tx]);
       const float4 kb1 = *reinterpret_cast<const float4*>(&ks[c + 1][64 + 4 * tx]);
       const float q0[4] = {qa.x, qa.y, qa.z, qa.w}, q1[4] = {qb.x, qb.y, qb.z, qb.w};
-      const float k0[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
-      const float k1[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+      const float2 k0[4] = {make_float2(ka0.x, ka0.y), make_float2(ka0.z, ka0.w),
+                            make_float2(ka1.x, ka1.y), make_float2(ka1.z, ka1.w)};
+      const float2 k1[4] = {make_float2(kb0.x, kb0.y), make_float2(kb0.z, kb0.w),
+                            make_float2(kb1.x, kb1.y), make_float2(kb1.z, kb1.w)};
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          acc0[r][u] = fmaf(q0[r], k0[u], acc0[r][u]);
-          acc1[r][u] = fmaf(q1[r], k1[u], acc1[r][u]);
+        for (int u = 0; u < 4; ++u) {
+          acc0[r][u] = tc::ffma2(make_float2(q0[r], q0[r]), k0[u], acc0[r][u]);
+          acc1[r][u] = tc::ffma2(make_float2(q1[r], q1[r]), k1[u], acc1[r][u]);
         }
     }
   }
@@ -342,7 +347,10 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
       const int j = j0 + 64 * half + 4 * tx;
       uint32_t kv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) kv[e] = float_to_key((acc0[r][4 * half + e] + acc1[r][4 * half + e]) * scale);
+      for (int e = 0; e < 4; ++e) {
+        const float2 a0 = acc0[r][2 * half + (e >> 1)], a1 = acc1[r][2 * half + (e >> 1)];
+        kv[e] = float_to_key(((e & 1) ? a0.y + a1.y : a0.x + a1.x) * scale);
+      }
       if (j + 3 < nbp) {
         *reinterpret_cast<uint4*>(dst + j) = make_uint4(kv[0], kv[1], kv[2], kv[3]);
       } else {
