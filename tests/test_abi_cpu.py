@@ -187,3 +187,15 @@ def test_host_forward_rejects_bad_arguments_before_any_cuda_call(spark):
     empty = spark.make_shape(0, 2, 64, 64, 0)
     assert lib.spark_forward_host(ctypes.byref(empty), ctypes.byref(cfg), None, None, None, None, None,
                                   None, 0, None) == 0
+
+
+def test_host_forward_binding_rejects_bad_host_tensors(spark):
+    import torch
+    s = spark.make_shape(1, 2, 64 * 4 + 8, 64, 8)
+    cfg = spark.fwd_config()
+    good = torch.zeros((1, 2, 64 * 4 + 8, 64), dtype=torch.bfloat16)
+    for bad in (good.float(), good.transpose(2, 3), good[:, :, ::2]):
+        with pytest.raises(ValueError):
+            spark.forward_host(bad, good, good, s, cfg)
+    with pytest.raises(ValueError):
+        spark.forward_host(good, good, good.float(), s, cfg)
