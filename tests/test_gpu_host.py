@@ -89,3 +89,25 @@ def test_host_forward_twice_on_one_workspace(spark):
     torch.cuda.synchronize()
     assert torch.equal(outs[0].view(torch.int16), O1.view(torch.int16))
     assert torch.equal(outs[1].view(torch.int16), O2.view(torch.int16))
+
+
+@pytest.mark.parametrize("q_tile", [64, 128])
+def test_host_forward_full_size_equals_device_forward(spark, q_tile):
+    # the configuration the benchmark's end-to-end leg times: 1152x640x243, 24 heads,
+    # top-k 10% with the compressed branch, automatic groups (one head at a time)
+    from tests.test_gpu_parity import full_inputs
+    (Q, K, V), ns = full_inputs("1152x640x243")
+    B, H, N, d = Q.shape
+    cfg = spark.ForwardConfig("topk", 0.1, True, q_tile=q_tile)
+    plan = spark.SparkAttention(B, H, N, d, ns, cfg, DEV)
+    O, L = plan.run(Q, K, V)
+    O, L = O.cpu(), L.cpu()
+    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+    del Q, K, V
+    hO = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
+    hL = torch.empty(L.shape, dtype=torch.float32).pin_memory()
+    plan.run_host(hQ, hK, hV, hO, hL)
+    torch.cuda.synchronize()
+    assert spark.device_error() == 0
+    assert torch.equal(hO.view(torch.int16), O.view(torch.int16))
+    assert torch.equal(hL, L)
