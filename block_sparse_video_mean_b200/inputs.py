@@ -16,6 +16,13 @@ The block-shared component makes mean-pooled block scores informative, the way
 neighbouring video tokens are correlated in a video-diffusion transformer; with
 ``amp = 0.5`` it carries 20% of the per-element variance.
 
+``q_offset > 0`` adds one more draw per head, after the six above (so the other tensors
+are unchanged): an offset vector ``o ~ N(0, 1)^d`` added to every query row as
+``q_offset * o``. Real attention heads have a strong mean query direction; without it
+the mean query (the compressed branch's anchor) is short and every anchor score of a
+block is nearly equal. With ``q_offset = 1`` at d = 128 the anchor scores of a block
+spread by about one unit, so the block's log-mass bias departs from log 64 by O(1).
+
 On ``device="cpu"`` the draw uses torch's CPU generator; on a CUDA device it uses
 torch's CUDA generator (a different stream of numbers). Either way, whichever side
 compares against the oracle copies the very same tensors to the host.
@@ -40,7 +47,8 @@ def _groups(n_video: int, n_sink: int, block: int) -> torch.Tensor:
 
 
 def make_qkv(B: int, H: int, n_video: int, n_sink: int, d: int, seed: int = 0,
-             device: str | torch.device = "cpu", block: int = BLOCK, amp: float = 0.5):
+             device: str | torch.device = "cpu", block: int = BLOCK, amp: float = 0.5,
+             q_offset: float = 0.0):
     """Return (Q, K, V), each bf16 [B, H, n_video + n_sink, d] on ``device``."""
     device = torch.device(device)
     N = n_video + n_sink
@@ -51,11 +59,18 @@ def make_qkv(B: int, H: int, n_video: int, n_sink: int, d: int, seed: int = 0,
         for h in range(H):
             g = torch.Generator(device=device)
             g.manual_seed(head_seed(seed, b, h, H))
+            xs = []
             for X in out:
                 c = torch.randn((max(ngroups, 1), d), generator=g, device=device, dtype=torch.float32)
                 eps = torch.randn((N, d), generator=g, device=device, dtype=torch.float32)
+                xs.append(amp * c[group] + eps if N else None)
+            if q_offset > 0:
+                o = torch.randn((d,), generator=g, device=device, dtype=torch.float32)
                 if N:
-                    X[b, h] = (amp * c[group] + eps).to(torch.bfloat16)
+                    xs[0] = xs[0] + q_offset * o
+            if N:
+                for X, x in zip(out, xs):
+                    X[b, h] = x.to(torch.bfloat16)
     return tuple(out)
 
 

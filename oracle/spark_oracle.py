@@ -52,6 +52,18 @@ Readings where the pages are silent (each the plainest one the rest supports):
   >= 0, orders its tokens by (x . v, token index) and sends the first floor(m/2)*64 to
   the left child; leaves are ordered by their smallest token index and hold their
   tokens in ascending order. Keys reuse the query partition (q_reuse_k).
+* extra tokens ([Core-node] "Block-sparse attention: one node, three backends": an
+  advanced option adds the highest-scoring tokens beyond the selected blocks, to stay
+  close to dense attention; the pages give neither the score nor the count's unit):
+  a per-head budget of E tokens, scored by the anchor score s_j = a . k_j * scale (the
+  per-token score the compressed branch already uses), ranked by (s desc, token index
+  asc) over the head's video keys. Every video query attends the extra tokens exactly
+  (those inside its selected blocks once, as part of the block); the compressed entry of
+  an unselected block then stands only for the block's remaining tokens R_b: its key
+  mean, value summary and log-mass bias are those of R_b (the mean-pool branch: mean
+  value of R_b, beta = log |R_b|), and a block whose 64 tokens are all extra has no
+  entry. Block scores (the selection) keep the whole-block means; sink queries stay
+  dense;
 * the 128-query x 64-key route ([H3-Opt] section "Manual Sparse Sage recovery": the
   sparse fallback backends consume a 128Q x 64KV route): a query tile is two consecutive video blocks
   (the last tile holds one block when nb is odd); its pooled query is the mean of the
@@ -92,11 +104,13 @@ def n_blocks(n_rows: int, n_sink: int, block: int = BLOCK) -> int:
 @dataclass
 class Pooled:
     qbar: np.ndarray    # [nt, d] mean query of each query tile (a block unless q_tile = 128)
-    kbar: np.ndarray    # [nb, d] mean key of each block
-    vtil: np.ndarray    # [nb, d] value summary of each block
-    beta: np.ndarray    # [nb]    log-mass bias of each block
+    kbar: np.ndarray    # [nb, d] mean key of each block (block scores)
+    vtil: np.ndarray    # [nb, d] value summary of each block's compressed entry
+    beta: np.ndarray    # [nb]    log-mass bias of each entry (-inf: the block has no entry)
     anchor: np.ndarray  # [d]     per-head anchor (mean video query)
-    lse: np.ndarray     # [nb]    logsumexp of the anchor scores inside each block
+    lse: np.ndarray     # [nb]    logsumexp of the anchor scores of each entry's tokens
+    kc: np.ndarray = None      # [nb, d] key mean of each entry's tokens (kbar without extra tokens)
+    extra: np.ndarray = None   # [E]  extra token indices, ascending (empty without extra tokens)
 
 
 def n_tiles(nb: int, q_tile: int = BLOCK, block: int = BLOCK) -> int:
@@ -109,7 +123,23 @@ def tile_rows(t: int, nv: int, q_tile: int = BLOCK) -> np.ndarray:
     return np.arange(t * q_tile, min((t + 1) * q_tile, nv))
 
 
-def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight", q_tile=BLOCK) -> Pooled:
+def anchor_scores(k_video, anchor, scale) -> np.ndarray:
+    """s_j = a . k_j * scale for every video key j."""
+    return (k_video @ anchor) * scale
+
+
+def select_extra_tokens(s, n_extra) -> np.ndarray:
+    """The n_extra video keys with the highest anchor scores, ranked by (s desc, index asc);
+    returned ascending."""
+    n_extra = int(min(max(n_extra, 0), s.shape[0]))
+    if n_extra == 0:
+        return np.zeros(0, dtype=np.int64)
+    j = np.arange(s.shape[0])
+    return np.sort(np.lexsort((j, -s))[:n_extra]).astype(np.int64)
+
+
+def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight", q_tile=BLOCK,
+              extra=0, extra_override=None) -> Pooled:
     """Mean pooling, anchor and Spark-Reweight summaries of one head.
 
     [Spark-H3] "What Spark-Attn changes", Spark-Reweight bullet and the figure caption:
@@ -119,6 +149,9 @@ def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight", q_tile=
     sum_j exp(s_j). ``mode="mean"`` gives the plain mean-pool branch instead.
     ``q_tile`` = 128 pools the queries over the tiles of the 128-query route (qbar has
     one row per tile); keys and the compressed branch keep 64-token blocks.
+    ``extra`` > 0 takes that many extra tokens (``extra_override``: a given token list
+    instead) out of their blocks' compressed entries, which then summarise the remaining
+    tokens of each block only (see the module header).
     """
     d = q.shape[1]
     scale = default_scale(d, scale)
@@ -134,22 +167,50 @@ def pool_head(q, k, v, n_sink, scale=None, block=BLOCK, mode="reweight", q_tile=
                          for t in range(n_tiles(nb, q_tile, block))]) if nb else np.zeros((0, d))
     kbar = kb.mean(axis=1)
     anchor = q[:nv].mean(axis=0) if nv else np.zeros(d)
-    s = (kb @ anchor) * scale                                   # [nb, block]
-    if nb:
-        smax = s.max(axis=1, keepdims=True)
-        lse = smax[:, 0] + np.log(np.exp(s - smax).sum(axis=1))
+    s = anchor_scores(k[:nv], anchor, scale).reshape(nb, block)  # [nb, block]
+    if extra_override is not None:
+        xt = np.sort(np.asarray(extra_override, dtype=np.int64))
     else:
-        lse = np.zeros(0)
-    if mode == "reweight":
-        w = np.exp(s - lse[:, None])                            # softmax inside each block
-        vtil = np.einsum("bj,bjd->bd", w, vb)
-        beta = lse - (kbar @ anchor) * scale
-    elif mode == "mean":
-        vtil = vb.mean(axis=1)
-        beta = np.full(nb, math.log(block))
-    else:
+        xt = select_extra_tokens(s.reshape(-1), extra)
+    if mode not in ("reweight", "mean"):
         raise ValueError(mode)
-    return Pooled(qbar, kbar, vtil, beta, anchor, lse)
+    if xt.size == 0:
+        if nb:
+            smax = s.max(axis=1, keepdims=True)
+            lse = smax[:, 0] + np.log(np.exp(s - smax).sum(axis=1))
+        else:
+            lse = np.zeros(0)
+        if mode == "reweight":
+            w = np.exp(s - lse[:, None])                        # softmax inside each block
+            vtil = np.einsum("bj,bjd->bd", w, vb)
+            beta = lse - (kbar @ anchor) * scale
+        else:
+            vtil = vb.mean(axis=1)
+            beta = np.full(nb, math.log(block))
+        return Pooled(qbar, kbar, vtil, beta, anchor, lse, kbar.copy(), xt)
+    # with extra tokens: each block's entry summarises its remaining tokens R_b
+    keep = np.ones(nv, dtype=bool)
+    keep[xt] = False
+    keep = keep.reshape(nb, block)
+    kc = np.zeros((nb, d))
+    vtil = np.zeros((nb, d))
+    lse = np.full(nb, -np.inf)
+    beta = np.full(nb, -np.inf)
+    for b in range(nb):
+        r = keep[b]
+        if not r.any():
+            continue                                            # every token is extra: no entry
+        kc[b] = kb[b][r].mean(axis=0)
+        sr = s[b][r]
+        m = sr.max()
+        lse[b] = m + math.log(np.exp(sr - m).sum())
+        if mode == "reweight":
+            vtil[b] = np.exp(sr - lse[b]) @ vb[b][r]
+            beta[b] = lse[b] - float(kc[b] @ anchor) * scale
+        else:
+            vtil[b] = vb[b][r].mean(axis=0)
+            beta[b] = math.log(int(r.sum()))
+    return Pooled(qbar, kbar, vtil, beta, anchor, lse, kc, xt)
 
 
 # --------------------------------------------------------------------------- scoring / selection
@@ -219,13 +280,14 @@ def _softmax_out(logits, vals):
 
 
 def attn_video_block(q, k, v, n_sink, i, sel, pooled: Pooled | None, scale=None, block=BLOCK,
-                     q_tile=BLOCK):
+                     q_tile=BLOCK, extra=None):
     """Output rows of video query tile i (block i unless ``q_tile`` = 128), in the order of q.
 
     [Spark-H3] "What Spark-Attn changes": the exact branch attends to the keys of the
     selected blocks, the compressed branch covers every other video block with one
     pooled entry each; [Core-node] sink_conditioning: every sink key is attended
-    exactly. All logits share one softmax (one log-sum-exp merge).
+    exactly, and extra_tokens adds the head's extra tokens (``extra``, token indices) to
+    the exact branch. All logits share one softmax (one log-sum-exp merge).
     """
     d = q.shape[1]
     scale = default_scale(d, scale)
@@ -233,13 +295,18 @@ def attn_video_block(q, k, v, n_sink, i, sel, pooled: Pooled | None, scale=None,
     nv = nb * block
     qi = q[tile_rows(i, nv, q_tile)]
     sel = np.asarray(sel, dtype=np.int64)
+    # extra tokens outside the selected blocks (those inside are attended as part of it)
+    xt = np.zeros(0, dtype=np.int64) if extra is None else np.asarray(extra, dtype=np.int64)
+    xt = xt[~np.isin(xt // block, sel)]
     key_rows = np.concatenate([np.arange(b * block, (b + 1) * block) for b in sel]
-                              + [np.arange(nv, q.shape[0])]).astype(np.int64)
+                              + [xt, np.arange(nv, q.shape[0])]).astype(np.int64)
     logits = (qi @ k[key_rows].T) * scale
     vals = v[key_rows]
     if pooled is not None:
         unsel = np.setdiff1d(np.arange(nb), sel)
-        logits = np.concatenate([logits, (qi @ pooled.kbar[unsel].T) * scale + pooled.beta[unsel]], axis=1)
+        unsel = unsel[np.isfinite(pooled.beta[unsel])]          # blocks left with an entry
+        kc = pooled.kbar if pooled.kc is None else pooled.kc
+        logits = np.concatenate([logits, (qi @ kc[unsel].T) * scale + pooled.beta[unsel]], axis=1)
         vals = np.concatenate([vals, pooled.vtil[unsel]], axis=0)
     return _softmax_out(logits, vals)
 
@@ -251,7 +318,7 @@ def attn_dense_rows(q, k, v, rows, scale=None):
 
 
 def attention_head(q, k, v, n_sink, sel_lists, pooled=None, scale=None, block=BLOCK,
-                   qblocks=None, dense_rows=True, q_tile=BLOCK):
+                   qblocks=None, dense_rows=True, q_tile=BLOCK, extra=None):
     """O [N, d] and LSE [N] of one head; rows not computed are NaN.
 
     ``sel_lists[i]`` is the selected block list of video query tile i (all tiles when
@@ -263,7 +330,7 @@ def attention_head(q, k, v, n_sink, sel_lists, pooled=None, scale=None, block=BL
     L = np.full(N, np.nan)
     blocks = range(n_tiles(nb, q_tile, block)) if qblocks is None else qblocks
     for t, i in enumerate(blocks):
-        o, l = attn_video_block(q, k, v, n_sink, i, sel_lists[t], pooled, scale, block, q_tile)
+        o, l = attn_video_block(q, k, v, n_sink, i, sel_lists[t], pooled, scale, block, q_tile, extra)
         rows = tile_rows(i, nb * block, q_tile)
         O[rows] = o
         L[rows] = l
@@ -403,7 +470,7 @@ def apply_perm(x, perm, n_sink, block=BLOCK):
 def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale=None,
                  block=BLOCK, reblock=False, qblocks=None, sel_override=None,
                  pool_mode="reweight", perm_override=None, reblock_kv=False,
-                 perm_k_override=None, q_tile=BLOCK):
+                 perm_k_override=None, q_tile=BLOCK, extra_tokens=0, extra_override=None):
     """The whole forward of one head, in the original token order.
 
     Returns (O [N, d], LSE [N], info) where info holds the selection lists, the pooled
@@ -414,6 +481,9 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
     keys, whitened by the queries' second moment) instead of reusing the queries'
     (the alternative to q_reuse_k in [Spark-H3] "Workflows"); K and V follow it.
     ``q_tile`` = 128: the 128-query route (``qblocks`` then lists query tiles).
+    ``extra_tokens``: the per-head budget of extra tokens (``extra_override``: the token
+    list to use instead of the oracle's own, e.g. when a near-tie lets the device take
+    another token); the tokens are indices of the (reblocked) video rows.
     """
     if q_tile not in (BLOCK, 2 * BLOCK) or block != BLOCK:
         raise ValueError("q_tile must be 64 or 128 with 64-token blocks")
@@ -438,8 +508,9 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
             kp, vp = (apply_perm(t, rb.perm, n_sink, block) for t in (k, v))
     else:
         qp, kp, vp = q, k, v
-    pooled = pool_head(qp, kp, vp, n_sink, scale, block, pool_mode, q_tile)
+    pooled = pool_head(qp, kp, vp, n_sink, scale, block, pool_mode, q_tile, extra_tokens, extra_override)
     info["pooled"] = pooled
+    info["extra"] = pooled.extra
     nb = pooled.kbar.shape[0]
     rows = np.arange(pooled.qbar.shape[0]) if qblocks is None else np.asarray(qblocks)
     if sel_override is not None:
@@ -448,7 +519,7 @@ def forward_head(q, k, v, n_sink, mode="topk", param=0.1, compressed=True, scale
         sel = select_head(pooled.qbar, pooled.kbar, scale, mode, param, rows)
     info["sel"] = sel
     O, L = attention_head(qp, kp, vp, n_sink, sel, pooled if compressed else None, scale,
-                          block, qblocks=rows, q_tile=q_tile)
+                          block, qblocks=rows, q_tile=q_tile, extra=pooled.extra)
     if reblock:
         nv = nb * block
         O2, L2 = O.copy(), L.copy()

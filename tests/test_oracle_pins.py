@@ -367,8 +367,8 @@ def test_planted_missing_scale_is_caught(monkeypatch):
 def test_planted_unweighted_summary_is_caught(monkeypatch):
     real = orc.pool_head
 
-    def bad(q, k, v, n_sink, scale=None, block=64, mode="reweight", q_tile=64):
-        P = real(q, k, v, n_sink, scale, block, mode, q_tile)
+    def bad(q, k, v, n_sink, scale=None, block=64, mode="reweight", q_tile=64, *extra_args):
+        P = real(q, k, v, n_sink, scale, block, mode, q_tile, *extra_args)
         nb = P.kbar.shape[0]
         P.vtil = v[: nb * block].reshape(nb, block, -1).mean(1)
         return P
@@ -426,13 +426,15 @@ def test_whitening_is_mahalanobis_cosine_via_reblock():
 # mean pooling gives exp(E[x]) where the softmax needs E[exp(x)]. On seeded synthetic
 # heads the oracle must order the three forwards by their distance to dense attention:
 # no compressed branch > mean-pooled branch > reweighted branch.
-@pytest.mark.parametrize("nv,ns,d,ratio,amp,seed", [
-    (64 * 48, 32, 64, 0.1, 0.5, 0),
-    (64 * 48, 32, 64, 0.2, 0.5, 1),
-    (64 * 48, 32, 64, 0.1, 1.0, 3),
+@pytest.mark.parametrize("nv,ns,d,ratio,amp,seed,q_offset", [
+    (64 * 48, 32, 64, 0.1, 0.5, 0, 0.0),
+    (64 * 48, 32, 64, 0.2, 0.5, 1, 0.0),
+    (64 * 48, 32, 64, 0.1, 1.0, 3, 0.0),
+    (64 * 48, 32, 64, 0.1, 0.5, 5, 1.0),   # queries with a mean direction: beta far from log 64
+    (64 * 48, 0, 128, 0.2, 0.5, 6, 1.0),
 ])
-def test_compressed_branch_fidelity_ordering(nv, ns, d, ratio, amp, seed):
-    Q, K, V = make_qkv(1, 1, nv, ns, d, seed=seed, amp=amp)
+def test_compressed_branch_fidelity_ordering(nv, ns, d, ratio, amp, seed, q_offset):
+    Q, K, V = make_qkv(1, 1, nv, ns, d, seed=seed, amp=amp, q_offset=q_offset)
     q, k, v = (orc.to_f64(t[0, 0]) for t in (Q, K, V))
     dense, _, _ = orc.forward_head(q, k, v, ns, "topk", 1.0, False)
     err = {}
@@ -441,6 +443,20 @@ def test_compressed_branch_fidelity_ordering(nv, ns, d, ratio, amp, seed):
         o, _, _ = orc.forward_head(q, k, v, ns, "topk", ratio, comp, pool_mode=pm)
         err[name] = np.linalg.norm(o[:nv] - dense[:nv]) / np.linalg.norm(dense[:nv])
     assert err["reweight"] < err["mean"] < err["none"], err
+
+
+def test_offset_queries_move_beta_away_from_log64():
+    """The query-offset input family exercises Spark-Reweight: with a mean query direction
+    the anchor is long, the anchor scores inside a block spread, and the log-mass bias
+    beta_b = lse_b - a . kbar_b * scale (>= log 64 by Jensen) departs from log 64 by O(1);
+    without the offset it stays within a few hundredths of it."""
+    for q_offset, lo, hi in ((0.0, 0.0, 0.05), (1.0, 0.2, 2.0)):
+        Q, K, V = make_qkv(1, 1, 64 * 64, 16, 128, seed=8, q_offset=q_offset)
+        q, k, v = (orc.to_f64(t[0, 0]) for t in (Q, K, V))
+        P = orc.pool_head(q, k, v, 16, 1 / math.sqrt(128))
+        excess = P.beta - math.log(64)
+        assert np.all(excess >= -1e-12)
+        assert lo <= float(excess.mean()) <= hi, (q_offset, float(excess.mean()))
 
 
 # --------------------------------------------------------------------------- keys' own partition
@@ -542,3 +558,174 @@ def test_planted_end_aligned_last_tile_is_caught(monkeypatch):
     monkeypatch.setattr(orc, "tile_rows", end_aligned)
     with pytest.raises(AssertionError):
         test_q128_tile_scores_are_means_of_block_scores()
+
+
+# --------------------------------------------------------------------------- extra tokens
+# [Core-node] "Block-sparse attention: one node, three backends": extra_tokens adds the
+# highest-scoring tokens beyond the selected blocks. Reading: a per-head budget of E tokens
+# ranked by the anchor score s_j = a . k_j * scale (ties to the lower index); they join
+# every video query's exact branch, and each compressed entry summarises only its block's
+# remaining tokens (no entry when all 64 are extra).
+
+def _anchor_head(nv=640, ns=16, d=32, seed=7):
+    """Queries whose mean is a known anchor a, some rows exactly a (as in the anchor pin)."""
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal(d)
+    delta = rng.standard_normal((nv // 2, d)) * 1.3
+    delta[::9] = 0.0
+    q = np.concatenate([a + delta, a - delta])
+    q = q[rng.permutation(nv)]
+    q = np.concatenate([q, rng.standard_normal((ns, d))])
+    k = rng.standard_normal((nv + ns, d)) + 0.4 * np.repeat(rng.standard_normal((nv // 64 + 1, d)), 64, 0)[: nv + ns]
+    v = rng.standard_normal((nv + ns, d))
+    return q, k, v, a
+
+
+@pytest.mark.parametrize("E,pool_mode", [(1, "reweight"), (37, "reweight"), (200, "reweight"),
+                                         (64 * 3 + 5, "reweight"), (37, "mean")])
+def test_extra_tokens_keep_anchor_rows_exact(E, pool_mode):
+    """Mass bookkeeping: for a query equal to the anchor every entry of the reweighted
+    branch carries exactly the mass and mass-weighted value of the tokens it stands for,
+    and the extra tokens are exact, so anchor rows still get dense attention whatever
+    tokens were taken out of the blocks (a recomputation over the wrong token set, or an
+    extra token counted twice, breaks this). The mean-pool branch is not exact there;
+    its entries must stand for |R_b| tokens at the pooled logit (closed form below)."""
+    q, k, v, a = _anchor_head()
+    nv, ns, d = 640, 16, 32
+    scale = 1 / math.sqrt(d)
+    O, L, info = orc.forward_head(q, k, v, ns, "topk", 0.2, compressed=True, extra_tokens=E,
+                                  pool_mode=pool_mode)
+    P = info["pooled"]
+    assert P.extra.shape == (E,) and np.all(np.diff(P.extra) > 0)
+    s = k[:nv] @ a * scale
+    # the extra set: the E largest anchor scores
+    assert s[P.extra].min() >= np.sort(s)[::-1][E - 1]
+    keep = np.ones(nv, bool)
+    keep[P.extra] = False
+    for b in range(nv // 64):
+        r = keep[b * 64:(b + 1) * 64]
+        if pool_mode == "mean" and r.any():
+            assert math.isclose(P.beta[b], math.log(r.sum()), rel_tol=0, abs_tol=1e-14)
+            np.testing.assert_allclose(P.vtil[b], v[b * 64:(b + 1) * 64][r].mean(0), atol=1e-14)
+        if pool_mode == "reweight" and r.any():
+            mass = np.exp(s[b * 64:(b + 1) * 64][r]).sum()
+            np.testing.assert_allclose(np.exp(P.kc[b] @ a * scale + P.beta[b]), mass, rtol=1e-13)
+        if not r.any():
+            assert P.beta[b] == -np.inf
+    if pool_mode == "reweight":
+        ref = sdpa64(q, k, v, scale)
+        rows = np.nonzero(np.all(np.abs(q[:nv] - a) < 1e-15, axis=1))[0]
+        np.testing.assert_allclose(O[rows], ref[rows], atol=1e-11, rtol=0)
+        np.testing.assert_allclose(L[rows], lse64(q, k, scale)[rows], atol=1e-11, rtol=0)
+
+
+def test_extra_tokens_covering_a_block_equal_selecting_it():
+    """When the E = 64 highest anchor scores are exactly the tokens of one block b (its keys
+    are shifted along the anchor), taking them as extra tokens gives the same forward as
+    adding b to every query block's selection without extra tokens."""
+    nv, ns, d = 64 * 12, 20, 32
+    q, k, v = head(nv, ns, d, seed=41)
+    a = q[:nv].mean(0)
+    b = 7
+    k[b * 64:(b + 1) * 64] += 6.0 * a / np.linalg.norm(a)
+    O1, L1, info = orc.forward_head(q, k, v, ns, "topk", 0.25, compressed=True, extra_tokens=64)
+    np.testing.assert_array_equal(info["extra"], np.arange(b * 64, (b + 1) * 64))
+    assert info["pooled"].beta[b] == -np.inf
+    sel = [np.union1d(s_, [b]) for s_ in info["sel"]]
+    assert any(b not in s_ for s_ in info["sel"])
+    O2, L2, _ = orc.forward_head(q, k, v, ns, "topk", 0.25, compressed=True, sel_override=sel)
+    np.testing.assert_allclose(O1, O2, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(L1, L2, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("compressed", [True, False])
+def test_all_tokens_extra_is_dense_attention(compressed):
+    """E >= the number of video tokens makes every key exact: dense attention for every row."""
+    nv, ns, d = 64 * 6 + 13, 9, 32
+    q, k, v = head(nv, ns, d, seed=2)
+    O, L, info = orc.forward_head(q, k, v, ns, "topk", 0.2, compressed=compressed, extra_tokens=10 ** 6)
+    scale = 1 / math.sqrt(d)
+    assert info["extra"].shape == (64 * 6,)
+    np.testing.assert_allclose(O, sdpa64(q, k, v, scale), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(L, lse64(q, k, scale), atol=1e-12, rtol=0)
+
+
+def test_extra_token_ties_go_to_the_lower_index():
+    """Hand-derived: keys 5 and 200 are the same vector, the largest anchor score; with a
+    budget of one token the lower index is taken, with two both are."""
+    nv, d = 64 * 4, 16
+    rng = np.random.default_rng(3)
+    a = rng.standard_normal(d)
+    k = rng.standard_normal((nv, d)) * 0.1
+    k[5] = k[200] = 3.0 * a
+    s = k @ a
+    np.testing.assert_array_equal(orc.select_extra_tokens(s, 1), [5])
+    np.testing.assert_array_equal(orc.select_extra_tokens(s, 2), [5, 200])
+    assert orc.select_extra_tokens(s, 0).size == 0
+
+
+def test_extra_tokens_zero_changes_nothing():
+    q, k, v = head(64 * 10, 12, 32, seed=9)
+    O0, L0, _ = orc.forward_head(q, k, v, 12, "tau", 0.8, compressed=True)
+    O1, L1, info = orc.forward_head(q, k, v, 12, "tau", 0.8, compressed=True, extra_tokens=0)
+    assert info["extra"].size == 0
+    np.testing.assert_array_equal(O0, O1)
+    np.testing.assert_array_equal(L0, L1)
+
+
+@pytest.mark.parametrize("q_offset", [0.0, 1.0])
+def test_extra_tokens_bring_the_forward_closer_to_dense(q_offset):
+    """Fidelity: taking the highest-scoring tokens out of the compressed entries into the
+    exact branch moves the output toward dense attention, with and without the compressed
+    branch."""
+    nv, ns, d = 64 * 40, 16, 64
+    Q, K, V = make_qkv(1, 1, nv, ns, d, seed=12, q_offset=q_offset)
+    q, k, v = (orc.to_f64(t[0, 0]) for t in (Q, K, V))
+    dense, _, _ = orc.forward_head(q, k, v, ns, "topk", 1.0, False)
+    for comp in (True, False):
+        err = []
+        for E in (0, 256, 1024):
+            o, _, _ = orc.forward_head(q, k, v, ns, "topk", 0.1, comp, extra_tokens=E)
+            err.append(np.linalg.norm(o[:nv] - dense[:nv]) / np.linalg.norm(dense[:nv]))
+        assert err[0] > err[1] > err[2], (comp, err)
+
+
+def test_planted_extra_token_counted_twice_is_caught(monkeypatch):
+    """An extra token inside a selected block attended a second time must break the
+    anchor-row pin."""
+    real = orc.attn_video_block
+
+    def bad(q, k, v, n_sink, i, sel, pooled, scale=None, block=64, q_tile=64, extra=None):
+        o, l = real(q, k, v, n_sink, i, sel, pooled, scale, block, q_tile, None)
+        if extra is None or len(extra) == 0:
+            return o, l
+        # recompute with every extra token appended, duplicates included
+        sel = np.asarray(sel, dtype=np.int64)
+        nv = orc.n_blocks(q.shape[0], n_sink, block) * block
+        rows = np.concatenate([np.arange(b * block, (b + 1) * block) for b in sel]
+                              + [np.asarray(extra, dtype=np.int64), np.arange(nv, q.shape[0])])
+        qi = q[orc.tile_rows(i, nv, q_tile)]
+        lg = (qi @ k[rows].T) * scale
+        unsel = np.setdiff1d(np.arange(nv // block), sel)
+        unsel = unsel[np.isfinite(pooled.beta[unsel])]
+        lg = np.concatenate([lg, (qi @ pooled.kc[unsel].T) * scale + pooled.beta[unsel]], axis=1)
+        vals = np.concatenate([v[rows], pooled.vtil[unsel]], axis=0)
+        return orc._softmax_out(lg, vals)
+    monkeypatch.setattr(orc, "attn_video_block", bad)
+    with pytest.raises(AssertionError):
+        test_extra_tokens_keep_anchor_rows_exact(200, "reweight")
+
+
+def test_planted_entry_over_the_whole_block_is_caught(monkeypatch):
+    """Keeping the whole-block summary after taking tokens out (mass counted twice) must
+    break the anchor-row pin."""
+    real = orc.pool_head
+
+    def bad(q, k, v, n_sink, scale=None, block=64, mode="reweight", q_tile=64, extra=0, extra_override=None):
+        P = real(q, k, v, n_sink, scale, block, mode, q_tile, extra, extra_override)
+        P0 = real(q, k, v, n_sink, scale, block, mode, q_tile, 0, None)
+        P.kc, P.vtil, P.beta, P.lse = P0.kc, P0.vtil, P0.beta, P0.lse
+        return P
+    monkeypatch.setattr(orc, "pool_head", bad)
+    with pytest.raises(AssertionError):
+        test_extra_tokens_keep_anchor_rows_exact(200, "reweight")
