@@ -11,8 +11,13 @@ exact-only call, the tau-threshold selection, the full-density run and the 1344x
 240-frame Spark-Reblock forward (reblock included in the step). ``--heads`` shrinks a
 workload for profiling.
 
-Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling); the
-only collectives are the timing barrier and the max-over-ranks of the elapsed time.
+Multi-GPU: ``--gpus N`` without a torchrun environment re-launches itself under torchrun
+with N ranks (one process per GPU). Every rank runs its own independent problem (weak
+scaling, replicas); the only collectives are the timing barrier and the max-over-ranks of
+the elapsed time.
+
+Before the timed region, rank 0 checks head 0's block selection against the fp64 oracle
+on sampled query tiles (tie window 1e-4) and fails the run on a mismatch.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a bounded
 sample of the same workload (rank 0 only).
@@ -36,6 +41,15 @@ sys.path.insert(0, ROOT)
 METRIC = "ms/call & dense-equiv TFLOP/s of sparse attn fwd at 10% density, N=175,680"
 
 
+def unit_of(w: "Workload") -> str:
+    """The unit string of a workload's line (the same on both arms)."""
+    return f"TFLOP/s dense-equivalent (4*B*H*N^2*d / time, N={w.nv + w.ns:,})"
+
+
+def metric_of(w: "Workload") -> str:
+    return METRIC if w.name == DEFAULT else f"ms/call & dense-equiv TFLOP/s of sparse attn fwd, workload {w.name}"
+
+
 @dataclass
 class Workload:
     name: str
@@ -51,6 +65,7 @@ class Workload:
     B: int = 1
     d: int = 128
     q_tile: int = 64
+    extra_tokens: int = 0
 
 
 WORKLOADS = {w.name: w for w in [
@@ -82,20 +97,23 @@ WORKLOADS = {w.name: w for w in [
              24, 175680, 512, param=1.0, compressed=False, q_tile=128),
     Workload("1344x768x240-reblock-q128", "as 1344x768x240-reblock on the 128-query route (a tile pairs "
              "two consecutive leaves)", 24, 245952, 512, reblock=True, q_tile=128),
+    Workload("1152x640x243-extra512", "as 1152x640x243 with 512 extra tokens per head (the highest "
+             "anchor scores) added to every video query's exact branch", 24, 175680, 512, extra_tokens=512),
 ]}
 DEFAULT = "1152x640x243"
 
 
-def flop_counts(w: Workload, nb: int, kept_qrows: int, h=None):
+def flop_counts(w: Workload, nb: int, kept_qrows: int, h=None, extra_qrows: int = 0):
     """Algorithmic FLOPs of one forward (4*d per query-key pair: QK^T and PV).
 
     kept_qrows = selected (video query row, key block) pairs over all heads: the sum over
-    query tiles of (kept blocks x rows of the tile)."""
+    query tiles of (kept blocks x rows of the tile); extra_qrows = (video query row, extra
+    token outside the row's selected blocks) pairs."""
     h = w.H if h is None else h
     nv = nb * 64
     n = nv + w.ns
     d, b = w.d, w.B
-    exact = kept_qrows * 64 * 4 * d
+    exact = kept_qrows * 64 * 4 * d + extra_qrows * 4 * d
     sink_keys = b * h * nv * w.ns * 4 * d          # video queries x dense keys
     sink_queries = b * h * w.ns * n * 4 * d        # dense queries x all keys
     compressed = (b * h * nv * nb - kept_qrows) * 4 * d if w.compressed else 0
@@ -199,6 +217,93 @@ def phase_bytes(w: Workload, h: int, nb: int, nt: int, kept_blocks: int, kcap: i
     return dict(pool=pool, select=select, reblock_gather=gather)
 
 
+# fp32 FMA peak of the score kernel's bound: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz
+FP32_PEAK_TFLOPS = round(148 * 128 * 2 * 1965e6 / 1e12, 1)
+# bf16 dense tensor rate per SM per clock (kind::f16, M = 128): 2.25 PFLOP/s nominal /
+# (148 SMs x 1.855 GHz) = 8,192 flop/clk/SM
+TENSOR_FLOP_PER_CLK_SM = 8192
+
+
+def clock_normalised(achieved_tflops, sm_mhz):
+    """The attention kernel's tensor work per SM clock at the median clock it ran at,
+    against the nominal rate and against cuBLAS at its own measured clock (the sustained
+    peak of MEASURED_PEAKS.json and the median clock under load it was taken at)."""
+    if not sm_mhz:
+        return None
+    per_clk = achieved_tflops * 1e12 / (148 * sm_mhz * 1e6)
+    out = {"sm_mhz": sm_mhz, "flop_per_clk_per_sm": round(per_clk, 1),
+           "frac_of_nominal_rate": round(per_clk / TENSOR_FLOP_PER_CLK_SM, 4)}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        mhz = mp["clocks_under_load"]["sm_mhz_median"]
+        cub = mp["bf16_tflops_sustained"] * 1e12 / (148 * mhz * 1e6)
+        out.update(cublas_flop_per_clk_per_sm=round(cub, 1), cublas_mhz=mhz,
+                   frac_of_cublas_at_same_clock=round(per_clk / cub, 4))
+    except Exception:
+        pass
+    return out
+
+
+def route_check(w: Workload, plan, Qc, Kc, Vc, n_rows, seed=0):
+    """The device's block selection of head (0, 0) against the fp64 oracle on ``n_rows``
+    sampled query tiles (plus the first and the last): each device row must equal the
+    oracle's, except blocks whose oracle score lies within the tie window (1e-4) of the
+    cut (the k-th score for top-k, the threshold for tau). Raises on a mismatch. With
+    Reblock, the oracle applies the device's permutation after checking that it is one
+    (every leaf 64 ascending tokens), as the parity tests do."""
+    import numpy as np
+
+    import oracle.spark_oracle as orc
+
+    TIE = 1e-4
+    t0 = time.perf_counter()
+    q, k, v = (orc.to_f64(t[0, 0]) for t in (Qc, Kc, Vc))
+    nb = plan.nb
+    if nb == 0:
+        return {"ok": True, "rows": 0, "note": "no video block"}
+    if w.reblock:
+        nv = nb * 64
+
+        def device_perm(name):
+            perm = plan.rb[name][0, 0].cpu().numpy().astype(np.int64)
+            leaves = perm.reshape(-1, 64)
+            if (sorted(perm.tolist()) != list(range(nv)) or np.any(np.diff(leaves, axis=1) <= 0)):
+                raise RuntimeError(f"route check: the device's {name} is not a leaf permutation")
+            return perm
+        perm = device_perm("perm")
+        q = orc.apply_perm(q, perm, w.ns)
+        kperm = device_perm("perm_k") if w.reblock_kv else perm
+        k = orc.apply_perm(k, kperm, w.ns)
+    scale = 1.0 / math.sqrt(w.d)
+    P = orc.pool_head(q, k, v, w.ns, scale, 64, "reweight", w.q_tile)
+    nt = P.qbar.shape[0]
+    rng = np.random.default_rng(seed + 17)
+    rows = np.unique(np.concatenate([[0, nt - 1], rng.choice(nt, min(n_rows, nt), replace=False)]))
+    S = orc.block_scores(P.qbar, P.kbar, scale, rows)
+    thr = orc.tau_threshold(orc.block_scores(P.qbar, P.kbar, scale), w.param) if w.mode == "tau" else None
+    idx = plan.idx[0, 0].cpu().numpy()
+    cnt = plan.cnt[0, 0].cpu().numpy()
+    n_tie = 0
+    for t, i in enumerate(rows):
+        g = np.sort(idx[i, : cnt[i]].astype(np.int64))
+        if w.mode == "topk":
+            kk = orc.topk_count(w.param, nb)
+            ref = orc.select_topk_row(S[t], kk)
+            cut = np.sort(S[t])[::-1][kk - 1]
+            if g.shape[0] != kk:
+                raise RuntimeError(f"route check: row {i} keeps {g.shape[0]} blocks, not {kk}")
+        else:
+            ref = orc.select_tau_row(S[t], thr)
+            cut = thr
+        diff = np.setxor1d(ref, g)
+        if diff.size and not np.all(np.abs(S[t][diff] - cut) < TIE):
+            raise RuntimeError(f"route check: row {i} of head 0 differs from the oracle beyond the tie window")
+        n_tie += int(diff.size)
+    return {"ok": True, "head": 0, "rows": int(rows.size), "tie_window": TIE,
+            "blocks_differing_at_ties": n_tie, "seconds": round(time.perf_counter() - t0, 2)}
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -227,7 +332,7 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     N = w.nv + w.ns
     Q, K, V = make_qkv(w.B, h, w.nv, w.ns, w.d, seed=args.seed + rank, device=dev)
     cfg = spark.ForwardConfig(w.mode, w.param, w.compressed, reblock=w.reblock, reblock_kv=w.reblock_kv,
-                              q_tile=w.q_tile)
+                              q_tile=w.q_tile, extra_tokens=w.extra_tokens)
     plan = spark.SparkAttention(w.B, h, N, w.d, w.ns, cfg, dev)
     nb, nt = plan.nb, plan.nt
     stream = torch.cuda.current_stream(dev)
@@ -238,13 +343,33 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
     err = spark.device_error(dev)
     if err != 0:
         raise RuntimeError(f"device error {err} ({spark.strerror(err)})")
+    # the route (block selection) of head 0 against the fp64 oracle before any timing; a
+    # mismatch outside the tie window fails the run
+    route = None
+    if rank == 0 and not args.no_route_check:
+        route = route_check(w, plan, Q[:1, :1].cpu(), K[:1, :1].cpu(), V[:1, :1].cpu(),
+                            args.route_rows, seed=args.seed)
     kept = int(plan.cnt.to(torch.int64).sum().item()) if nb > 0 else 0
     rows = torch.full((nt,), w.q_tile, dtype=torch.int64, device=dev)
     if nt:
         rows[-1] = nb * 64 - (nt - 1) * w.q_tile   # a one-block last tile on the 128-query route
     kept_qrows = int((plan.cnt.to(torch.int64) * rows).sum().item()) if nb > 0 else 0
-    fl = flop_counts(w, nb, kept_qrows, h)
+    extra_qrows = 0
+    if w.extra_tokens and nb > 0:
+        # extra tokens outside each tile's selected blocks, times the tile's rows
+        sel = torch.zeros((w.B, h, nt, nb), dtype=torch.int32, device=dev)
+        slot = torch.arange(plan.kcap, device=dev)[None, None, None, :] < plan.cnt[..., None]
+        sel.scatter_add_(3, torch.where(slot, plan.idx, 0).long(), slot.to(torch.int32))
+        xb = (plan.extra_rows().long() // 64)[:, :, None, :].expand(-1, -1, nt, -1)
+        outside = (torch.gather(sel, 3, xb) == 0).sum(dim=3)
+        extra_qrows = int((outside * rows).sum().item())
+        del sel, xb
+    fl = flop_counts(w, nb, kept_qrows, h, extra_qrows)
     by = phase_bytes(w, h, nb, nt, kept, plan.kcap)
+
+    cpu_line = None
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        cpu_line = cpu_baseline(w, Q[:, :1].cpu(), K[:, :1].cpu(), V[:, :1].cpu(), args.cpu_blocks or 200)
 
     ev = []
     if world > 1:
@@ -306,13 +431,19 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
 
     def gbs(nbytes, t_ms):
         return round(nbytes / (t_ms * 1e-3) / 1e9, 1) if t_ms > 0 else None
+    score_flops = 2 * w.B * h * nt * nb * w.d
     phases = {
         "pool": {"ms": round(phase_ms["pool"], 3), "bytes": by["pool"],
                  "GB/s": gbs(by["pool"], phase_ms["pool"]),
                  "frac_hbm": round(by["pool"] / (phase_ms["pool"] * 1e-3) / 1e9 / hbm, 3)},
         "select": {"ms": round(phase_ms["select"], 3), "bytes": by["select"],
                    "GB/s": gbs(by["select"], phase_ms["select"]),
-                   "score_flops": 2 * w.B * h * nt * nb * w.d},
+                   "frac_hbm": round(by["select"] / (phase_ms["select"] * 1e-3) / 1e9 / hbm, 4),
+                   "score_flops": score_flops,
+                   "fp32_tflops": round(score_flops / (phase_ms["select"] * 1e-3) / 1e12, 2),
+                   "frac_fp32": round(score_flops / (phase_ms["select"] * 1e-3) / 1e12 / FP32_PEAK_TFLOPS, 4),
+                   "bound": f"fp32 FMA (scores), peak {FP32_PEAK_TFLOPS} TFLOP/s = 148 SMs x 128 lanes "
+                            "x 2 flop x 1965 MHz"},
         "attn": {"ms": round(attn_ms, 3), "selected_flops": fl["selected"],
                  "compressed_flops": fl["compressed"]},
     }
@@ -320,10 +451,9 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
         phases["reblock"] = {"ms": round(phase_ms["reblock"], 3),
                              "gather_bytes": by["reblock_gather"]}
     line = {
-        "metric": METRIC if w.name == DEFAULT else
-        f"ms/call & dense-equiv TFLOP/s of sparse attn fwd, workload {w.name}",
+        "metric": metric_of(w),
         "value": round(value, 2),
-        "unit": f"TFLOP/s dense-equivalent (4*B*H*N^2*d / time, N={N:,})",
+        "unit": unit_of(w),
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -352,7 +482,8 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
                      "frac": round(achieved / (bf16_sust or bf16_peak), 4),
                      "peak_source": f"{peak_src} bf16 sustained (burst {bf16_peak})",
                      "algorithmic_flops_per_launch": fl["attn_total"],
-                     "traffic": ATTN_TRAFFIC_BYTES.get(w.name) if not args.heads else None},
+                     "traffic": ATTN_TRAFFIC_BYTES.get(w.name) if not args.heads else None,
+                     "clock_normalised": clock_normalised(achieved, clocks.get("sm_mhz"))},
         "e2e": {"value": round(world * fl["dense_equiv"] / (e2e_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s dense-equivalent, host buffers, copies inside the timed region",
                 "ms_per_step": round(e2e_ms, 3),
@@ -362,10 +493,12 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
                 "d2h_bytes_per_step": plan.O.numel() * plan.O.element_size()},
         "gpu_launches": launches,
         "clocks": clocks,
+        "route_checked": bool(route and route["ok"]),
     }
-    if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, Q[:, :1].cpu(), K[:, :1].cpu(), V[:, :1].cpu(),
-                                            args.cpu_blocks or 200)
+    if route is not None:
+        line["route_check"] = route
+    if cpu_line is not None:
+        line["cpu_baseline"] = cpu_line
     return line
 
 
@@ -428,19 +561,42 @@ def run_reference(args, w: Workload, rank, world):
     cb = dict(info)
     cb["value"] = round(value, 6)
     return {
-        "impl": "reference", "metric": METRIC if w.name == DEFAULT else
-        f"ms/call & dense-equiv TFLOP/s of sparse attn fwd, workload {w.name}",
+        "impl": "reference", "metric": metric_of(w),
         "value": round(value, 6),
-        "unit": "TFLOP/s dense-equivalent", "n_gpus": world, "steps": args.steps,
+        "unit": unit_of(w), "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded block-correlated N(0,1) Q/K/V, one head drawn on the host)",
         "config": {"workload": w.name, "sample": info["sample"]},
         "cpu_baseline": cb,
-        "e2e": {"value": round(value, 6), "unit": "TFLOP/s dense-equivalent",
+        "e2e": {"value": round(value, 6), "unit": unit_of(w),
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
+
+
+def spawn_ranks_command(argv, n, port):
+    """torchrun command that runs this benchmark with the same arguments on n local ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+            *argv]
+
+
+def spawn_ranks(argv, n, timeout_s=3600):
+    """Run the benchmark on n ranks (torchrun, rendezvous on 127.0.0.1) and return its exit
+    status; the whole process group is killed if it outlives ``timeout_s``."""
+    import signal
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    proc = subprocess.Popen(spawn_ranks_command(argv, n, port), start_new_session=True)
+    try:
+        return proc.wait(timeout=timeout_s)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGKILL)
+        proc.wait()
+        return 124
 
 
 def main():
@@ -456,11 +612,18 @@ def main():
     ap.add_argument("--cpu-blocks", type=int, default=0,
                     help="query blocks in the oracle sample (default: 200 for cpu_baseline, 64 per reference step)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-route-check", action="store_true",
+                    help="skip the check of head 0's selection against the oracle before timing")
+    ap.add_argument("--route-rows", type=int, default=24,
+                    help="query tiles of head 0 whose selection is checked against the oracle")
     args = ap.parse_args()
     if args.impl == "spark" and args.warmup < 3:
         args.warmup = 3
     w = WORKLOADS[args.workload]
 
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: re-launch this command under torchrun with N ranks
+        sys.exit(spawn_ranks(sys.argv[1:], args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

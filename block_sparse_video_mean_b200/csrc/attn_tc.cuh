@@ -41,19 +41,11 @@
 #include "spark_common.cuh"
 #include "tc_util.cuh"
 
-// Timing hooks for out-of-tree instrumented builds; no-ops here.
-#ifndef SPARK_TC_T0
-#define SPARK_TC_T0(v)
-#define SPARK_TC_ACC(slot, v)
-#define SPARK_TC_EV(who, what)
-#define SPARK_TC_DECL
-#define SPARK_TC_FLUSH
-#endif
-
 namespace spark {
 
 struct TcMaps {
   CUtensorMap k, v, kp, vp;  // K, V over [B*H*N, D]; pooled pack over [B*H*nb, D]
+  CUtensorMap kx, vx;        // extra-token rows over [B*H*ep, D] (the extra pack)
 };
 
 struct TcParams {
@@ -68,6 +60,9 @@ struct TcParams {
   int nt;  // video query tiles per head (the 128-query route; nb for 64-query tiles)
   float scale_log2;
   int* item_ctr;  // per-launch counter of items handed out (zeroed before the launch)
+  long long wait_clocks;  // limit of every pipeline wait (the drains keep the default)
+  const int32_t* xidx;    // extra tokens [B*H, ep] (video rows, -1 past n_extra); extra only
+  int n_xh, n_extra, ep;  // extra halves per video item, extra tokens per head, padded rows
 };
 
 // Items handed out at run time: the claiming warp takes the next item index from the
@@ -82,7 +77,7 @@ struct TcQueue {
   // The claiming warp (all lanes): entry j gets the next item index (or -1).
   __device__ __forceinline__ bool claim(uint32_t j, const TcParams& p, volatile int* abort_flag, int* id) {
     const int e = j % kQueueLen;
-    const bool ok = j < (uint32_t)kQueueLen || tc::mbar_wait(&empty[e], ((j / kQueueLen) - 1) & 1, abort_flag);
+    const bool ok = j < (uint32_t)kQueueLen || tc::mbar_wait(&empty[e], ((j / kQueueLen) - 1) & 1, abort_flag, p.wait_clocks);
     if (!__all_sync(0xffffffffu, ok)) return false;
     int v = 0;
     if ((threadIdx.x & 31) == 0) {
@@ -95,9 +90,10 @@ struct TcQueue {
     return true;
   }
   // A reading warp (all lanes) or a single reading thread (one_thread): entry j.
-  __device__ __forceinline__ bool read(uint32_t j, volatile int* abort_flag, int* id, bool one_thread) {
+  __device__ __forceinline__ bool read(uint32_t j, volatile int* abort_flag, int* id, bool one_thread,
+                                       long long limit) {
     const int e = j % kQueueLen;
-    bool ok = tc::mbar_wait(&full[e], (j / kQueueLen) & 1, abort_flag);
+    bool ok = tc::mbar_wait(&full[e], (j / kQueueLen) & 1, abort_flag, limit);
     if (!one_thread) ok = __all_sync(0xffffffffu, ok);
     if (!ok) return false;
     *id = ids[e];
@@ -172,7 +168,7 @@ __device__ __forceinline__ TcItem tc_item(const TcParams& p, int it) {
     int c = p.cnt[r.row];
     c = c < 0 ? 0 : (c > p.kcap ? p.kcap : c);
     r.cnt = c;
-    r.nhalf = c + n_dk + (p.pooled ? p.nbp / kBlock : 0);
+    r.nhalf = c + n_dk + p.n_xh + (p.pooled ? p.nbp / kBlock : 0);
   }
   r.ntiles = (r.nhalf + 1) / 2;
   r.nq = min(kBlock, p.N - r.q0);
@@ -215,16 +211,40 @@ __device__ __forceinline__ uint64_t tc_vdesc(uint32_t stage_addr, int kk) {
   return tc::make_sdesc(stage_addr + kk * 2048, TcCfg<D>::kPanelBytes, 1024, tc::kSwizzle128);
 }
 
-// The four 64-key half kinds of a tile.
-enum : int { kHalfExact = 0, kHalfDense = 1, kHalfPooled = 2, kHalfMissing = 3 };
+// The 64-key half kinds of a tile. A video item runs its halves in the order: selected
+// blocks, dense key rows, extra tokens, pooled entries.
+enum : int { kHalfExact = 0, kHalfDense = 1, kHalfPooled = 2, kHalfMissing = 3, kHalfExtra = 4 };
 
-// Kind and first key / pooled entry of half `hi` of item I (video or dense).
-__device__ __forceinline__ int tc_half_kind(const TcItem& I, int hi, int n_dk) {
+// Kind of half `hi` of item I (video or dense).
+__device__ __forceinline__ int tc_half_kind(const TcItem& I, int hi, int n_dk, int n_xh) {
   if (hi >= I.nhalf) return kHalfMissing;
   if (I.dense) return kHalfDense;
   if (hi < I.cnt) return kHalfExact;
   if (hi < I.cnt + n_dk) return kHalfDense;
+  if (hi < I.cnt + n_dk + n_xh) return kHalfExtra;
   return kHalfPooled;
+}
+
+// Masks the extra-token entries of half `e0 / 64` in x: entries past the head's count and
+// tokens whose block the item selected (already attended there).
+__device__ __forceinline__ void tc_mask_extra(float* x, const int32_t* xs, int e0, int n_extra,
+                                              const uint32_t* bm) {
+#pragma unroll
+  for (int q4 = 0; q4 < 16; ++q4) {
+    const int4 t4 = __ldg(reinterpret_cast<const int4*>(xs + e0) + q4);
+    const int tt[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 4 * q4 + i;
+      const int tok = tt[i];
+      bool masked = e0 + e >= n_extra || tok < 0;
+      if (!masked) {
+        const int blk = tok >> 6;
+        masked = (bm[blk >> 5] >> (blk & 31)) & 1u;
+      }
+      if (masked) x[e] = -INFINITY;
+    }
+  }
 }
 
 template <int D>
@@ -259,7 +279,6 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  SPARK_TC_DECL
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       tc::mbar_init(&kfull[i], 1);
@@ -296,6 +315,8 @@ __global__ void __launch_bounds__(384, 1)
     tc::tma_prefetch_desc(&maps.v);
     tc::tma_prefetch_desc(&maps.kp);
     tc::tma_prefetch_desc(&maps.vp);
+    tc::tma_prefetch_desc(&maps.kx);
+    tc::tma_prefetch_desc(&maps.vx);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -319,6 +340,7 @@ __global__ void __launch_bounds__(384, 1)
     unsigned char* rbase = is_v ? vring : ring;
     const CUtensorMap* map_x = is_v ? &maps.v : &maps.k;
     const CUtensorMap* map_p = is_v ? &maps.vp : &maps.kp;
+    const CUtensorMap* map_e = is_v ? &maps.vx : &maps.kx;
     // The whole warp walks the tile sequence (warp 8 claims each slot's items, warp 10
     // reads them from the slot's queue); the selected block indices are fetched 32 halves
     // at a time, one chunk ahead, so no global load sits on the issue path.
@@ -327,7 +349,7 @@ __global__ void __launch_bounds__(384, 1)
     auto take_nonempty = [&](int s, TcItem* I) -> bool {
       while (true) {
         int id;
-        if (!(is_v ? queue[s].read(qj[s], abort_flag, &id, false) : queue[s].claim(qj[s], p, abort_flag, &id))) {
+        if (!(is_v ? queue[s].read(qj[s], abort_flag, &id, false, p.wait_clocks) : queue[s].claim(qj[s], p, abort_flag, &id))) {
           ok = false;
           return false;
         }
@@ -372,42 +394,46 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < 2; ++s) {
         if (ok && have[s]) {
           const int stage = q % C::kStages;
-          SPARK_TC_T0(t_ew);
           if (q >= (uint32_t)C::kStages &&
-              !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag)) {
+              !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag, p.wait_clocks)) {
             ok = false;
           } else {
-            SPARK_TC_ACC(4, t_ew);
             const TcItem& I = cur[s];
-            int y[2], pooled[2];
+            int y[2], src[2];  // src: 0 K/V, 1 pooled pack, 2 extra pack
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
               int hi = 2 * t[s] + hf;
               if (hi >= I.nhalf) hi = 2 * t[s];  // a missing second half repeats the first (masked)
               const int bsel = __shfl_sync(0xffffffffu, ic[s], hi & 31);
-              pooled[hf] = 0;
+              src[hf] = 0;
               if (I.dense) {
                 y[hf] = I.bh * p.N + hi * kBlock;
               } else if (hi < I.cnt) {
                 y[hf] = I.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
               } else if (hi < I.cnt + n_dk) {
                 y[hf] = I.bh * p.N + nv + (hi - I.cnt) * kBlock;
+              } else if (hi < I.cnt + n_dk + p.n_xh) {
+                src[hf] = 2;
+                y[hf] = I.bh * p.ep + (hi - I.cnt - n_dk) * kBlock;
               } else {
                 // pooled entries past nb read rows of the next head (or TMA zero fill);
                 // their bias is -inf, so they carry no weight
-                pooled[hf] = 1;
-                y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk) * kBlock;
+                src[hf] = 1;
+                y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk - p.n_xh) * kBlock;
               }
             }
-            if (lane == 0) {
-              unsigned char* st = rbase + stage * C::kTileBytes;
-              tc::mbar_expect_tx(&full[stage], C::kTileBytes);
-#pragma unroll
-              for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-                for (int pn = 0; pn < C::kPanels; ++pn)
-                  tc::tma_load_2d(st + pn * C::kPanelBytes + hf * C::kHalfBytes,
-                                  pooled[hf] ? map_p : map_x, pn * 64, y[hf], &full[stage]);
+            // one box per lane (lanes 0 .. 2 kPanels - 1): TMA issue throughput is per
+            // issuing lane and warp, so spreading a tile's boxes over lanes raises the
+            // delivery rate (measured on this SM: 22 B/clk with one lane, 31 with four)
+            unsigned char* st = rbase + stage * C::kTileBytes;
+            if (lane == 0) tc::mbar_expect_tx(&full[stage], C::kTileBytes);
+            __syncwarp();
+            if (lane < 2 * C::kPanels) {
+              const int hf = lane / C::kPanels, pn = lane % C::kPanels;
+              const int sk = hf ? src[1] : src[0];
+              tc::tma_load_2d(st + pn * C::kPanelBytes + hf * C::kHalfBytes,
+                              sk == 1 ? map_p : (sk == 2 ? map_e : map_x), pn * 64, hf ? y[1] : y[0],
+                              &full[stage]);
             }
             __syncwarp();
             ++q;
@@ -449,7 +475,7 @@ __global__ void __launch_bounds__(384, 1)
       auto next_nonempty = [&](int o, TcItem* I) -> bool {
         while (true) {
           int id;
-          if (!queue[o].read(qj[o], abort_flag, &id, true)) {
+          if (!queue[o].read(qj[o], abort_flag, &id, true, p.wait_clocks)) {
             ok = false;
             return false;
           }
@@ -473,17 +499,10 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t vring_addr = tc::smem_addr(vring);
       auto issue_pv = [&]() -> bool {
         const uint32_t b = pg & 1;
-        SPARK_TC_T0(t_pw);
-        if (!tc::mbar_wait(&pfull[2 * s + b], (pg >> 1) & 1, abort_flag)) return false;
-        SPARK_TC_ACC(0, t_pw);
+        if (!tc::mbar_wait(&pfull[2 * s + b], (pg >> 1) & 1, abort_flag, p.wait_clocks)) return false;
         const int stage = pq % C::kStages;
-        SPARK_TC_T0(t_vw);
-        if (!tc::mbar_wait(&vfull[stage], (pq / C::kStages) & 1, abort_flag)) return false;
-        SPARK_TC_ACC(1, t_vw);
-        SPARK_TC_T0(t_ow);
-        if (pfirst && pitem > 0 && !tc::mbar_wait(&ofree[s], (pitem - 1) & 1, abort_flag)) return false;
-        SPARK_TC_ACC(9, t_ow);
-        SPARK_TC_T0(t_pv);
+        if (!tc::mbar_wait(&vfull[stage], (pq / C::kStages) & 1, abort_flag, p.wait_clocks)) return false;
+        if (pfirst && pitem > 0 && !tc::mbar_wait(&ofree[s], (pitem - 1) & 1, abort_flag, p.wait_clocks)) return false;
         tc::tc_fence_after();
         const uint32_t st = vring_addr + stage * C::kTileBytes;
 #pragma unroll
@@ -493,7 +512,6 @@ __global__ void __launch_bounds__(384, 1)
         tc::mma_commit(&vempty[stage]);
         tc::mma_commit(&oready[s]);
         if (plast) tc::mma_commit(&odone[s]);
-        SPARK_TC_ACC(10, t_pv);
         return true;
       };
       uint32_t q = 0;  // ring position of the producers' next tile
@@ -503,17 +521,12 @@ __global__ void __launch_bounds__(384, 1)
           if (ok && have[o]) {
             if (o == s) {
               const uint32_t qb = nitem & 1;
-              SPARK_TC_T0(t_qw);
-              bool good = t[o] != 0 || tc::mbar_wait(&qfull[2 * s + qb], (nitem >> 1) & 1, abort_flag);
-              SPARK_TC_ACC(3, t_qw);
+              bool good = t[o] != 0 || tc::mbar_wait(&qfull[2 * s + qb], (nitem >> 1) & 1, abort_flag, p.wait_clocks);
               const int stage = q % C::kStages;
-              SPARK_TC_T0(t_kw);
-              good = good && tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag);
-              SPARK_TC_ACC(2, t_kw);
+              good = good && tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag, p.wait_clocks);
               if (!good) {
                 ok = false;
               } else {
-                SPARK_TC_T0(t_si);
                 tc::tc_fence_after();
                 const uint32_t b = g & 1;
                 const uint32_t st = ring_addr + stage * C::kTileBytes;
@@ -524,7 +537,6 @@ __global__ void __launch_bounds__(384, 1)
                              tc_kdesc<D>(st, kk), idS, kk > 0 ? 1u : 0u);
                 tc::mma_commit(&sfull[2 * s + b]);
                 tc::mma_commit(&kempty[stage]);
-                SPARK_TC_ACC(11, t_si);
                 // then the PV of the previous tile of this slot
                 if (pend) ok = issue_pv();
                 pend = true;
@@ -598,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&qfull[2 * s + qb]);
       }
-      if (!J.dense && (p.pooled || J.cnt > 0)) {
+      if (!J.dense && (p.pooled || J.cnt > 0 || p.n_xh > 0)) {
         uint32_t* bm = bm2 + qb * nbwp;
         for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
         __syncwarp();
@@ -633,7 +645,7 @@ __global__ void __launch_bounds__(384, 1)
     auto epilogue = [&](const TcItem& I, float m_run, float l_run) -> bool {
       // odone completes once per item, after its last PV; it cannot run an item ahead
       // because the next item's PVs need this slot's P tiles.
-      if (!tc::mbar_wait(&odone[s], ndone & 1, abort_flag)) return false;
+      if (!tc::mbar_wait(&odone[s], ndone & 1, abort_flag, p.wait_clocks)) return false;
       ++ndone;
       tc::tc_fence_after();
       uint32_t o[D / 2];
@@ -679,7 +691,7 @@ __global__ void __launch_bounds__(384, 1)
     auto next_item = [&](TcItem* I) -> bool {
       while (true) {
         int id;
-        if (!queue[s].read(qj, abort_flag, &id, false)) {
+        if (!queue[s].read(qj, abort_flag, &id, false, p.wait_clocks)) {
           ok = false;
           return false;
         }
@@ -727,23 +739,18 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t b = g & 1;
         // warm L1 with the biases of a pooled half (their loads follow the S wait)
         const int hi = 2 * t + h;
-        const int kind = tc_half_kind(I, hi, n_dk);
+        const int kind = tc_half_kind(I, hi, n_dk, p.n_xh);
         const float* bias_src =
-            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk) * kBlock : 0);
+            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk - p.n_xh) * kBlock : 0);
         if (kind == kHalfPooled && lh < 2) prefetch_l1(bias_src + 32 * lh);
-        SPARK_TC_T0(t_sw);
-        if (!tc::mbar_wait(&sfull[2 * s + b], (g >> 1) & 1, abort_flag)) {
+        if (!tc::mbar_wait(&sfull[2 * s + b], (g >> 1) & 1, abort_flag, p.wait_clocks)) {
           ok = false;
           break;
         }
-        SPARK_TC_ACC(5, t_sw);
         tc::tc_fence_after();
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h+63 of the S buffer)
         float x[64];
-        SPARK_TC_T0(t_ld);
         tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, reinterpret_cast<uint32_t*>(x));
-        SPARK_TC_ACC(6, t_ld);
-        SPARK_TC_T0(t_cp);
         // ---- logits (base 2) and masks of this half
         // Exact and dense halves keep raw scores (the scale is folded into the exponent's
         // FFMA); pooled halves become scale*logit + beta*log2(e), with the selected blocks
@@ -755,7 +762,7 @@ __global__ void __launch_bounds__(384, 1)
           } else if (kind == kHalfDense) {
             const int key0 = I.dense ? hi * kBlock : nv + (hi - I.cnt) * kBlock;
             valid = min(kBlock, p.N - key0);
-          } else if (cur_bad) {
+          } else if (kind == kHalfExact && cur_bad) {
             const int bb = p.idx[I.row * (size_t)p.kcap + hi];
             if (bb < 0 || bb >= p.nb) valid = 0;
           }
@@ -764,10 +771,12 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = 0; j < 64; ++j)
               if (j >= valid) x[j] = -INFINITY;
           }
+          if (kind == kHalfExtra)
+            tc_mask_extra(x, p.xidx + (size_t)I.bh * p.ep, (hi - I.cnt - n_dk) * kBlock, p.n_extra, bm);
         }
         if (kind == kHalfPooled) {
           const float4* bsrc = reinterpret_cast<const float4*>(bias_src);
-          const int j0 = (hi - I.cnt - n_dk) * kBlock;
+          const int j0 = (hi - I.cnt - n_dk - p.n_xh) * kBlock;
           const int wb = j0 >> 5;  // j0 is a multiple of 64, wb + 1 < nbwp
           const uint32_t w0 = bm[wb], w1 = bm[wb + 1];
 #pragma unroll
@@ -788,8 +797,6 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         const float xs = kind == kHalfPooled ? 1.0f : p.scale_log2;  // factor still to apply
-        SPARK_TC_ACC(14 + (kind == kHalfPooled), t_cp);
-        SPARK_TC_T0(t_mx);
         // row max: 3-input max tree over this thread's 64 keys, then the partner half
         float mx;
         {
@@ -809,7 +816,7 @@ __global__ void __launch_bounds__(384, 1)
         const float alpha = need ? ex2f(m_run - m_new) : 1.0f;
         if (__any_sync(0xffffffffu, need && t > 0)) {
           // rescale the O rows of this warp once the previous PV has landed
-          if (!tc::mbar_wait(&oready[s], (g - 1) & 1, abort_flag)) {
+          if (!tc::mbar_wait(&oready[s], (g - 1) & 1, abort_flag, p.wait_clocks)) {
             ok = false;
             break;
           }
@@ -827,8 +834,6 @@ __global__ void __launch_bounds__(384, 1)
           l_run *= alpha;
           m_run = m_new;
         }
-        SPARK_TC_ACC(16, t_mx);
-        SPARK_TC_T0(t_ex);
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
         // P over S (packed columns 32h .. 32h+31 of the buffer), 32 keys at a time
@@ -852,14 +857,10 @@ __global__ void __launch_bounds__(384, 1)
           ls[0] = l2[0].x; ls[1] = l2[0].y; ls[2] = l2[1].x; ls[3] = l2[1].y;
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        SPARK_TC_ACC(17, t_ex);
-        SPARK_TC_ACC(7, t_cp);
-        SPARK_TC_T0(t_st);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&pfull[2 * s + b]);
-        SPARK_TC_ACC(8, t_st);
         // ---- the previous item's epilogue, once this item's first P is on its way
         if (t == 0 && have_prev) {
           if (!epilogue(prev, m_prev, l_prev)) {
@@ -884,7 +885,6 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && have_prev) epilogue(prev, m_prev, l_prev);
   }
 
-  SPARK_TC_FLUSH
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();

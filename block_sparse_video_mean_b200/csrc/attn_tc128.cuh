@@ -81,7 +81,7 @@ __device__ __forceinline__ TcItem tc128_item(const TcParams& p, int it) {
     int c = p.cnt[r.row];
     c = c < 0 ? 0 : (c > p.kcap ? p.kcap : c);
     r.cnt = c;
-    r.nhalf = c + n_dk + (p.pooled ? p.nbp / kBlock : 0);
+    r.nhalf = c + n_dk + p.n_xh + (p.pooled ? p.nbp / kBlock : 0);
     r.nq = min(128, nv - r.q0);
   }
   r.ntiles = (r.nhalf + 1) / 2;
@@ -151,6 +151,8 @@ __global__ void __launch_bounds__(384, 1)
     tc::tma_prefetch_desc(&maps.v);
     tc::tma_prefetch_desc(&maps.kp);
     tc::tma_prefetch_desc(&maps.vp);
+    tc::tma_prefetch_desc(&maps.kx);
+    tc::tma_prefetch_desc(&maps.vx);
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -172,6 +174,7 @@ __global__ void __launch_bounds__(384, 1)
     unsigned char* rbase = is_v ? vring : ring;
     const CUtensorMap* map_x = is_v ? &maps.v : &maps.k;
     const CUtensorMap* map_p = is_v ? &maps.vp : &maps.kp;
+    const CUtensorMap* map_e = is_v ? &maps.vx : &maps.kx;
     // The whole warp walks the tile sequence (warp 8 claims the items, warp 10 reads
     // them from the queue); the selected block indices are fetched 32 halves at a time,
     // one chunk ahead.
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(384, 1)
     auto take_nonempty = [&](TcItem* I) -> bool {
       while (true) {
         int id;
-        if (!(is_v ? queue.read(qj, abort_flag, &id, false) : queue.claim(qj, p, abort_flag, &id))) {
+        if (!(is_v ? queue.read(qj, abort_flag, &id, false, p.wait_clocks) : queue.claim(qj, p, abort_flag, &id))) {
           ok = false;
           return false;
         }
@@ -218,39 +221,42 @@ __global__ void __launch_bounds__(384, 1)
     while (ok && have) {
       const int stage = q % C::kStages;
       if (q >= (uint32_t)C::kStages &&
-          !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag)) {
+          !tc::mbar_wait(&empty[stage], ((q / C::kStages) - 1) & 1, abort_flag, p.wait_clocks)) {
         ok = false;
         break;
       }
-      int y[2], pooled[2];
+      int y[2], src[2];  // src: 0 K/V, 1 pooled pack, 2 extra pack
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         int hi = 2 * t + hf;
         if (hi >= cur.nhalf) hi = 2 * t;  // a missing second half repeats the first (masked)
         const int bsel = __shfl_sync(0xffffffffu, ic, hi & 31);
-        pooled[hf] = 0;
+        src[hf] = 0;
         if (cur.dense) {
           y[hf] = cur.bh * p.N + hi * kBlock;
         } else if (hi < cur.cnt) {
           y[hf] = cur.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
         } else if (hi < cur.cnt + n_dk) {
           y[hf] = cur.bh * p.N + nv + (hi - cur.cnt) * kBlock;
+        } else if (hi < cur.cnt + n_dk + p.n_xh) {
+          src[hf] = 2;
+          y[hf] = cur.bh * p.ep + (hi - cur.cnt - n_dk) * kBlock;
         } else {
           // pooled entries past nb read rows of the next head (or TMA zero fill); their
           // bias is -inf, so they carry no weight
-          pooled[hf] = 1;
-          y[hf] = cur.bh * p.nb + (hi - cur.cnt - n_dk) * kBlock;
+          src[hf] = 1;
+          y[hf] = cur.bh * p.nb + (hi - cur.cnt - n_dk - p.n_xh) * kBlock;
         }
       }
-      if (lane == 0) {
-        unsigned char* st = rbase + stage * C::kTileBytes;
-        tc::mbar_expect_tx(&full[stage], C::kTileBytes);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn)
-            tc::tma_load_2d(st + pn * TcCfg<D>::kPanelBytes + hf * C::kHalfBytes,
-                            pooled[hf] ? map_p : map_x, pn * 64, y[hf], &full[stage]);
+      // one box per lane: TMA issue throughput is per issuing lane and warp
+      unsigned char* st = rbase + stage * C::kTileBytes;
+      if (lane == 0) tc::mbar_expect_tx(&full[stage], C::kTileBytes);
+      __syncwarp();
+      if (lane < 2 * C::kPanels) {
+        const int hf = lane / C::kPanels, pn = lane % C::kPanels;
+        const int sk = hf ? src[1] : src[0];
+        tc::tma_load_2d(st + pn * TcCfg<D>::kPanelBytes + hf * C::kHalfBytes,
+                        sk == 1 ? map_p : (sk == 2 ? map_e : map_x), pn * 64, hf ? y[1] : y[0], &full[stage]);
       }
       __syncwarp();
       ++q;
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(384, 1)
       auto next_nonempty = [&](TcItem* I) -> bool {
         while (true) {
           int id;
-          if (!queue.read(qj, abort_flag, &id, true)) {
+          if (!queue.read(qj, abort_flag, &id, true, p.wait_clocks)) {
             ok = false;
             return false;
           }
@@ -306,10 +312,10 @@ __global__ void __launch_bounds__(384, 1)
         const int stage = g % C::kStages;
         if (!is_pv) {
           const uint32_t qb = nitem & 1;
-          bool good = t != 0 || tc::mbar_wait(&qfull[qb], (nitem >> 1) & 1, abort_flag);
-          good = good && tc::mbar_wait(&kfull[stage], (g / C::kStages) & 1, abort_flag);
+          bool good = t != 0 || tc::mbar_wait(&qfull[qb], (nitem >> 1) & 1, abort_flag, p.wait_clocks);
+          good = good && tc::mbar_wait(&kfull[stage], (g / C::kStages) & 1, abort_flag, p.wait_clocks);
           // S buffer b is free once the PV of tile g - 2 (its P) completed
-          good = good && (g < 2 || tc::mbar_wait(&sfree[b], ((g >> 1) - 1) & 1, abort_flag));
+          good = good && (g < 2 || tc::mbar_wait(&sfree[b], ((g >> 1) - 1) & 1, abort_flag, p.wait_clocks));
           if (!good) {
             ok = false;
             break;
@@ -324,10 +330,10 @@ __global__ void __launch_bounds__(384, 1)
           tc::mma_commit(&sfull[b]);
           tc::mma_commit(&kempty[stage]);
         } else {
-          bool good = tc::mbar_wait(&pfull[b], (g >> 1) & 1, abort_flag);
-          good = good && tc::mbar_wait(&vfull[stage], (g / C::kStages) & 1, abort_flag);
+          bool good = tc::mbar_wait(&pfull[b], (g >> 1) & 1, abort_flag, p.wait_clocks);
+          good = good && tc::mbar_wait(&vfull[stage], (g / C::kStages) & 1, abort_flag, p.wait_clocks);
           // the first PV of an item overwrites O: the previous item's epilogue read it
-          if (good && t == 0 && nitem > 0) good = tc::mbar_wait(ofree, (nitem - 1) & 1, abort_flag);
+          if (good && t == 0 && nitem > 0) good = tc::mbar_wait(ofree, (nitem - 1) & 1, abort_flag, p.wait_clocks);
           if (!good) {
             ok = false;
             break;
@@ -391,7 +397,7 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&qfull[qb]);
       }
-      if (!J.dense && (p.pooled || J.cnt > 0)) {
+      if (!J.dense && (p.pooled || J.cnt > 0 || p.n_xh > 0)) {
         uint32_t* bm = bm2 + qb * nbwp;
         for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
         __syncwarp();
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(384, 1)
 
     uint32_t ndone = 0;  // non-empty items whose epilogue ran
     auto epilogue = [&](const TcItem& I, float m_run, float l_run) -> bool {
-      if (!tc::mbar_wait(odone, ndone & 1, abort_flag)) return false;
+      if (!tc::mbar_wait(odone, ndone & 1, abort_flag, p.wait_clocks)) return false;
       tc::tc_fence_after();
       uint32_t o[D / 2];
       if constexpr (D == 128)
@@ -469,7 +475,7 @@ __global__ void __launch_bounds__(384, 1)
     auto next_item = [&](TcItem* I) -> bool {
       while (true) {
         int id;
-        if (!queue.read(qj, abort_flag, &id, false)) {
+        if (!queue.read(qj, abort_flag, &id, false, p.wait_clocks)) {
           ok = false;
           return false;
         }
@@ -517,11 +523,11 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t b = g & 1;
         // warm L1 with the biases of a pooled half (their loads follow the S wait)
         const int hi = 2 * t + h;
-        const int kind = tc_half_kind(I, hi, n_dk);
+        const int kind = tc_half_kind(I, hi, n_dk, p.n_xh);
         const float* bias_src =
-            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk) * kBlock : 0);
+            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk - p.n_xh) * kBlock : 0);
         if (kind == kHalfPooled && lane < 2) prefetch_l1(bias_src + 32 * lane);
-        if (!tc::mbar_wait(&sfull[b], (g >> 1) & 1, abort_flag)) {
+        if (!tc::mbar_wait(&sfull[b], (g >> 1) & 1, abort_flag, p.wait_clocks)) {
           ok = false;
           break;
         }
@@ -537,7 +543,7 @@ __global__ void __launch_bounds__(384, 1)
           } else if (kind == kHalfDense) {
             const int key0 = I.dense ? hi * kBlock : nv + (hi - I.cnt) * kBlock;
             valid = min(kBlock, p.N - key0);
-          } else if (cur_bad) {
+          } else if (kind == kHalfExact && cur_bad) {
             const int bb = p.idx[I.row * (size_t)p.kcap + hi];
             if (bb < 0 || bb >= p.nb) valid = 0;
           }
@@ -546,9 +552,11 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = 0; j < 64; ++j)
               if (j >= valid) x[j] = -INFINITY;
           }
+          if (kind == kHalfExtra)
+            tc_mask_extra(x, p.xidx + (size_t)I.bh * p.ep, (hi - I.cnt - n_dk) * kBlock, p.n_extra, bm);
         } else {
           const float4* bsrc = reinterpret_cast<const float4*>(bias_src);
-          const int j0 = (hi - I.cnt - n_dk) * kBlock;
+          const int j0 = (hi - I.cnt - n_dk - p.n_xh) * kBlock;
           const int wb = j0 >> 5;  // j0 is a multiple of 64, wb + 1 < nbwp
           const uint32_t w0 = bm[wb], w1 = bm[wb + 1];
 #pragma unroll
@@ -611,7 +619,7 @@ __global__ void __launch_bounds__(384, 1)
           const float alpha = need ? ex2f(m_run - m_new) : 1.0f;
           if (t > 0) {
             // rescale this thread's half of its O row once the previous PV has landed
-            if (!tc::mbar_wait(oready, (g - 1) & 1, abort_flag)) {
+            if (!tc::mbar_wait(oready, (g - 1) & 1, abort_flag, p.wait_clocks)) {
               ok = false;
               break;
             }

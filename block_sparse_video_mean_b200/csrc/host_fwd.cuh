@@ -21,7 +21,7 @@ struct HostPlan {
   size_t head_x = 0;    // elements of one head's Q (or K, V, O): N * d
   size_t slot_q[2], slot_k[2], slot_v[2], slot_o[2], slot_lse[2];
   size_t q_pool, k_pool, v_summ, beta, anchor, pack, pack_bytes, idx, cnt, sel, sel_bytes, attn,
-      attn_bytes, perm, perm_k, qp, kp, vp, rb, rb_bytes;
+      attn_bytes, perm, perm_k, qp, kp, vp, rb, rb_bytes, extra, extra_bytes;
   size_t total = 0;
 };
 
@@ -41,6 +41,7 @@ int host_plan(const spark_shape* s, const spark_fwd_config* c, HostPlan* p) {
     return SPARK_EINVAL;
   if (c->pool_mode != SPARK_POOL_REWEIGHT && c->pool_mode != SPARK_POOL_MEAN) return SPARK_EINVAL;
   if (c->reblock < 0 || c->reblock > 2) return SPARK_EINVAL;
+  if (c->extra_tokens < 0) return SPARK_EINVAL;
   if (!std::isfinite(c->param)) return SPARK_EINVAL;
   p->bh = (int64_t)s->B * s->H;
   p->nb = (int)num_blocks(s);
@@ -90,6 +91,8 @@ int host_plan(const spark_shape* s, const spark_fwd_config* c, HostPlan* p) {
   p->sel = take(p->sel_bytes);
   p->attn_bytes = spark_workspace_bytes(&g, SPARK_CALL_ATTN);
   p->attn = take(p->attn_bytes);
+  p->extra_bytes = spark_extra_pack_bytes(&g, c->extra_tokens);
+  p->extra = p->extra_bytes ? take(p->extra_bytes) : 0;
   p->perm = p->perm_k = p->qp = p->kp = p->vp = p->rb = p->rb_bytes = 0;
   if (c->reblock != 0) {
     p->perm = take(Gs * p->nb * kBlock * 4);
@@ -134,15 +137,21 @@ int host_group(const spark_shape* g, const spark_fwd_config* c, const HostPlan& 
                      static_cast<float*>(at(p.beta)), static_cast<float*>(at(p.anchor)),
                      at(p.pack), p.pack_bytes, cs);
   if (st != SPARK_OK) return st;
+  if (p.extra_bytes > 0) {
+    st = spark_extra_tokens(g, K, V, static_cast<const float*>(at(p.anchor)), c->extra_tokens, c->pool_mode,
+                            static_cast<float*>(at(p.v_summ)), static_cast<float*>(at(p.beta)), at(p.pack),
+                            p.pack_bytes, at(p.extra), p.extra_bytes, cs);
+    if (st != SPARK_OK) return st;
+  }
   int32_t* idx = static_cast<int32_t*>(at(p.idx));
   int32_t* cnt = static_cast<int32_t*>(at(p.cnt));
   st = spark_score_select(g, q_pool, k_pool, c->select_mode, c->param, p.kcap, idx, cnt, at(p.sel),
                           p.sel_bytes, cs);
   if (st != SPARK_OK) return st;
   return spark_attn_fwd(g, Q, K, V, idx, cnt, p.kcap, c->compressed ? at(p.pack) : nullptr,
-                        static_cast<const float*>(at(p.beta)), perm,
-                        static_cast<uint16_t*>(at(p.slot_o[k])), static_cast<float*>(at(p.slot_lse[k])),
-                        at(p.attn), p.attn_bytes, cs);
+                        static_cast<const float*>(at(p.beta)), perm, p.extra_bytes ? at(p.extra) : nullptr,
+                        p.extra_bytes ? c->extra_tokens : 0, static_cast<uint16_t*>(at(p.slot_o[k])),
+                        static_cast<float*>(at(p.slot_lse[k])), at(p.attn), p.attn_bytes, cs);
 }
 
 }  // namespace

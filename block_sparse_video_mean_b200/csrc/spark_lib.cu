@@ -10,6 +10,7 @@
 
 #include "spark_common.cuh"
 #include "pool.cuh"
+#include "extra.cuh"
 #include "select.cuh"
 #include "attn_tc.cuh"
 #include "attn_tc128.cuh"
@@ -106,6 +107,9 @@ bool bf16_tile_map(CUtensorMap* m, const void* base, uint64_t rows, int d) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Limit of the attention kernels' pipeline waits, in SM clocks (spark_set_wait_limit).
+std::atomic<long long> g_wait_limit{tc::kWaitClocks};
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -115,7 +119,7 @@ int num_sms() {
 
 template <int D, bool Q128>
 int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, const void* pack,
-                   cudaStream_t cs) {
+                   const uint16_t* kx, const uint16_t* vx, cudaStream_t cs) {
   TcMaps maps;
   const uint64_t rows = (uint64_t)tp.BH * tp.N;
   if (!bf16_tile_map(&maps.k, K, rows, D) || !bf16_tile_map(&maps.v, V, rows, D)) return SPARK_ECUDA;
@@ -127,6 +131,13 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
   } else {
     maps.kp = maps.k;
     maps.vp = maps.v;
+  }
+  if (tp.n_xh > 0) {
+    const uint64_t xrow = (uint64_t)tp.BH * tp.ep;
+    if (!bf16_tile_map(&maps.kx, kx, xrow, D) || !bf16_tile_map(&maps.vx, vx, xrow, D)) return SPARK_ECUDA;
+  } else {
+    maps.kx = maps.k;
+    maps.vx = maps.v;
   }
   const size_t smem = Q128 ? tc128_smem_bytes<D>(tp.nb) : tc_smem_bytes<D>(tp.nb);
   if (smem > 227 * 1024) return SPARK_EUNSUPPORTED;
@@ -144,25 +155,58 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
 }
 
 // Scratch of spark_score_select_noalloc: a file-scope device array (no allocation). In
-// host code its name is only a stand-in, so its device address is looked up per device.
+// host code its name is only a stand-in, so its device address is looked up per device
+// (with that device current) and cached together with the unique ID of the context it
+// belongs to: a device reset replaces the primary context, the module is loaded again,
+// possibly elsewhere, and the next call looks the address up anew.
 __device__ __align__(256) double g_noalloc_select_scratch[2 * SPARK_NOALLOC_MAX_HEADS];
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[128] = {};
+struct NoallocSlot {
+  void* ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+NoallocSlot g_noalloc[128];
+
+// Unique ID of the context current on this thread (0 if none is current yet).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPARK_ECUDA;
   if (dev < 0 || dev >= 128) return SPARK_EUNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocSlot& slot = g_noalloc[dev];
+  const unsigned long long id = current_context_id();
+  if (slot.ptr == nullptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_select_scratch) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
       return SPARK_ECUDA;
     }
-    g_noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_context_id();  // the lookup made the device's context current
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return SPARK_OK;
 }
 
@@ -254,6 +298,73 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
   }
   SPARK_LAUNCH_CHECK();
   note_launches(3);
+  return SPARK_OK;
+}
+
+size_t spark_extra_pack_bytes(const spark_shape* s, int32_t extra_tokens) {
+  if (check_shape(s) != SPARK_OK || extra_tokens <= 0) return 0;
+  const int nb = (int)num_blocks(s);
+  if (nb == 0) return 0;
+  return extra_layout((size_t)s->B * s->H, nb * kBlock, s->d, extra_tokens).total;
+}
+
+int spark_extra_tokens(const spark_shape* s, const uint16_t* K, const uint16_t* V, const float* anchor,
+                       int32_t extra_tokens, int pool_mode, float* v_summ, float* beta, void* pool_pack,
+                       size_t pool_pack_bytes, void* extra_pack, size_t extra_pack_bytes, void* stream) {
+  int st = check_shape(s);
+  if (st != SPARK_OK) return st;
+  if (extra_tokens < 0) return SPARK_EINVAL;
+  if (pool_mode != SPARK_POOL_REWEIGHT && pool_mode != SPARK_POOL_MEAN) return SPARK_EINVAL;
+  const int nb = (int)num_blocks(s);
+  if (empty(s) || nb == 0 || extra_tokens == 0) return SPARK_OK;
+  const size_t bh = (size_t)s->B * s->H;
+  const int nv = nb * kBlock;
+  if (!K || !V || !anchor || !extra_pack) return SPARK_EINVAL;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(anchor) || !aligned16(extra_pack)) return SPARK_EINVAL;
+  const ExtraLayout xl = extra_layout(bh, nv, s->d, extra_tokens);
+  if (extra_pack_bytes < xl.total) return SPARK_EINVAL;
+  if (pool_pack != nullptr) {
+    if (!aligned16(pool_pack) || pool_pack_bytes < spark_workspace_bytes(s, SPARK_CALL_POOL)) return SPARK_EINVAL;
+    if ((v_summ && !aligned16(v_summ)) || (beta && !aligned16(beta))) return SPARK_EINVAL;
+  }
+  unsigned char* xb = static_cast<unsigned char*>(extra_pack);
+  int32_t* xidx = reinterpret_cast<int32_t*>(xb + xl.xidx);
+  float* scores = reinterpret_cast<float*>(xb + xl.scores);
+  uint16_t* kx = reinterpret_cast<uint16_t*>(xb + xl.k);
+  uint16_t* vx = reinterpret_cast<uint16_t*>(xb + xl.v);
+  const float scale = eff_scale(s);
+  cudaStream_t cs = as_stream(stream);
+  const dim3 gs((nb + kPoolWarps - 1) / kPoolWarps, (unsigned)bh);
+  const dim3 gg(xl.ep / 8, (unsigned)bh);
+  const dim3 gf((xl.ne + kPoolWarps - 1) / kPoolWarps, (unsigned)bh);
+  uint16_t* k16 = static_cast<uint16_t*>(pool_pack);
+  uint16_t* v16 = k16 ? k16 + bh * nb * s->d : nullptr;
+  float* bl2 = pool_pack ? reinterpret_cast<float*>(static_cast<unsigned char*>(pool_pack) +
+                                                    pack_bias_offset(bh, nb, s->d))
+                         : nullptr;
+  const int nbp = (int)padded_blocks(nb);
+  int launches = 3;
+  if (s->d == 128) {
+    extra_scores_kernel<128><<<gs, kPoolWarps * 32, 0, cs>>>(K, anchor, scores, s->N, nb, scale);
+    extra_select_kernel<<<(unsigned)bh, kExtraThreads, 0, cs>>>(scores, nv, xl.ne, xl.ep, xidx);
+    extra_gather_kernel<128><<<gg, 256, 0, cs>>>(K, V, xidx, s->N, nv, xl.ep, kx, vx);
+    if (pool_pack) {
+      extra_fixup_kernel<128><<<gf, kPoolWarps * 32, 0, cs>>>(K, V, anchor, scores, xidx, s->N, nb, xl.ne, xl.ep,
+                                                              scale, pool_mode, v_summ, beta, k16, v16, bl2, nbp);
+      ++launches;
+    }
+  } else {
+    extra_scores_kernel<64><<<gs, kPoolWarps * 32, 0, cs>>>(K, anchor, scores, s->N, nb, scale);
+    extra_select_kernel<<<(unsigned)bh, kExtraThreads, 0, cs>>>(scores, nv, xl.ne, xl.ep, xidx);
+    extra_gather_kernel<64><<<gg, 256, 0, cs>>>(K, V, xidx, s->N, nv, xl.ep, kx, vx);
+    if (pool_pack) {
+      extra_fixup_kernel<64><<<gf, kPoolWarps * 32, 0, cs>>>(K, V, anchor, scores, xidx, s->N, nb, xl.ne, xl.ep,
+                                                             scale, pool_mode, v_summ, beta, k16, v16, bl2, nbp);
+      ++launches;
+    }
+  }
+  SPARK_LAUNCH_CHECK();
+  note_launches(launches);
   return SPARK_OK;
 }
 
@@ -378,10 +489,11 @@ int spark_score_select_noalloc(const spark_shape* s, const float* q_pool, const 
 
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
-                   const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,
-                   size_t ws_bytes, void* stream) {
+                   const float* beta, const int32_t* perm, const void* extra_pack, int32_t extra_tokens,
+                   uint16_t* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
+  if (extra_tokens < 0) return SPARK_EINVAL;
   if (empty(s)) return SPARK_OK;
   if (!ws || ws_bytes < spark_workspace_bytes(s, SPARK_CALL_ATTN) || !aligned16(ws)) return SPARK_EINVAL;
   const int nb = (int)num_blocks(s);
@@ -422,12 +534,31 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
   tp.n_items = (int)items;
   tp.scale_log2 = eff_scale(s) * kLog2e;
   tp.item_ctr = static_cast<int*>(ws);
+  tp.wait_clocks = g_wait_limit.load(std::memory_order_relaxed);
+  tp.xidx = nullptr;
+  tp.n_xh = tp.n_extra = tp.ep = 0;
+  const uint16_t* kx = nullptr;
+  const uint16_t* vx = nullptr;
+  if (extra_tokens > 0 && nb > 0) {
+    if (!extra_pack || !aligned16(extra_pack)) return SPARK_EINVAL;
+    const ExtraLayout xl = extra_layout((size_t)bh, nv, s->d, extra_tokens);
+    const unsigned char* xb = static_cast<const unsigned char*>(extra_pack);
+    tp.xidx = reinterpret_cast<const int32_t*>(xb + xl.xidx);
+    tp.n_xh = xl.ep / kBlock;
+    tp.n_extra = xl.ne;
+    tp.ep = xl.ep;
+    kx = reinterpret_cast<const uint16_t*>(xb + xl.k);
+    vx = reinterpret_cast<const uint16_t*>(xb + xl.v);
+    if ((int64_t)bh * xl.ep >= ((int64_t)1 << 31)) return SPARK_EUNSUPPORTED;
+  }
   cudaStream_t cs = as_stream(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(int), cs) != cudaSuccess) return SPARK_ECUDA;
   const void* pack = tp.pooled ? pool_pack : nullptr;
   if (qt == 2 * kBlock)
-    return s->d == 128 ? launch_attn_tc<128, true>(tp, K, V, pack, cs) : launch_attn_tc<64, true>(tp, K, V, pack, cs);
-  return s->d == 128 ? launch_attn_tc<128, false>(tp, K, V, pack, cs) : launch_attn_tc<64, false>(tp, K, V, pack, cs);
+    return s->d == 128 ? launch_attn_tc<128, true>(tp, K, V, pack, kx, vx, cs)
+                       : launch_attn_tc<64, true>(tp, K, V, pack, kx, vx, cs);
+  return s->d == 128 ? launch_attn_tc<128, false>(tp, K, V, pack, kx, vx, cs)
+                     : launch_attn_tc<64, false>(tp, K, V, pack, kx, vx, cs);
 }
 
 }  // extern "C"
@@ -485,6 +616,11 @@ int spark_device_error(int32_t* host_word, void* stream) {
 }
 
 uint64_t spark_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
+
+int spark_set_wait_limit(int64_t clocks) {
+  g_wait_limit.store(clocks > 0 ? (long long)clocks : tc::kWaitClocks, std::memory_order_relaxed);
+  return SPARK_OK;
+}
 
 const char* spark_strerror(int status) {
   switch (status) {

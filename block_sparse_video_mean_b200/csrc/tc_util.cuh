@@ -71,17 +71,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: gives up after ~2^31 clocks (about a second), records SPARK_ETIMEOUT and
-// raises the CTA's abort flag so every other role stops too. Returns false on give-up or
-// when another role already aborted.
+// Bounded wait: gives up after `limit` clocks (by default ~2^31, about a second), records
+// SPARK_ETIMEOUT and raises the CTA's abort flag so every other role stops too. Returns
+// false on give-up or when another role already aborted.
 constexpr long long kWaitClocks = 1ll << 31;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = kWaitClocks) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitClocks) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       set_error(SPARK_ETIMEOUT);
       return false;

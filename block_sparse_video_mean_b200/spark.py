@@ -29,7 +29,8 @@ BLOCK = 64
 EXPORTS = ("spark_num_blocks", "spark_workspace_bytes", "spark_topk_count", "spark_pool_kv",
            "spark_score_select", "spark_attn_fwd", "spark_reblock", "spark_device_error",
            "spark_strerror", "spark_score_select_noalloc", "spark_kernel_launches", "spark_reblock_kv",
-           "spark_num_query_tiles", "spark_forward_host", "spark_forward_host_workspace_bytes")
+           "spark_num_query_tiles", "spark_forward_host", "spark_forward_host_workspace_bytes",
+           "spark_set_wait_limit", "spark_extra_pack_bytes", "spark_extra_tokens")
 NOALLOC_MAX_HEADS = 4096
 
 
@@ -49,7 +50,7 @@ class FwdConfig(ctypes.Structure):
     _fields_ = [("param", ctypes.c_double), ("select_mode", ctypes.c_int32),
                 ("kcap", ctypes.c_int32), ("pool_mode", ctypes.c_int32),
                 ("compressed", ctypes.c_int32), ("reblock", ctypes.c_int32),
-                ("heads_per_group", ctypes.c_int32)]
+                ("heads_per_group", ctypes.c_int32), ("extra_tokens", ctypes.c_int32)]
 
 
 _lib = None
@@ -80,8 +81,13 @@ def load() -> ctypes.CDLL:
     lib.spark_score_select.restype = I
     lib.spark_score_select_noalloc.argtypes = [SP, P, P, I, D, ctypes.c_int32, P, P, P]
     lib.spark_score_select_noalloc.restype = I
-    lib.spark_attn_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_int32, P, P, P, P, P, P, Z, P]
+    lib.spark_attn_fwd.argtypes = [SP, P, P, P, P, P, ctypes.c_int32, P, P, P, P, ctypes.c_int32, P, P, P,
+                                   Z, P]
     lib.spark_attn_fwd.restype = I
+    lib.spark_extra_pack_bytes.argtypes = [SP, ctypes.c_int32]
+    lib.spark_extra_pack_bytes.restype = Z
+    lib.spark_extra_tokens.argtypes = [SP, P, P, P, ctypes.c_int32, I, P, P, P, Z, P, Z, P]
+    lib.spark_extra_tokens.restype = I
     lib.spark_reblock.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
     lib.spark_reblock.restype = I
     lib.spark_reblock_kv.argtypes = [SP, P, P, P, P, P, P, P, P, P, Z, P]
@@ -97,6 +103,8 @@ def load() -> ctypes.CDLL:
     lib.spark_strerror.restype = ctypes.c_char_p
     lib.spark_kernel_launches.argtypes = []
     lib.spark_kernel_launches.restype = ctypes.c_uint64
+    lib.spark_set_wait_limit.argtypes = [ctypes.c_int64]
+    lib.spark_set_wait_limit.restype = I
     _lib = lib
     return lib
 
@@ -142,6 +150,12 @@ def workspace_bytes(shape: Shape, call_id: int) -> int:
 def kernel_launches() -> int:
     """Kernels launched through the library by this process so far (host-side count)."""
     return int(load().spark_kernel_launches())
+
+
+def set_wait_limit(clocks: int = 0) -> None:
+    """Limit (SM clocks) of the attention kernels' pipeline waits for later launches;
+    0 restores the default (about a second)."""
+    _check(load().spark_set_wait_limit(int(clocks)), "spark_set_wait_limit")
 
 
 def device_error(device=None) -> int:
@@ -229,8 +243,40 @@ def score_select_noalloc(q_pool, k_pool, n_sink, N, mode, param, kcap=None, scal
     return idx, cnt
 
 
+def extra_pack_bytes(shape: Shape, extra_tokens: int) -> int:
+    return int(load().spark_extra_pack_bytes(ctypes.byref(shape), int(extra_tokens)))
+
+
+def extra_tokens(K, V, pool, n_sink, n_extra, pool_mode=POOL_REWEIGHT, scale=None, out=None, q_tile=BLOCK,
+                 compressed=True):
+    """spark_extra_tokens after pool_kv (``pool`` = its dict): returns the extra pack (uint8
+    device buffer). With ``compressed`` the pooled entries of the blocks that lost tokens
+    are rewritten in ``pool`` (pack, v_summ, beta)."""
+    for t, n in ((K, "K"), (V, "V")):
+        _need(t, n)
+    shape = _shape_of(K, n_sink, scale, q_tile)
+    dev = K.device
+    if out is None:
+        out = torch.empty(max(extra_pack_bytes(shape, n_extra), 16), dtype=torch.uint8, device=dev)
+    pack = pool["pack"] if compressed else None
+    _check(load().spark_extra_tokens(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(pool["anchor"]),
+                                     int(n_extra), int(pool_mode),
+                                     _ptr(pool["v_summ"]) if compressed else None,
+                                     _ptr(pool["beta"]) if compressed else None, _ptr(pack),
+                                     0 if pack is None else pack.numel(), _ptr(out), out.numel(),
+                                     _stream(dev)), "spark_extra_tokens")
+    return out
+
+
+def extra_token_rows(xpack, B, H, nb, n_extra):
+    """The extra token indices [B, H, E] (ascending) held in an extra pack."""
+    ne = min(int(n_extra), nb * BLOCK)
+    ep = (ne + BLOCK - 1) // BLOCK * BLOCK
+    return xpack[: B * H * ep * 4].view(torch.int32).view(B, H, ep)[:, :, :ne]
+
+
 def attn_fwd(Q, K, V, idx, cnt, n_sink, pack=None, beta=None, perm=None, scale=None,
-             out=None, lse=True, q_tile=BLOCK, ws=None):
+             out=None, lse=True, q_tile=BLOCK, ws=None, extra_pack=None, n_extra=0):
     """spark_attn_fwd: returns (O bf16 [B,H,N,d], LSE fp32 [B,H,N] or None)."""
     for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
         _need(t, n)
@@ -245,8 +291,9 @@ def attn_fwd(Q, K, V, idx, cnt, n_sink, pack=None, beta=None, perm=None, scale=N
     O, L = out
     kcap = idx.shape[-1] if idx is not None else 1
     _check(load().spark_attn_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
-                                 _ptr(cnt), int(kcap), _ptr(pack), _ptr(beta), _ptr(perm), _ptr(O),
-                                 _ptr(L), _ptr(ws), ws.numel(), _stream(dev)), "spark_attn_fwd")
+                                 _ptr(cnt), int(kcap), _ptr(pack), _ptr(beta), _ptr(perm),
+                                 _ptr(extra_pack), int(n_extra), _ptr(O), _ptr(L), _ptr(ws), ws.numel(),
+                                 _stream(dev)), "spark_attn_fwd")
     return O, L
 
 
@@ -295,10 +342,10 @@ def reblock_kv(Q, K, V, n_sink, out=None, ws=None):
 
 
 def fwd_config(mode=SELECT_TOPK_RATIO, param=0.1, kcap=0, pool_mode=POOL_REWEIGHT, compressed=True,
-               reblock=0, heads_per_group=0) -> FwdConfig:
+               reblock=0, heads_per_group=0, extra_tokens=0) -> FwdConfig:
     """spark_fwd_config of spark_forward_host (reblock: 0 none, 1 shared, 2 own key partition)."""
     return FwdConfig(float(param), int(mode), int(kcap or 0), int(pool_mode), int(bool(compressed)),
-                     int(reblock), int(heads_per_group or 0))
+                     int(reblock), int(heads_per_group or 0), int(extra_tokens or 0))
 
 
 def forward_host_workspace_bytes(shape: Shape, cfg: FwdConfig) -> int:
@@ -341,6 +388,7 @@ class ForwardConfig:
     scale: float | None = None
     kcap: int | None = None     # slots per selection row (default: k, or nb for tau)
     q_tile: int = BLOCK         # query tile: 64, or 128 (the 128-query x 64-key route)
+    extra_tokens: int = 0       # extra tokens per head added to the exact branch (0: none)
 
 
 class SparkAttention:
@@ -372,6 +420,10 @@ class SparkAttention:
         self.attn_ws = torch.empty(max(workspace_bytes(self.shape, CALL_ATTN), 16), dtype=torch.uint8, device=dev)
         self.O = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, H, N), **f32)
+        self.xpack = None
+        if cfg.extra_tokens > 0 and nb > 0:
+            self.xpack = torch.empty(max(extra_pack_bytes(self.shape, cfg.extra_tokens), 16),
+                                     dtype=torch.uint8, device=dev)
         self.rb = None
         if cfg.reblock:
             levels = 0 if nb <= 1 else math.ceil(math.log2(nb))
@@ -406,6 +458,9 @@ class SparkAttention:
             Q, K, V, perm = self.rb["Qp"], self.rb["Kp"], self.rb["Vp"], self.rb["perm"]
         mark(1)
         pool_kv(Q, K, V, self.n_sink, self.pool_mode, cfg.scale, out=self.pool, q_tile=cfg.q_tile)
+        if self.xpack is not None:
+            extra_tokens(K, V, self.pool, self.n_sink, cfg.extra_tokens, self.pool_mode, cfg.scale,
+                         out=self.xpack, q_tile=cfg.q_tile, compressed=cfg.compressed)
         mark(2)
         score_select(self.pool["q_pool"], self.pool["k_pool"], self.n_sink, Q.shape[2], self.mode,
                      cfg.param, self.kcap, cfg.scale, out=(self.idx, self.cnt), ws=self.sel_ws,
@@ -413,7 +468,8 @@ class SparkAttention:
         mark(3)
         attn_fwd(Q, K, V, self.idx, self.cnt, self.n_sink,
                  pack=self.pool["pack"] if cfg.compressed else None, beta=self.pool["beta"],
-                 perm=perm, scale=cfg.scale, out=(self.O, self.lse), q_tile=cfg.q_tile, ws=self.attn_ws)
+                 perm=perm, scale=cfg.scale, out=(self.O, self.lse), q_tile=cfg.q_tile, ws=self.attn_ws,
+                 extra_pack=self.xpack, n_extra=cfg.extra_tokens if self.xpack is not None else 0)
         mark(4)
         return self.O, self.lse
 
@@ -421,7 +477,7 @@ class SparkAttention:
         cfg = self.cfg
         rb = 0 if not cfg.reblock else (2 if cfg.reblock_kv else 1)
         return fwd_config(self.mode, cfg.param, self.kcap, self.pool_mode, cfg.compressed, rb,
-                          heads_per_group)
+                          heads_per_group, cfg.extra_tokens)
 
     def run_host(self, hQ, hK, hV, hO=None, hlse=None, heads_per_group=0):
         """One forward from host tensors into host ``hO`` (and ``hlse``): the copies of
@@ -432,3 +488,10 @@ class SparkAttention:
         if getattr(self, "host_ws", None) is None or self.host_ws.numel() < need:
             self.host_ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.O.device)
         return forward_host(hQ, hK, hV, self.shape, hcfg, hO, hlse, self.host_ws, self.O.device)
+
+    def extra_rows(self):
+        """The extra tokens of every head, [B, H, E] int32 (rows of the video tokens the
+        attention ran on: the reblocked order with Reblock), or None without extra tokens."""
+        if self.xpack is None:
+            return None
+        return extra_token_rows(self.xpack, self.shape.B, self.shape.H, self.nb, self.cfg.extra_tokens)

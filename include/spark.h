@@ -155,12 +155,41 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
  * q_tile = 64 runs 64-query tiles on M = 64 tensor-core MMAs, q_tile = 128 runs 128-query
  * tiles (dense rows too) on M = 128 MMAs; the 128-query kernel hands the tiles out to the
  * CTAs at run time, head by head (each head's dense-row tiles, the longest, lead its tiles).
+ * extra_pack / extra_tokens: with extra_tokens > 0 the extra pack written by
+ * spark_extra_tokens (same shape, same extra_tokens, 16-byte aligned, not NULL): every
+ * video query also attends exactly to the head's extra tokens that lie outside its selected
+ * blocks (those inside are attended as part of the block); dense query rows already attend
+ * to every key and are unchanged. extra_tokens = 0: extra_pack is not read (may be NULL).
  * ws: spark_workspace_bytes(s, SPARK_CALL_ATTN) bytes, 16-byte aligned, not shared with a
  * launch in flight on another stream. */
 int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
-                   const float* beta, const int32_t* perm, uint16_t* O, float* lse, void* ws,
-                   size_t ws_bytes, void* stream);
+                   const float* beta, const int32_t* perm, const void* extra_pack, int32_t extra_tokens,
+                   uint16_t* O, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Extra tokens ("ComfyUI adds a core sparse-attention node and the Comfy Compiler",
+ * section "Block-sparse attention: one node, three backends": extra_tokens adds the
+ * highest-scoring tokens beyond the selected blocks, to stay close to dense attention).
+ * The pages give neither the score nor the count's unit; this library reads it as a
+ * per-head budget E = min(extra_tokens, nb*64) of video keys ranked by the anchor score
+ * s_j = anchor . k_j * scale (the per-token score of the compressed branch), ties to the
+ * lower token index. Runs after spark_pool_kv on the same (reblocked) K, V and its anchor:
+ *   - writes the extra pack: the tokens' row indices (ascending, int32 [B*H, ep], -1 past
+ *     E; ep = 64 * ceil(E / 64)), the anchor scores of every video key (fp32 [B*H, nb*64])
+ *     and the tokens' K and V rows (bf16 [B*H*ep, d] each, zero past E);
+ *   - when pool_pack is not NULL, rewrites the compressed entry of every block that lost
+ *     tokens so that it stands for the block's remaining tokens R_b only: bf16 key mean of
+ *     R_b and value summary over R_b in pool_pack, log-mass bias lse(s over R_b) -
+ *     anchor . mean_k(R_b) * scale (pool_mode SPARK_POOL_MEAN: mean value of R_b and
+ *     log |R_b|) in pool_pack and in v_summ / beta when those are not NULL; a block whose
+ *     64 tokens are all extra gets beta = -inf (no entry). k_pool (the block scores) is
+ *     not changed.
+ * extra_pack: spark_extra_pack_bytes(s, extra_tokens) bytes, 16-byte aligned, caller-owned.
+ * extra_tokens = 0 (or no video block) does nothing. */
+size_t spark_extra_pack_bytes(const spark_shape* s, int32_t extra_tokens);
+int spark_extra_tokens(const spark_shape* s, const uint16_t* K, const uint16_t* V, const float* anchor,
+                       int32_t extra_tokens, int pool_mode, float* v_summ, float* beta, void* pool_pack,
+                       size_t pool_pack_bytes, void* extra_pack, size_t extra_pack_bytes, void* stream);
 
 /* Spark-Reblock ("What Spark-Attn changes", Spark-Reblock bullet; "Workflows":
  * reblock_layout=q_reuse_k). Per (b, h): M = mean over video keys of k k^T;
@@ -228,6 +257,7 @@ typedef struct spark_fwd_config {
   int32_t compressed;      /* compressed branch on (!= 0) or off */
   int32_t reblock;         /* 0 none, 1 spark_reblock, 2 spark_reblock_kv */
   int32_t heads_per_group; /* heads per pipeline group; <= 0: automatic (see above) */
+  int32_t extra_tokens;    /* extra tokens per head (spark_extra_tokens); 0: none */
 } spark_fwd_config;
 
 /* Device workspace bytes of spark_forward_host; 0 for an invalid shape or config. */
@@ -250,8 +280,12 @@ int spark_forward_host(const spark_shape* s, const spark_fwd_config* cfg, const 
  * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  * - B*H above SPARK_NOALLOC_MAX_HEADS returns SPARK_ESCRATCH before any launch.
  * - The first call on a device looks the array's device address up (cudaGetSymbolAddress,
- *   with that device current) and caches it; make that first call before any stream
- *   capture on the device.
+ *   with that device current) and caches it with the unique ID of the device's current
+ *   context; make that first call before any stream capture on the device. After a
+ *   device reset (cudaDeviceReset, or the primary context released and created again)
+ *   the context ID changes and the next call looks the address up again, so that call
+ *   too should come before any capture. A call from a host thread on which the runtime
+ *   has not yet made the context current also repeats the lookup.
  * - Every call shares the one array: calls whose work overlaps on the GPU (different
  *   streams, or different host threads without ordering) race on it. The part that must
  *   start at zero is cleared by each call. */
@@ -271,6 +305,16 @@ const char* spark_strerror(int status);
  * and threads), counted on the host as each launch is issued. No counterpart in the
  * method: it lets a caller account for the device work of a region of calls. */
 uint64_t spark_kernel_launches(void);
+
+/* Limit, in SM clocks, of every pipeline wait of the attention kernels launched after this
+ * call (all devices and threads of the process); clocks <= 0 restores the default of
+ * 2^31 clocks (about a second). No counterpart in the method: it exists so that the
+ * failure path can be exercised without faulting a GPU. A wait that runs out records
+ * SPARK_ETIMEOUT in the device error word, every role of the CTA stops, the copies and
+ * MMAs still in flight are drained (those drains keep the default limit) and tensor
+ * memory is released; the call's outputs are then undefined, and the device stays usable.
+ * A limit of a few hundred clocks makes the first waits of a launch give up. */
+int spark_set_wait_limit(int64_t clocks);
 
 #ifdef __cplusplus
 }

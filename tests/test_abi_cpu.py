@@ -70,7 +70,7 @@ def test_query_tiles_of_the_128_query_route(spark):
     bad_tile = spark.make_shape(1, 1, 128, 64, 0, q_tile=96)
     dummy = ctypes.c_void_p(16)
     assert lib.spark_attn_fwd(ctypes.byref(bad_tile), dummy, dummy, dummy, dummy, dummy, 1, None,
-                              None, None, dummy, None, None, 0, None) == -2
+                              None, None, None, 0, dummy, None, None, 0, None) == -2
     assert spark.num_query_tiles(bad_tile) == 0
 
 
@@ -83,10 +83,10 @@ def test_bad_arguments_are_rejected_on_the_host(spark):
                              dummy, dummy, dummy, 1 << 20, None) == -2
     bad_block = spark.Shape(1, 1, 128, 64, 0, 32, 0.0, 0)
     assert lib.spark_attn_fwd(ctypes.byref(bad_block), dummy, dummy, dummy, dummy, dummy, 1, None,
-                              None, None, dummy, None, None, 0, None) == -2
+                              None, None, None, 0, dummy, None, None, 0, None) == -2
     neg = spark.make_shape(1, 1, 128, 64, 200)
     assert lib.spark_attn_fwd(ctypes.byref(neg), dummy, dummy, dummy, dummy, dummy, 1, None, None,
-                              None, dummy, None, None, 0, None) == -1
+                              None, None, 0, dummy, None, None, 0, None) == -1
     ok = spark.make_shape(1, 1, 128, 64, 0)
     # null inputs, misaligned pointers, bad ratio, kcap below k, unknown mode, bad pool mode
     assert lib.spark_pool_kv(ctypes.byref(ok), None, dummy, dummy, 0, dummy, dummy, dummy, dummy,
@@ -110,16 +110,44 @@ def test_bad_arguments_are_rejected_on_the_host(spark):
                              dummy, 1 << 30, None) == -1
     # the attention call needs its item-counter workspace
     assert lib.spark_attn_fwd(ctypes.byref(ok), dummy, dummy, dummy, dummy, dummy, 1, None, None,
-                              None, dummy, None, None, 0, None) == -1
+                              None, None, 0, dummy, None, None, 0, None) == -1
     assert lib.spark_attn_fwd(ctypes.byref(ok), dummy, dummy, dummy, dummy, dummy, 1, None, None,
-                              None, dummy, None, dummy, 64, None) == -1
+                              None, None, 0, dummy, None, dummy, 64, None) == -1
+
+
+def test_extra_token_arguments_are_checked_on_the_host(spark):
+    lib = spark.load()
+    dummy = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    s = spark.make_shape(1, 2, 64 * 10 + 7, 64, 7)
+    # layout: xidx [2, 64] int32, scores [2, 640] fp32, K and V rows [2 * 64, 64] bf16, each
+    # part on a 256-byte boundary
+    assert spark.extra_pack_bytes(s, 37) == 512 + 5120 + 16384 + 16384
+    assert spark.extra_pack_bytes(s, 0) == 0
+    assert spark.extra_pack_bytes(s, 10 ** 6) == spark.extra_pack_bytes(s, 640)
+    need = spark.extra_pack_bytes(s, 37)
+    assert lib.spark_extra_tokens(ctypes.byref(s), dummy, dummy, dummy, -1, 0, None, None, None, 0,
+                                  dummy, need, None) == -1
+    assert lib.spark_extra_tokens(ctypes.byref(s), dummy, dummy, dummy, 37, 0, None, None, None, 0,
+                                  dummy, need - 16, None) == -1
+    assert lib.spark_extra_tokens(ctypes.byref(s), dummy, dummy, dummy, 37, 3, None, None, None, 0,
+                                  dummy, need, None) == -1
+    assert lib.spark_extra_tokens(ctypes.byref(s), dummy, dummy, None, 37, 0, None, None, None, 0,
+                                  dummy, need, None) == -1
+    assert lib.spark_extra_tokens(ctypes.byref(s), dummy, dummy, dummy, 0, 0, None, None, None, 0,
+                                  None, 0, None) == 0          # nothing to do
+    assert lib.spark_attn_fwd(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, 1, None, None,
+                              None, None, -3, dummy, None, dummy, 256, None) == -1
+    assert lib.spark_attn_fwd(ctypes.byref(s), dummy, dummy, dummy, dummy, dummy, 1, None, None,
+                              None, None, 37, dummy, None, dummy, 256, None) == -1   # no pack
+    cfg = spark.fwd_config(extra_tokens=-2)
+    assert spark.forward_host_workspace_bytes(s, cfg) == 0
 
 
 def test_empty_inputs_are_a_no_op(spark):
     lib = spark.load()
     empty = spark.make_shape(0, 4, 128, 64, 0)
     assert lib.spark_attn_fwd(ctypes.byref(empty), None, None, None, None, None, 1, None, None,
-                              None, None, None, None, 0, None) == 0
+                              None, None, 0, None, None, None, 0, None) == 0
     zero_n = spark.make_shape(1, 4, 0, 64, 0)
     assert lib.spark_pool_kv(ctypes.byref(zero_n), None, None, None, 0, None, None, None, None,
                              None, None, 0, None) == 0
@@ -131,7 +159,7 @@ def test_strerror(spark):
 
 
 def test_host_forward_config_and_workspace(spark):
-    assert ctypes.sizeof(spark.FwdConfig) == 32
+    assert ctypes.sizeof(spark.FwdConfig) == 40   # double + 7 int32, padded to 8 bytes
     s = spark.make_shape(2, 3, 64 * 10 + 7 + 16, 64, 16)
     nb, N, d = 10, 64 * 10 + 7 + 16, 64
     cfg = spark.fwd_config(heads_per_group=2)
@@ -147,6 +175,9 @@ def test_host_forward_config_and_workspace(spark):
              + up(spark.workspace_bytes(g, spark.CALL_POOL)) + up(G * nb * k * 4) + up(G * nb * 4)
              + up(spark.workspace_bytes(g, spark.CALL_SELECT)) + up(256))
     assert ws == slots + inter
+    # extra tokens add the extra pack of one group
+    ex = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=2, extra_tokens=37))
+    assert ex == ws + up(spark.extra_pack_bytes(g, 37))
     # reblock adds the permutation, the permuted copies and its own scratch
     rb = spark.forward_host_workspace_bytes(s, spark.fwd_config(heads_per_group=2, reblock=1))
     assert rb == ws + up(G * nb * 64 * 4) + 3 * up(G * N * d * 2) + up(spark.workspace_bytes(g, spark.CALL_REBLOCK))

@@ -68,3 +68,30 @@ def test_reference_arm_under_torchrun_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_flag_spawns_ranks_without_torchrun():
+    """`bench.py --gpus 2` outside torchrun re-launches itself on two ranks; rank 0 alone
+    prints the (reference-arm) line, whose unit string is the one the device arm prints."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+           "--warmup", "0", "--cpu-blocks", "2", "--workload", "32k-exact"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    sys.path.insert(0, ROOT)
+    import bench
+    assert d["n_gpus"] == 2 and d["impl"] == "reference"
+    assert d["unit"] == bench.unit_of(bench.WORKLOADS["32k-exact"]) == d["e2e"]["unit"]
+
+
+def test_spawn_command_keeps_arguments():
+    sys.path.insert(0, ROOT)
+    import bench
+    cmd = bench.spawn_ranks_command(["--gpus", "4", "--steps", "7"], 4, 29555)
+    i = cmd.index("--nproc-per-node")
+    assert cmd[i + 1] == "4" and "127.0.0.1" in cmd and cmd[-3:] == ["--gpus", "4", "--steps", "7"][-3:]
+    assert cmd[cmd.index("--master-port") + 1] == "29555"

@@ -6,11 +6,18 @@ plain mean-pooled entry. At the 1152x640x243 shape (2 heads), top-k 10%, the for
 without a compressed branch, with the mean-pooled branch and with the reweighted branch
 are compared with the dense forward (density 1.0, which the parity tests tie to dense
 softmax attention). Dropping the unselected blocks must be far worse than either
-compressed branch, and the reweighted branch must not be worse than the mean-pooled one
-(on this synthetic data the two differ by about 1e-5 relative: the anchor, the mean of
-near-isotropic queries, is short, so beta stays close to log 64 and the two entries
-nearly coincide; the oracle orders them strictly on smaller heads).
+compressed branch.
+
+Two input families: the plain block-correlated one, where the mean query (the anchor) is
+short, so beta stays close to log 64 and the two compressed entries nearly coincide (they
+differ by about 1e-5 relative, and the reweighted one must not be worse); and queries
+with a per-head mean direction (``q_offset = 1``), where the anchor scores inside a block
+spread by about one unit, beta departs from log 64 by about 0.5, and the reweighted branch
+must be clearly closer to dense attention than the mean-pooled one (the oracle orders them
+the same way on smaller heads).
 """
+import math
+
 import pytest
 import torch
 
@@ -19,13 +26,14 @@ from block_sparse_video_mean_b200.inputs import make_qkv
 pytestmark = pytest.mark.gpu
 
 
-def test_compressed_branch_fidelity_at_full_length():
+@pytest.mark.parametrize("q_offset", [0.0, 1.0])
+def test_compressed_branch_fidelity_at_full_length(q_offset):
     import block_sparse_video_mean_b200.spark as spark
 
     spark.load()
     dev = torch.device("cuda", 0)
     B, H, nv, ns, d = 1, 2, 175680, 512, 128
-    Q, K, V = make_qkv(B, H, nv, ns, d, seed=4, device=dev)
+    Q, K, V = make_qkv(B, H, nv, ns, d, seed=4, device=dev, q_offset=q_offset)
     N = nv + ns
 
     def run(cfg):
@@ -33,14 +41,22 @@ def test_compressed_branch_fidelity_at_full_length():
         O, _ = plan.run(Q, K, V)
         torch.cuda.synchronize()
         assert spark.device_error(dev) == 0
-        return O[:, :, :nv].float().clone()
+        return O[:, :, :nv].float().clone(), plan
 
-    dense = run(spark.ForwardConfig("topk", 1.0, False))
+    dense, _ = run(spark.ForwardConfig("topk", 1.0, False))
     err = {}
     for name, comp, pm in (("none", False, "reweight"), ("mean", True, "mean"),
                            ("reweight", True, "reweight")):
-        o = run(spark.ForwardConfig("topk", 0.1, comp, pm))
+        o, plan = run(spark.ForwardConfig("topk", 0.1, comp, pm))
         err[name] = float(torch.linalg.vector_norm(o - dense) / torch.linalg.vector_norm(dense))
-    print("relative distance to dense attention:", err)
+        if name == "reweight":
+            excess = float((plan.pool["beta"] - math.log(64)).mean())
+    print(f"q_offset {q_offset}: relative distance to dense attention:", err,
+          "mean beta - log 64:", excess)
     assert err["none"] > 2.0 * max(err["mean"], err["reweight"]), err
-    assert err["reweight"] <= err["mean"] * 1.001, err
+    if q_offset == 0:
+        assert err["reweight"] <= err["mean"] * 1.001, err
+        assert excess < 0.05
+    else:
+        assert err["reweight"] < 0.9 * err["mean"], err
+        assert excess > 0.2

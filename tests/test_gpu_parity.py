@@ -104,6 +104,27 @@ def test_small_every_element(spark, d, nv, ns, mode, param, compressed, pool_mod
         compare_head(plan, O, L, Q, K, V, 0, h, ns, cfg)
 
 
+# queries with a per-head mean direction: beta departs from log 64 by O(1) and a few key
+# blocks are selected by most query blocks (the compressed branch is stressed)
+OFFSET = [
+    # d, n_video, n_sink, mode, param, pool_mode
+    (128, 64 * 60, 40, "topk", 0.1, "reweight"),
+    (64, 64 * 45 + 9, 17, "tau", 1.0, "reweight"),
+    (128, 64 * 33, 0, "topk", 0.2, "mean"),
+]
+
+
+@pytest.mark.parametrize("d,nv,ns,mode,param,pool_mode", OFFSET)
+@pytest.mark.parametrize("q_tile", [64, 128])
+def test_small_offset_queries_every_element(spark, d, nv, ns, mode, param, pool_mode, q_tile):
+    Q, K, V = make_qkv(1, 2, nv, ns, d, seed=21, q_offset=1.0)
+    cfg = spark.ForwardConfig(mode, param, True, pool_mode, q_tile=q_tile)
+    plan, O, L = run_plan(spark, Q, K, V, ns, cfg)
+    assert spark.device_error() == 0
+    for h in range(2):
+        compare_head(plan, O, L, Q, K, V, 0, h, ns, cfg)
+
+
 def test_empty_rows_give_zero_and_neg_inf(spark):
     Q, K, V = make_qkv(1, 1, 64 * 16, 0, 64, seed=1)
     cfg = spark.ForwardConfig("tau", 50.0, False)

@@ -2,8 +2,9 @@
 memory themselves (an engine that owns one arena, a plugin inside another framework's
 allocator, a loop that must never reach the driver's allocator).
 
-spark_score_select_noalloc keeps its scratch in a fixed device array of the library and
-must select exactly what spark_score_select selects with caller scratch; it is called
+spark_score_select_noalloc keeps its scratch in a fixed device array of the library. Its
+selection and that of spark_score_select (caller scratch) are both checked, row by row,
+against the fp64 oracle's selection of the same inputs on both query routes; it is called
 twice in a row to show that the shared array is cleared between calls. This file runs
 last so that a failure here leaves the rest of the suite already run."""
 import ctypes
@@ -30,37 +31,43 @@ def spark():
     return spark
 
 
-def _same_selection(a, b, q_pool, k_pool, mode, param, d):
-    """Identical, or different only at near-ties (the suite's selection tolerance)."""
-    ia, ca = (t.cpu().numpy() for t in a)
-    ib, cb = (t.cpu().numpy() for t in b)
-    B, H, nb = ca.shape
+def _check_against_oracle(sels, Q, K, V, ns, mode, param, q_tile):
+    """Every row of every (idx, cnt) selection in ``sels`` against the fp64 oracle's
+    selection of the same inputs (pooled by the oracle), up to near-ties."""
+    B, H, N, d = Q.shape
     scale = 1.0 / math.sqrt(d)
-    for bb in range(B):
+    host = [(gi.cpu().numpy(), gc.cpu().numpy()) for gi, gc in sels]
+    for b in range(B):
         for h in range(H):
-            ra, rb = gpu_rows(ia[bb, h], ca[bb, h]), gpu_rows(ib[bb, h], cb[bb, h])
-            if all(np.array_equal(x, y) for x, y in zip(ra, rb)):
-                continue
-            qp = q_pool[bb, h].cpu().double().numpy()
-            kp = k_pool[bb, h].cpu().double().numpy()
-            S = orc.block_scores(qp, kp, scale)
+            q, k, v = (orc.to_f64(t[b, h]) for t in (Q, K, V))
+            P = orc.pool_head(q, k, v, ns, scale, 64, "reweight", q_tile)
+            S = orc.block_scores(P.qbar, P.kbar, scale)
             thr = orc.tau_threshold(S, param) if mode == "tau" else None
-            for i in range(nb):
-                assert check_selection_row(rb[i], S[i], mode, param, thr)[0], (bb, h, i)
+            for gi, gc in host:
+                sel = gpu_rows(gi[b, h], gc[b, h])
+                assert len(sel) == S.shape[0]
+                for i in range(S.shape[0]):
+                    ok, ndiff = check_selection_row(sel[i], S[i], mode, param, thr)
+                    assert ok, (b, h, i, ndiff)
 
 
-@pytest.mark.parametrize("mode,param", [("tau", 1.0), ("tau", 2.0), ("topk", 0.1)])
-def test_noalloc_matches_scratch_entry_point(spark, mode, param):
-    B, H, nv, ns, d = 1, 6, 64 * 300, 40, 128
-    Q, K, V = make_qkv(B, H, nv, ns, d, seed=9, device=DEV)
-    pool = spark.pool_kv(Q, K, V, ns)
+@pytest.mark.parametrize("mode,param,q_tile", [("tau", 1.0, 64), ("tau", 2.0, 64), ("topk", 0.1, 64),
+                                               ("topk", 0.1, 128), ("tau", 1.5, 128)])
+def test_noalloc_matches_scratch_entry_point(spark, mode, param, q_tile):
+    B, H, nv, ns, d = 1, 6, 64 * 301, 40, 128
+    Q, K, V = make_qkv(B, H, nv, ns, d, seed=9)
+    Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
+    pool = spark.pool_kv(Qd, Kd, Vd, ns, q_tile=q_tile)
     m = spark.SELECT_TAU if mode == "tau" else spark.SELECT_TOPK_RATIO
-    ref = spark.score_select(pool["q_pool"], pool["k_pool"], ns, Q.shape[2], m, param)
+    ref = spark.score_select(pool["q_pool"], pool["k_pool"], ns, Q.shape[2], m, param, q_tile=q_tile)
+    got = []
     for _ in range(2):  # twice in a row: the shared scratch must be cleared by each call
-        got = spark.score_select_noalloc(pool["q_pool"], pool["k_pool"], ns, Q.shape[2], m, param)
+        sel = spark.score_select_noalloc(pool["q_pool"], pool["k_pool"], ns, Q.shape[2], m, param,
+                                         q_tile=q_tile)
         torch.cuda.synchronize()
         assert spark.device_error() == 0
-        _same_selection(ref, got, pool["q_pool"], pool["k_pool"], mode, param, d)
+        got.append(tuple(t.clone() for t in sel))
+    _check_against_oracle([ref] + got, Q, K, V, ns, mode, param, q_tile)
 
 
 def test_noalloc_rejects_more_heads_than_its_scratch(spark):
