@@ -448,8 +448,18 @@ def run_gpu(args, w: Workload, rank, world, local_rank):
                  "compressed_flops": fl["compressed"]},
     }
     if w.reblock:
-        phases["reblock"] = {"ms": round(phase_ms["reblock"], 3),
-                             "gather_bytes": by["reblock_gather"]}
+        # the covariance sums of every bisection level, the keys' second moment and the
+        # whitening: 2 * N_v * d^2 flops each per head (fp32 products, fp64 sums)
+        levels = max(1, math.ceil(math.log2(max(nb, 2))))
+        passes = (levels + 2) * (2 if w.reblock_kv else 1)
+        cov = 2 * w.B * h * nb * 64 * w.d * w.d * passes
+        rb_ms = phase_ms["reblock"]
+        phases["reblock"] = {"ms": round(rb_ms, 3), "gather_bytes": by["reblock_gather"],
+                             "covariance_flops": cov,
+                             "fp32_tflops": round(cov / (rb_ms * 1e-3) / 1e12, 2),
+                             "frac_fp32": round(cov / (rb_ms * 1e-3) / 1e12 / FP32_PEAK_TFLOPS, 4),
+                             "bound": "fp32 FMA (covariance sums; fp64 eigen-solves beside them), "
+                                      "HBM for the gather"}
     line = {
         "metric": metric_of(w),
         "value": round(value, 2),

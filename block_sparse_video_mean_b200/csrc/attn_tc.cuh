@@ -225,11 +225,13 @@ __device__ __forceinline__ int tc_half_kind(const TcItem& I, int hi, int n_dk, i
   return kHalfPooled;
 }
 
-// Masks the extra-token entries of half `e0 / 64` in x: entries past the head's count and
-// tokens whose block the item selected (already attended there).
-__device__ __forceinline__ void tc_mask_extra(float* x, const int32_t* xs, int e0, int n_extra,
-                                              const uint32_t* bm) {
-#pragma unroll
+// Keep-mask (bit e set: entry e attended) of the extra-token half starting at entry e0:
+// entries past the head's count and tokens whose block the item selected (attended there)
+// are dropped. One 16-byte load at a time, so that the few registers it needs do not
+// compete with the thread's 64 scores.
+__device__ __forceinline__ uint64_t tc_extra_keep(const int32_t* xs, int e0, int n_extra, const uint32_t* bm) {
+  uint64_t keep = 0;
+#pragma unroll 1
   for (int q4 = 0; q4 < 16; ++q4) {
     const int4 t4 = __ldg(reinterpret_cast<const int4*>(xs + e0) + q4);
     const int tt[4] = {t4.x, t4.y, t4.z, t4.w};
@@ -237,19 +239,24 @@ __device__ __forceinline__ void tc_mask_extra(float* x, const int32_t* xs, int e
     for (int i = 0; i < 4; ++i) {
       const int e = 4 * q4 + i;
       const int tok = tt[i];
-      bool masked = e0 + e >= n_extra || tok < 0;
-      if (!masked) {
+      bool on = e0 + e < n_extra && tok >= 0;
+      if (on) {
         const int blk = tok >> 6;
-        masked = (bm[blk >> 5] >> (blk & 31)) & 1u;
+        on = !((bm[blk >> 5] >> (blk & 31)) & 1u);
       }
-      if (masked) x[e] = -INFINITY;
+      keep |= (uint64_t)(on ? 1u : 0u) << e;
     }
   }
+  return keep;
 }
 
-template <int D>
+// kExtra: the extra-token half kind is compiled in only when a launch has extra tokens
+// (launches without them run code without it: it changes how the rest is compiled, and
+// the 128-query kernel's results then varied from run to run within the tolerance).
+template <int D, bool kExtra>
 __global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  const int n_xh = kExtra ? p.n_xh : 0;
   using C = TcCfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem =
@@ -412,14 +419,14 @@ __global__ void __launch_bounds__(384, 1)
                 y[hf] = I.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
               } else if (hi < I.cnt + n_dk) {
                 y[hf] = I.bh * p.N + nv + (hi - I.cnt) * kBlock;
-              } else if (hi < I.cnt + n_dk + p.n_xh) {
+              } else if (hi < I.cnt + n_dk + n_xh) {
                 src[hf] = 2;
                 y[hf] = I.bh * p.ep + (hi - I.cnt - n_dk) * kBlock;
               } else {
                 // pooled entries past nb read rows of the next head (or TMA zero fill);
                 // their bias is -inf, so they carry no weight
                 src[hf] = 1;
-                y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk - p.n_xh) * kBlock;
+                y[hf] = I.bh * p.nb + (hi - I.cnt - n_dk - n_xh) * kBlock;
               }
             }
             // one box per lane (lanes 0 .. 2 kPanels - 1): TMA issue throughput is per
@@ -604,13 +611,13 @@ __global__ void __launch_bounds__(384, 1)
         }
 #pragma unroll
         for (int c = 0; c < C::kQPieces; ++c)
-          tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + qb * (D / 2) + 16 * c, qv + 16 * c);
+          tc::tmem_st_16x32bx2_x16_sync<D / 4>(tbase + lanes + C::kColQ + qb * (D / 2) + 16 * c, qv + 16 * c);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&qfull[2 * s + qb]);
       }
-      if (!J.dense && (p.pooled || J.cnt > 0 || p.n_xh > 0)) {
+      if (!J.dense && (p.pooled || J.cnt > 0 || n_xh > 0)) {
         uint32_t* bm = bm2 + qb * nbwp;
         for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
         __syncwarp();
@@ -645,7 +652,7 @@ __global__ void __launch_bounds__(384, 1)
     auto epilogue = [&](const TcItem& I, float m_run, float l_run) -> bool {
       // odone completes once per item, after its last PV; it cannot run an item ahead
       // because the next item's PVs need this slot's P tiles.
-      if (!tc::mbar_wait(&odone[s], ndone & 1, abort_flag, p.wait_clocks)) return false;
+      if (!tc::mbar_wait_warp(&odone[s], ndone & 1, abort_flag, p.wait_clocks)) return false;
       ++ndone;
       tc::tc_fence_after();
       uint32_t o[D / 2];
@@ -739,18 +746,25 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t b = g & 1;
         // warm L1 with the biases of a pooled half (their loads follow the S wait)
         const int hi = 2 * t + h;
-        const int kind = tc_half_kind(I, hi, n_dk, p.n_xh);
+        const int kind = tc_half_kind(I, hi, n_dk, n_xh);
         const float* bias_src =
-            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk - p.n_xh) * kBlock : 0);
+            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk - n_xh) * kBlock : 0);
         if (kind == kHalfPooled && lh < 2) prefetch_l1(bias_src + 32 * lh);
-        if (!tc::mbar_wait(&sfull[2 * s + b], (g >> 1) & 1, abort_flag, p.wait_clocks)) {
+        if (!tc::mbar_wait_warp(&sfull[2 * s + b], (g >> 1) & 1, abort_flag, p.wait_clocks)) {
           ok = false;
           break;
         }
         tc::tc_fence_after();
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h+63 of the S buffer)
+        // loaded as words, then converted: the scores are not read through a pointer of
+        // another type (the compiler may reorder accesses it believes cannot alias)
         float x[64];
-        tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, reinterpret_cast<uint32_t*>(x));
+        {
+          uint32_t xw[64];
+          tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, xw);
+#pragma unroll
+          for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(xw[j]);
+        }
         // ---- logits (base 2) and masks of this half
         // Exact and dense halves keep raw scores (the scale is folded into the exponent's
         // FFMA); pooled halves become scale*logit + beta*log2(e), with the selected blocks
@@ -771,12 +785,19 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = 0; j < 64; ++j)
               if (j >= valid) x[j] = -INFINITY;
           }
-          if (kind == kHalfExtra)
-            tc_mask_extra(x, p.xidx + (size_t)I.bh * p.ep, (hi - I.cnt - n_dk) * kBlock, p.n_extra, bm);
+          if constexpr (kExtra) {
+            if (kind == kHalfExtra) {
+              const uint64_t keep = tc_extra_keep(p.xidx + (size_t)I.bh * p.ep, (hi - I.cnt - n_dk) * kBlock,
+                                                  p.n_extra, bm);
+#pragma unroll
+              for (int j = 0; j < 64; ++j)
+                if (!((keep >> j) & 1ull)) x[j] = -INFINITY;
+            }
+          }
         }
         if (kind == kHalfPooled) {
           const float4* bsrc = reinterpret_cast<const float4*>(bias_src);
-          const int j0 = (hi - I.cnt - n_dk - p.n_xh) * kBlock;
+          const int j0 = (hi - I.cnt - n_dk - n_xh) * kBlock;
           const int wb = j0 >> 5;  // j0 is a multiple of 64, wb + 1 < nbwp
           const uint32_t w0 = bm[wb], w1 = bm[wb + 1];
 #pragma unroll
@@ -816,7 +837,7 @@ __global__ void __launch_bounds__(384, 1)
         const float alpha = need ? ex2f(m_run - m_new) : 1.0f;
         if (__any_sync(0xffffffffu, need && t > 0)) {
           // rescale the O rows of this warp once the previous PV has landed
-          if (!tc::mbar_wait(&oready[s], (g - 1) & 1, abort_flag, p.wait_clocks)) {
+          if (!tc::mbar_wait_warp(&oready[s], (g - 1) & 1, abort_flag, p.wait_clocks)) {
             ok = false;
             break;
           }
@@ -827,7 +848,7 @@ __global__ void __launch_bounds__(384, 1)
             tc::tmem_ld_16x32bx2_x16_sync<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-            tc::tmem_st_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
+            tc::tmem_st_16x32bx2_x16_sync<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
           }
         }
         if (need) {
@@ -852,7 +873,7 @@ __global__ void __launch_bounds__(384, 1)
               l2[j & 1] = tc::fadd2(l2[j & 1], make_float2(p0, p1));
               pk[j] = pack_bf16x2(p0, p1);
             }
-            tc::tmem_st_16x32bx2_x16<32>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
+            tc::tmem_st_16x32bx2_x16_sync<32>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
           }
           ls[0] = l2[0].x; ls[1] = l2[0].y; ls[2] = l2[1].x; ls[3] = l2[1].y;
         }

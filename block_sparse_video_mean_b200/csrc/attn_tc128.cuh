@@ -88,9 +88,13 @@ __device__ __forceinline__ TcItem tc128_item(const TcParams& p, int it) {
   return r;
 }
 
-template <int D>
+// kExtra: the extra-token half kind is compiled in only when a launch has extra tokens
+// (launches without them run code without it: it changes how the rest is compiled, and
+// the 128-query kernel's results then varied from run to run within the tolerance).
+template <int D, bool kExtra>
 __global__ void __launch_bounds__(384, 1)
     attn_tc128_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  const int n_xh = kExtra ? p.n_xh : 0;
   using C = Tc128Cfg<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem =
@@ -238,14 +242,14 @@ __global__ void __launch_bounds__(384, 1)
           y[hf] = cur.bh * p.N + ((bsel >= 0 && bsel < p.nb) ? bsel : 0) * kBlock;
         } else if (hi < cur.cnt + n_dk) {
           y[hf] = cur.bh * p.N + nv + (hi - cur.cnt) * kBlock;
-        } else if (hi < cur.cnt + n_dk + p.n_xh) {
+        } else if (hi < cur.cnt + n_dk + n_xh) {
           src[hf] = 2;
           y[hf] = cur.bh * p.ep + (hi - cur.cnt - n_dk) * kBlock;
         } else {
           // pooled entries past nb read rows of the next head (or TMA zero fill); their
           // bias is -inf, so they carry no weight
           src[hf] = 1;
-          y[hf] = cur.bh * p.nb + (hi - cur.cnt - n_dk - p.n_xh) * kBlock;
+          y[hf] = cur.bh * p.nb + (hi - cur.cnt - n_dk - n_xh) * kBlock;
         }
       }
       // one box per lane: TMA issue throughput is per issuing lane and warp
@@ -391,13 +395,13 @@ __global__ void __launch_bounds__(384, 1)
         }
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tc::tmem_st_16x32bx2_x16<D / 4>(tbase + lanes + C::kColQ + qb * (D / 2) + 16 * c, qv + 16 * c);
+          tc::tmem_st_16x32bx2_x16_sync<D / 4>(tbase + lanes + C::kColQ + qb * (D / 2) + 16 * c, qv + 16 * c);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&qfull[qb]);
       }
-      if (!J.dense && (p.pooled || J.cnt > 0 || p.n_xh > 0)) {
+      if (!J.dense && (p.pooled || J.cnt > 0 || n_xh > 0)) {
         uint32_t* bm = bm2 + qb * nbwp;
         for (int i = lane; i < nbwp; i += 32) bm[i] = 0u;
         __syncwarp();
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(384, 1)
 
     uint32_t ndone = 0;  // non-empty items whose epilogue ran
     auto epilogue = [&](const TcItem& I, float m_run, float l_run) -> bool {
-      if (!tc::mbar_wait(odone, ndone & 1, abort_flag, p.wait_clocks)) return false;
+      if (!tc::mbar_wait_warp(odone, ndone & 1, abort_flag, p.wait_clocks)) return false;
       tc::tc_fence_after();
       uint32_t o[D / 2];
       if constexpr (D == 128)
@@ -523,18 +527,25 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t b = g & 1;
         // warm L1 with the biases of a pooled half (their loads follow the S wait)
         const int hi = 2 * t + h;
-        const int kind = tc_half_kind(I, hi, n_dk, p.n_xh);
+        const int kind = tc_half_kind(I, hi, n_dk, n_xh);
         const float* bias_src =
-            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk - p.n_xh) * kBlock : 0);
+            p.bias + (size_t)I.bh * p.nbp + (kind == kHalfPooled ? (hi - I.cnt - n_dk - n_xh) * kBlock : 0);
         if (kind == kHalfPooled && lane < 2) prefetch_l1(bias_src + 32 * lane);
-        if (!tc::mbar_wait(&sfull[b], (g >> 1) & 1, abort_flag, p.wait_clocks)) {
+        if (!tc::mbar_wait_warp(&sfull[b], (g >> 1) & 1, abort_flag, p.wait_clocks)) {
           ok = false;
           break;
         }
         tc::tc_fence_after();
         // this thread's 64 keys: half h of the tile (columns 64h .. 64h + 63 of the buffer)
+        // loaded as words, then converted: the scores are not read through a pointer of
+        // another type (the compiler may reorder accesses it believes cannot alias)
         float x[64];
-        tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, reinterpret_cast<uint32_t*>(x));
+        {
+          uint32_t xw[64];
+          tc::tmem_ld_16x32bx2_x64_sync<64>(tbase + lanes + C::kColS + 128 * b, xw);
+#pragma unroll
+          for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(xw[j]);
+        }
         // ---- logits (base 2) and masks of this half
         if (kind != kHalfPooled) {
           int valid = kBlock;
@@ -552,11 +563,18 @@ __global__ void __launch_bounds__(384, 1)
             for (int j = 0; j < 64; ++j)
               if (j >= valid) x[j] = -INFINITY;
           }
-          if (kind == kHalfExtra)
-            tc_mask_extra(x, p.xidx + (size_t)I.bh * p.ep, (hi - I.cnt - n_dk) * kBlock, p.n_extra, bm);
+          if constexpr (kExtra) {
+            if (kind == kHalfExtra) {
+              const uint64_t keep = tc_extra_keep(p.xidx + (size_t)I.bh * p.ep, (hi - I.cnt - n_dk) * kBlock,
+                                                  p.n_extra, bm);
+#pragma unroll
+              for (int j = 0; j < 64; ++j)
+                if (!((keep >> j) & 1ull)) x[j] = -INFINITY;
+            }
+          }
         } else {
           const float4* bsrc = reinterpret_cast<const float4*>(bias_src);
-          const int j0 = (hi - I.cnt - n_dk - p.n_xh) * kBlock;
+          const int j0 = (hi - I.cnt - n_dk - n_xh) * kBlock;
           const int wb = j0 >> 5;  // j0 is a multiple of 64, wb + 1 < nbwp
           const uint32_t w0 = bm[wb], w1 = bm[wb + 1];
 #pragma unroll
@@ -595,7 +613,7 @@ __global__ void __launch_bounds__(384, 1)
               l2[j & 1] = tc::fadd2(l2[j & 1], make_float2(p0, p1));
               pk[j] = pack_bf16x2(p0, p1);
             }
-            tc::tmem_st_16x32bx2_x16<64>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
+            tc::tmem_st_16x32bx2_x16_sync<64>(tbase + lanes + C::kColS + 128 * b + 16 * hc, pk);
           }
           ls[0] = l2[0].x; ls[1] = l2[0].y; ls[2] = l2[1].x; ls[3] = l2[1].y;
         };
@@ -619,7 +637,7 @@ __global__ void __launch_bounds__(384, 1)
           const float alpha = need ? ex2f(m_run - m_new) : 1.0f;
           if (t > 0) {
             // rescale this thread's half of its O row once the previous PV has landed
-            if (!tc::mbar_wait(oready, (g - 1) & 1, abort_flag, p.wait_clocks)) {
+            if (!tc::mbar_wait_warp(oready, (g - 1) & 1, abort_flag, p.wait_clocks)) {
               ok = false;
               break;
             }
@@ -630,7 +648,7 @@ __global__ void __launch_bounds__(384, 1)
               tc::tmem_ld_16x32bx2_x16_sync<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
 #pragma unroll
               for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-              tc::tmem_st_16x32bx2_x16<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
+              tc::tmem_st_16x32bx2_x16_sync<D / 2>(tbase + lanes + C::kColO + 16 * c, v);
             }
           }
           if (need) {

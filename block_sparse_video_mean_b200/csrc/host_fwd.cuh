@@ -167,6 +167,7 @@ size_t spark_forward_host_workspace_bytes(const spark_shape* s, const spark_fwd_
 int spark_forward_host(const spark_shape* s, const spark_fwd_config* cfg, const uint16_t* hQ,
                        const uint16_t* hK, const uint16_t* hV, uint16_t* hO, float* hlse,
                        void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_forward_host");
   HostPlan p;
   int st = host_plan(s, cfg, &p);
   if (st != SPARK_OK) return st;

@@ -727,6 +727,359 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
   __syncthreads();
 }
 
+// ------------------------------------------------------------------ Lanczos
+// Leading eigenvector by the Lanczos method (Lanczos 1950; the three-term recurrence with
+// one local re-orthogonalisation against the newest vector), with C in registers as in
+// eigen_top. Pass 1 runs the recurrence and checks the top eigenpair (theta, s) of the
+// Lanczos tridiagonal T_n every kLzCheck steps (multisection on Sturm counts, inverse
+// iteration) until the Ritz residual beta_n |s_n| is below kLzTol * theta. Pass 2 runs the
+// same recurrence again from the same start - the same operations in the same order, so
+// the same vectors bit for bit - and sums the Ritz vector v = sum_j s_j q_j in fp64 as it
+// goes, so no basis is stored. The true residual |C v - theta v| is then measured; the call
+// returns false, with C untouched in shared memory, when it is above kLzAccept * theta or
+// nothing converged within kMax steps, and the caller runs eigen_top. With the residual
+// below 1e-9 theta the eigenvector error is below 1e-9 / relative gap: 1e-5 at the 1e-4
+// gap under which a node counts as a tie.
+constexpr int kLzCheck = 16;
+constexpr double kLzTol = 1e-12;
+constexpr double kLzAccept = 1e-9;
+
+template <int D>
+struct LzScratch {
+  static constexpr int kMax = 2 * D;  // Lanczos steps at most
+  static constexpr int kDoubles = 9 * kMax + 3 * D + 32;  // (2 D used for C q)
+  static constexpr int kBytes = kDoubles * 8 + kMax * 4;
+};
+
+// Largest eigenvalue of the n x n tridiagonal (a, e; e2 = e^2) by multisection on Sturm
+// counts over the Gershgorin interval (all threads). Returns the midpoint of the bracket.
+__device__ double tridiag_top_value(const double* a, const double* e, const double* e2, int n,
+                                    double* red, double* misc) {
+  const int tid = threadIdx.x;
+  double glo = 1e300, ghi = -1e300, emax = 0.0;
+  for (int i = tid; i < n; i += kThreads) {
+    const double r = (i > 0 ? fabs(e[i - 1]) : 0.0) + (i < n - 1 ? fabs(e[i]) : 0.0);
+    glo = fmin(glo, a[i] - r);
+    ghi = fmax(ghi, a[i] + r);
+    if (i < n - 1) emax = fmax(emax, e2[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    glo = fmin(glo, __shfl_xor_sync(0xffffffffu, glo, o));
+    ghi = fmax(ghi, __shfl_xor_sync(0xffffffffu, ghi, o));
+    emax = fmax(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  }
+  if ((tid & 31) == 0) {
+    red[tid >> 5] = glo;
+    red[8 + (tid >> 5)] = ghi;
+    red[16 + (tid >> 5)] = emax;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double lo = red[0], hi = red[8], em = red[16];
+    for (int i = 1; i < kThreads / 32; ++i) {
+      lo = fmin(lo, red[i]);
+      hi = fmax(hi, red[8 + i]);
+      em = fmax(em, red[16 + i]);
+    }
+    const double span = fmax(fabs(lo), fabs(hi)) + 1e-300;
+    misc[0] = lo - 1e-12 * span;
+    misc[1] = hi + 1e-12 * span;
+    misc[2] = 2.2250738585072014e-308 * fmax(1.0, em);
+  }
+  __syncthreads();
+  const double pivmin = misc[2];
+  for (int round = 0; round < 12; ++round) {
+    const double lo = misc[0], hi = misc[1];
+    if (hi - lo <= 1e-14 * fmax(fabs(lo), fabs(hi))) break;
+    const double x = lo + (hi - lo) * (double)(tid + 1) / (double)(kThreads + 1);
+    const int c = sturm_count(a, e2, n, x, pivmin);
+    double clo = (c <= n - 1) ? x : -1e300;  // at or below the top eigenvalue
+    double chi = (c == n) ? x : 1e300;       // above it
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      clo = fmax(clo, __shfl_xor_sync(0xffffffffu, clo, o));
+      chi = fmin(chi, __shfl_xor_sync(0xffffffffu, chi, o));
+    }
+    __syncthreads();
+    if ((tid & 31) == 0) {
+      red[tid >> 5] = clo;
+      red[8 + (tid >> 5)] = chi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double nlo = misc[0], nhi = misc[1];
+      for (int i = 0; i < kThreads / 32; ++i) {
+        nlo = fmax(nlo, red[i]);
+        nhi = fmin(nhi, red[8 + i]);
+      }
+      misc[0] = nlo;
+      misc[1] = nhi;
+    }
+    __syncthreads();
+  }
+  const double theta = 0.5 * (misc[0] + misc[1]);
+  __syncthreads();
+  return theta;
+}
+
+// Unit eigenvector y of the n x n tridiagonal (a, e) at the eigenvalue theta by two steps
+// of inverse iteration (LU with partial pivoting, Newton-refined reciprocals); one thread.
+__device__ void tridiag_inverse_iteration(const double* a, const double* e, int n, double theta,
+                                          double* dd, double* du, double* du2, double* dl, int* piv,
+                                          double* y) {
+  const double tiny = 1e-30 * (fabs(theta) + 1e-300);
+  for (int i = 0; i < n; ++i) {
+    dd[i] = a[i] - theta;
+    if (i < n - 1) dl[i] = du[i] = e[i];
+    du2[i] = 0.0;
+  }
+  for (int i = 0; i < n - 1; ++i) {
+    if (fabs(dd[i]) >= fabs(dl[i])) {
+      if (dd[i] == 0.0) dd[i] = tiny;
+      const double f = dl[i] * rcp_nr(dd[i]);
+      dl[i] = f;
+      dd[i + 1] -= f * du[i];
+      piv[i] = 0;
+    } else {
+      const double f = dd[i] * rcp_nr(dl[i]);
+      dd[i] = dl[i];
+      dl[i] = f;
+      const double tmp = du[i];
+      du[i] = dd[i + 1];
+      dd[i + 1] = tmp - f * dd[i + 1];
+      if (i < n - 2) {
+        du2[i] = du[i + 1];
+        du[i + 1] = -f * du[i + 1];
+      }
+      piv[i] = 1;
+    }
+  }
+  if (dd[n - 1] == 0.0) dd[n - 1] = tiny;
+  for (int i = 0; i < n; ++i) dd[i] = rcp_nr(dd[i]);
+  for (int i = 0; i < n; ++i) y[i] = 1.0 + 0.001 * i;
+  for (int it = 0; it < 2; ++it) {
+    for (int i = 0; i < n - 1; ++i) {
+      if (piv[i] == 0) {
+        y[i + 1] -= dl[i] * y[i];
+      } else {
+        const double tmp = y[i] - dl[i] * y[i + 1];
+        y[i] = y[i + 1];
+        y[i + 1] = tmp;
+      }
+    }
+    y[n - 1] *= dd[n - 1];
+    if (n >= 2) y[n - 2] = (y[n - 2] - du[n - 2] * y[n - 1]) * dd[n - 2];
+    for (int i = n - 3; i >= 0; --i) y[i] = (y[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) * dd[i];
+    double nn = 0.0;
+    for (int i = 0; i < n; ++i) nn += y[i] * y[i];
+    const double inv = 1.0 / sqrt(nn);
+    for (int i = 0; i < n; ++i) y[i] *= inv;
+  }
+}
+
+// Returns true with the unit leading eigenvector of the symmetric C (fp64, shared memory)
+// in v; false when the Lanczos iteration did not reach the accepted residual, with C as it
+// was. `work`: LzScratch<D>::kBytes bytes of shared memory. While C is in registers its
+// buffer holds the first D Lanczos vectors in fp64; when more steps are needed the Ritz
+// vector is summed by a second pass of the same recurrence instead.
+template <int D>
+__device__ bool eigen_top_lanczos(double* C, double* v, unsigned char* work) {
+  using L = LzScratch<D>;
+  constexpr int R = D / 16;
+  constexpr int M = D / 32;  // vector entries per lane (every warp holds whole vectors)
+  constexpr int K = L::kMax;
+  double* al = reinterpret_cast<double*>(work);  // alpha_j
+  double* be = al + K;                            // beta_j
+  double* b2 = be + K;
+  double* s = b2 + K;
+  double* dd = s + K;
+  double* du = dd + K;
+  double* du2 = du + K;
+  double* dl = du2 + K;
+  double* ev = dl + K;                            // off-diagonal copy for the solves
+  double* wv = ev + K;                            // C q_j, double-buffered (2 D)
+  double* red = wv + 3 * D;                       // 24
+  double* misc = red + 24;                        // 8
+  int* piv = reinterpret_cast<int*>(misc + 8);
+  double* basis = C;                              // q_j, j < D, once C is in registers
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15, lane = tid & 31, warp = tid >> 5;
+
+  double c[R][R];
+#pragma unroll
+  for (int ra = 0; ra < R; ++ra)
+#pragma unroll
+    for (int rb = 0; rb < R; ++rb) c[ra][rb] = C[(ty + 16 * ra) * D + tx + 16 * rb];
+  __syncthreads();  // every thread has C in registers: its buffer is free
+
+  // Lanczos state, identical in every warp: lane l holds entries l + 32 m of q_j, q_{j-1}
+  double q[M], qp[M];
+  double beta_prev = 0.0;
+  auto start = [&]() {  // all-positive, slowly varying start vector, normalised
+    double nn = 0.0;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const int i = lane + 32 * m;
+      q[m] = 1.0 + 0.37 * (double)((i * 7919) % 97) / 97.0;
+      qp[m] = 0.0;
+      nn = fma(q[m], q[m], nn);
+    }
+    nn = warp_sum_d(nn);
+    const double inv = 1.0 / sqrt(nn);
+#pragma unroll
+    for (int m = 0; m < M; ++m) q[m] *= inv;
+    beta_prev = 0.0;
+  };
+  // one step from q_j to q_{j+1} (one barrier); stores alpha_j and beta_j (warp 0) and
+  // returns whether the Krylov space became invariant
+  auto step = [&](int j) -> bool {
+    double* w_out = wv + (j & 1) * D;
+    {
+      // the thread's columns tx + 16 rb: entry e lives in lane e % 32, slot e / 32
+      double qv[R];
+#pragma unroll
+      for (int rb = 0; rb < R; ++rb) qv[rb] = __shfl_sync(0xffffffffu, q[rb >> 1], tx + 16 * (rb & 1));
+#pragma unroll
+      for (int ra = 0; ra < R; ++ra) {
+        double acc = 0.0;
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) acc = fma(c[ra][rb], qv[rb], acc);
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (tx == 0) w_out[ty + 16 * ra] = acc;
+      }
+    }
+    __syncthreads();
+    double r[M], w[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) w[m] = w_out[lane + 32 * m];
+    double t = 0.0;
+#pragma unroll
+    for (int m = 0; m < M; ++m) t = fma(q[m], w[m], t);
+    double alpha = warp_sum_d(t);
+#pragma unroll
+    for (int m = 0; m < M; ++m) r[m] = w[m] - alpha * q[m] - beta_prev * qp[m];
+    t = 0.0;  // one local re-orthogonalisation against q_j
+#pragma unroll
+    for (int m = 0; m < M; ++m) t = fma(q[m], r[m], t);
+    const double c2 = warp_sum_d(t);
+#pragma unroll
+    for (int m = 0; m < M; ++m) r[m] -= c2 * q[m];
+    alpha += c2;
+    double bb = 0.0;
+#pragma unroll
+    for (int m = 0; m < M; ++m) bb = fma(r[m], r[m], bb);
+    const double beta = sqrt(warp_sum_d(bb));
+    const bool invariant = !(beta > 1e-13 * (fabs(alpha) + 1e-300));
+    const double inv = invariant ? 0.0 : 1.0 / beta;
+    if (warp == 0 && lane == 0) {
+      al[j] = alpha;
+      be[j] = beta;
+      b2[j] = beta * beta;
+    }
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      qp[m] = q[m];
+      q[m] = r[m] * inv;
+    }
+    beta_prev = beta;
+    return invariant;
+  };
+
+  // ---- pass 1: steps until the Ritz pair has converged (the first D vectors kept)
+  start();
+  int n = 0;
+  double theta = 0.0;
+  bool done = false;
+  for (int j = 0; j < K && !done; ++j) {
+    if (warp == 0 && j < D) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) basis[j * D + lane + 32 * m] = q[m];
+    }
+    const bool invariant = step(j);
+    n = j + 1;
+    if (invariant || (n >= 2 * kLzCheck && n % kLzCheck == 0) || n == K) {
+      __syncthreads();  // al / be of step j are written
+      theta = tridiag_top_value(al, be, b2, n, red, misc);
+      if (tid == 0) {
+        for (int i = 0; i < n; ++i) ev[i] = be[i];
+        tridiag_inverse_iteration(al, ev, n, theta, dd, du, du2, dl, piv, s);
+        const double rho = invariant ? 0.0 : fabs(be[n - 1] * s[n - 1]);
+        misc[3] = (rho <= kLzTol * fabs(theta) || n == K || invariant) ? 1.0 : 0.0;
+      }
+      __syncthreads();
+      done = misc[3] != 0.0;
+      __syncthreads();
+    }
+  }
+  // ---- Ritz vector v = sum_j s_j q_j: from the kept vectors, or by a second pass of the
+  //      same recurrence (the same vectors bit for bit)
+  double acc[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) acc[m] = 0.0;
+  if (n <= D) {
+    for (int j = 0; j < n; ++j) {
+      const double sj = s[j];
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[m] = fma(sj, basis[j * D + lane + 32 * m], acc[m]);
+    }
+  } else {
+    start();
+    for (int j = 0; j < n; ++j) {
+      const double sj = s[j];
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[m] = fma(sj, q[m], acc[m]);
+      if (j + 1 < n) step(j);
+    }
+  }
+  {
+    double t = 0.0;
+#pragma unroll
+    for (int m = 0; m < M; ++m) t = fma(acc[m], acc[m], t);
+    const double inv = 1.0 / sqrt(warp_sum_d(t));
+    if (warp == 0) {
+#pragma unroll
+      for (int m = 0; m < M; ++m) v[lane + 32 * m] = acc[m] * inv;
+    }
+  }
+  __syncthreads();
+  // ---- true residual |C v - theta v| (C still in registers)
+  bool accepted;
+  {
+    double vv[R];
+#pragma unroll
+    for (int rb = 0; rb < R; ++rb) vv[rb] = v[tx + 16 * rb];
+    double part = 0.0;
+#pragma unroll
+    for (int ra = 0; ra < R; ++ra) {
+      double a2 = 0.0;
+#pragma unroll
+      for (int rb = 0; rb < R; ++rb) a2 = fma(c[ra][rb], vv[rb], a2);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) a2 += __shfl_xor_sync(0xffffffffu, a2, off);
+      const double rr = a2 - theta * v[ty + 16 * ra];
+      if (tx == 0) part = fma(rr, rr, part);
+    }
+    const double tot = block_sum_d(part, red);
+    accepted = fabs(theta) > 0.0 && sqrt(tot) <= kLzAccept * fabs(theta);
+  }
+  if (!accepted) {
+    // give C back to the full solver
+#pragma unroll
+    for (int ra = 0; ra < R; ++ra)
+#pragma unroll
+      for (int rb = 0; rb < R; ++rb) C[(ty + 16 * ra) * D + tx + 16 * rb] = c[ra][rb];
+  }
+  __syncthreads();
+  return accepted;
+}
+
+// The leading eigenvector: Lanczos first, the full tridiagonalisation solve as fallback.
+template <int D>
+__device__ __forceinline__ void leading_eigvec(double* C, double* scr, unsigned char* work, double* v) {
+  if (!eigen_top_lanczos<D>(C, v, work)) eigen_top<D>(C, scr, v);
+}
+
 // ------------------------------------------------------------------ one bisection
 struct SplitScratch {
   int hist[256];
@@ -884,7 +1237,8 @@ template <int D>
 struct SplitSmem {
   static constexpr int kC = D * D * 8;
   static constexpr int kVec = 2 * D * 8;
-  static constexpr int kStage = 2 * kTile * (D + 4) * 4;
+  static constexpr int kStage = 2 * kTile * (D + 4) * 4;  // also the Lanczos scratch
+  static_assert(kStage >= LzScratch<D>::kBytes, "Lanczos scratch exceeds the staging buffer");
   static constexpr int kBytes = kC + kVec + EigScratch<D>::kBytes + kStage + (int)sizeof(SplitScratch) + 64;
 };
 
@@ -959,7 +1313,7 @@ __global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, const
   __syncthreads();
   for (int e = threadIdx.x; e < D * D; e += kThreads) C[e] = src[e] * inv - mu[e / D] * mu[e % D];
   __syncthreads();
-  eigen_top<D>(C, scr, v);
+  leading_eigvec<D>(C, scr, reinterpret_cast<unsigned char*>(stage), v);
   split_node<D>(v, a.X + bh * (size_t)a.nv * D, a.tin + hoff, a.tout + hoff, a.proj + hoff, n, m, c,
                 tree_next, sc);
 }
@@ -994,7 +1348,7 @@ __global__ void __launch_bounds__(kThreads) subtree_kernel(LevelArgs a, int32_t*
       }
       const int n = m * kBlock;
       node_covariance<D>(Xh, tin + hoff, n, stage, C, mu);
-      eigen_top<D>(C, scr, v);
+      leading_eigvec<D>(C, scr, reinterpret_cast<unsigned char*>(stage), v);
       split_node<D>(v, Xh, tin + hoff, tout + hoff, a.proj + hoff, n, m, cc, tree_next, sc);
     }
     __syncthreads();  // the next level reads what this level wrote (same CTA)

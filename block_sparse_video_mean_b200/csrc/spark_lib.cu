@@ -2,6 +2,7 @@
 // every step of the computation runs in the kernels included below. The whole library
 // is this one translation unit.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cmath>
 #include <cstdint>
@@ -21,6 +22,15 @@ using namespace spark;
 namespace {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// An NVTX range around each entry point of the library (host side: the validation and the
+// launches it issues), named after the call; a no-op unless a profiler is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -145,7 +155,8 @@ int launch_attn_tc(const TcParams& tp, const uint16_t* K, const uint16_t* V, con
   if (sms <= 0) return SPARK_ECUDA;
   // one CTA per SM; the 64-query kernel runs two items at a time per CTA
   const int grid = (int)std::min<int64_t>(sms, Q128 ? (int64_t)tp.n_items : ((int64_t)tp.n_items + 1) / 2);
-  auto kern = Q128 ? attn_tc128_kernel<D> : attn_tc_kernel<D>;
+  auto kern = Q128 ? (tp.n_xh > 0 ? attn_tc128_kernel<D, true> : attn_tc128_kernel<D, false>)
+                   : (tp.n_xh > 0 ? attn_tc_kernel<D, true> : attn_tc_kernel<D, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SPARK_ECUDA;
   kern<<<grid, Q128 ? Tc128Cfg<D>::kThreads : TcCfg<D>::kThreads, smem, cs>>>(maps, tp);
@@ -254,6 +265,7 @@ size_t spark_workspace_bytes(const spark_shape* s, int call_id) {
 int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                   int pool_mode, float* q_pool, float* k_pool, float* v_summ, float* beta,
                   float* anchor, void* pool_pack, size_t pool_pack_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_pool_kv");
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   if (pool_mode != SPARK_POOL_REWEIGHT && pool_mode != SPARK_POOL_MEAN) return SPARK_EINVAL;
@@ -311,6 +323,7 @@ size_t spark_extra_pack_bytes(const spark_shape* s, int32_t extra_tokens) {
 int spark_extra_tokens(const spark_shape* s, const uint16_t* K, const uint16_t* V, const float* anchor,
                        int32_t extra_tokens, int pool_mode, float* v_summ, float* beta, void* pool_pack,
                        size_t pool_pack_bytes, void* extra_pack, size_t extra_pack_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_extra_tokens");
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   if (extra_tokens < 0) return SPARK_EINVAL;
@@ -470,6 +483,7 @@ extern "C" {
 int spark_score_select(const spark_shape* s, const float* q_pool, const float* k_pool, int mode,
                        double param, int32_t kcap, int32_t* idx, int32_t* cnt, void* ws,
                        size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_score_select");
   return score_select_impl(s, q_pool, k_pool, mode, param, kcap, idx, cnt, ws, ws_bytes, stream,
                            /*fused=*/false);
 }
@@ -477,6 +491,7 @@ int spark_score_select(const spark_shape* s, const float* q_pool, const float* k
 int spark_score_select_noalloc(const spark_shape* s, const float* q_pool, const float* k_pool,
                                int mode, double param, int32_t kcap, int32_t* idx, int32_t* cnt,
                                void* stream) {
+  NvtxRange nvtx_range("spark_score_select_noalloc");
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   if ((int64_t)s->B * s->H > SPARK_NOALLOC_MAX_HEADS) return SPARK_ESCRATCH;
@@ -491,6 +506,7 @@ int spark_attn_fwd(const spark_shape* s, const uint16_t* Q, const uint16_t* K, c
                    const int32_t* idx, const int32_t* cnt, int32_t kcap, const void* pool_pack,
                    const float* beta, const int32_t* perm, const void* extra_pack, int32_t extra_tokens,
                    uint16_t* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_attn_fwd");
   int st = check_shape(s);
   if (st != SPARK_OK) return st;
   if (extra_tokens < 0) return SPARK_EINVAL;
@@ -590,12 +606,14 @@ extern "C" {
 int spark_reblock(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                   int32_t* perm, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp, int32_t* tree, void* ws,
                   size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_reblock");
   return reblock_impl(s, Q, K, V, perm, nullptr, false, Qp, Kp, Vp, tree, ws, ws_bytes, stream);
 }
 
 int spark_reblock_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                      int32_t* perm_q, int32_t* perm_k, uint16_t* Qp, uint16_t* Kp, uint16_t* Vp,
                      void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("spark_reblock_kv");
   return reblock_impl(s, Q, K, V, perm_q, perm_k, true, Qp, Kp, Vp, nullptr, ws, ws_bytes, stream);
 }
 

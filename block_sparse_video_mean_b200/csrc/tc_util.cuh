@@ -90,6 +90,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same wait by every lane of a warp, with one answer for all of them: the warp leaves
+// converged, as the warp-collective (.sync.aligned) tensor-memory accesses that follow
+// require (lanes leave a polling loop at different times, and a lane that saw the abort
+// flag must not go on alone).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               long long limit = kWaitClocks) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, limit));
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -158,11 +167,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
           smem_addr(bar))
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // 32 lanes x 32 bit, 16 consecutive columns: thread t of the warp gets lane (base + t).
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
       "%15}, [%16];"
@@ -172,6 +188,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) 
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
       "%14,%15,%16};" ::"r"(taddr),
@@ -183,6 +200,7 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
 // threads 16-31 the same lanes at columns c+IMM..c+IMM+15.
 template <int IMM>
 __device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
       "%14,%15}, [%16], %17;"
@@ -191,8 +209,11 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, uint32_t* r
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr), "n"(IMM));
 }
+// Asynchronous form: the source registers must stay untouched until tcgen05.wait::st,
+// which plain C++ cannot guarantee; the kernels use the _sync form above.
 template <int IMM>
 __device__ __forceinline__ void tmem_st_16x32bx2_x16(uint32_t taddr, const uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
       "%13,%14,%15,%16,%17};" ::"r"(taddr),
@@ -201,11 +222,30 @@ __device__ __forceinline__ void tmem_st_16x32bx2_x16(uint32_t taddr, const uint3
       "r"(r[14]), "r"(r[15]));
 }
 
+// Stores fused with their tcgen05.wait::st in one asm statement: tcgen05.st reads its
+// source registers asynchronously, so the compiler must not reuse them (for the next
+// piece's values, say) before the wait; with a separate wait it may, and the tensor memory
+// then receives whatever the registers hold by the time they are read (measured: run-to-run
+// differences of the 128-query kernel after an unrelated code change).
+template <int IMM>
+__device__ __forceinline__ void tmem_st_16x32bx2_x16_sync(uint32_t taddr, const uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "n"(IMM), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+      "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+      "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // Loads fused with their tcgen05.wait::ld in one asm statement: tcgen05.ld writes its
 // destination registers asynchronously, so no compiler-generated move or spill of them
 // may come between the load and the wait.
 template <int IMM>
 __device__ __forceinline__ void tmem_ld_16x32bx2_x16_sync(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;\n\t"
       "tcgen05.wait::ld.sync.aligned;"
@@ -215,6 +255,7 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x16_sync(uint32_t taddr, uint32
 }
 template <int IMM>
 __device__ __forceinline__ void tmem_ld_16x32bx2_x32_sync(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;\n\t"
       "tcgen05.wait::ld.sync.aligned;"
@@ -224,6 +265,7 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x32_sync(uint32_t taddr, uint32
 }
 template <int IMM>
 __device__ __forceinline__ void tmem_ld_16x32bx2_x64_sync(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.16x32bx2.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64], %65;\n\t"
       "tcgen05.wait::ld.sync.aligned;"
@@ -232,6 +274,7 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x64_sync(uint32_t taddr, uint32
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_32x32b_x16_sync(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
@@ -240,6 +283,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16_sync(uint32_t taddr, uint32_t
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_32x32b_x64_sync(uint32_t taddr, uint32_t* r) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
       "tcgen05.wait::ld.sync.aligned;"

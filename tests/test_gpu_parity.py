@@ -142,14 +142,21 @@ def test_batch_and_heads_are_independent(spark):
             compare_head(plan, O, L, Q, K, V, b, h, 9, cfg)
 
 
-def test_repeat_calls_are_bitwise_stable(spark):
-    Q, K, V = make_qkv(1, 2, 64 * 30, 20, 128, seed=2)
-    cfg = spark.ForwardConfig("topk", 0.1, True)
+@pytest.mark.parametrize("q_tile,extra,nv,H", [(64, 0, 64 * 30, 2), (128, 0, 64 * 33 + 17, 5),
+                                                (64, 300, 64 * 30, 2), (128, 300, 64 * 33 + 17, 3),
+                                                (128, 0, 175680, 2), (64, 0, 175680, 2)])
+def test_repeat_calls_are_bitwise_stable(spark, q_tile, extra, nv, H):
+    """Every output is a fixed function of the inputs: no run-to-run differences, whichever
+    CTA a work item lands on (a hazard between an asynchronous TMEM access and the
+    registers it reads or writes shows up here first)."""
+    Q, K, V = make_qkv(1, H, nv, 20, 128, seed=2, device=DEV)
+    cfg = spark.ForwardConfig("topk", 0.1, True, q_tile=q_tile, extra_tokens=extra)
     plan, O, L = run_plan(spark, Q, K, V, 20, cfg)
     O1, L1, idx1 = O.clone(), L.clone(), plan.idx.clone()
-    plan.run(Q.to(DEV), K.to(DEV), V.to(DEV))
-    torch.cuda.synchronize()
-    assert torch.equal(O1, plan.O) and torch.equal(L1, plan.lse) and torch.equal(idx1, plan.idx)
+    for _ in range(3):
+        plan.run(Q, K, V)
+        torch.cuda.synchronize()
+        assert torch.equal(O1, plan.O) and torch.equal(L1, plan.lse) and torch.equal(idx1, plan.idx)
 
 
 # ------------------------------------------------------------------- device-side faults
