@@ -134,10 +134,11 @@ def load_peaks():
 
 
 # DRAM bytes (read + write) of one attention launch: dram__bytes_read.sum +
-# dram__bytes_write.sum from one full-size (24-head) capture of the current kernels
-# (profiles/attn_tc_1152x640x243_launches.md, profiles/attn_tc128_1152x640x243_launches.md).
-# A workload without a capture of its current kernel reports None.
-ATTN_TRAFFIC_BYTES = {"1152x640x243": 106.27e9, "1152x640x243-q128": 30.10e9}
+# dram__bytes_write.sum of the current kernel from one capture at 4 of the 24 heads (items
+# go out head by head, so the traffic grows with the heads), scaled by 24 / 4
+# (profiles/attn_tc_1152x640x243_h4_dram.md). A workload without a capture of its current
+# kernel reports None.
+ATTN_TRAFFIC_BYTES = {"1152x640x243": (13.70267e9 + 0.18733e9) * 6}
 
 
 class ClockSampler:

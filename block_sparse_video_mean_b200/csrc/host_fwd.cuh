@@ -56,9 +56,12 @@ int host_plan(const spark_shape* s, const spark_fwd_config* c, HostPlan* p) {
   // automatic groups carry at least 32 MiB of Q/K/V: large heads go one at a time (a
   // head's K/V then stays in L2 while it is computed), small ones share a copy
   const int64_t head_in = (int64_t)3 * s->N * s->d * 2;
-  const int64_t G = c->heads_per_group > 0
-                        ? c->heads_per_group
-                        : (head_in > 0 ? ((int64_t)1 << 25) / head_in + (((int64_t)1 << 25) % head_in != 0) : 1);
+  int64_t G = c->heads_per_group > 0
+                  ? c->heads_per_group
+                  : (head_in > 0 ? ((int64_t)1 << 25) / head_in + (((int64_t)1 << 25) % head_in != 0) : 1);
+  // Reblock's first levels run one CTA per node and head: a group of one head would leave
+  // most SMs idle there, so automatic groups hold at least 8 heads when it runs
+  if (c->heads_per_group <= 0 && c->reblock != 0) G = std::max<int64_t>(G, 8);
   p->G = (int)std::max<int64_t>(1, std::min<int64_t>(G, std::max<int64_t>(p->bh, 1)));
   p->groups = p->bh == 0 ? 0 : (int)((p->bh + p->G - 1) / p->G);
   const spark_shape g = group_shape(s, p->G);

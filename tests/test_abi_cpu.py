@@ -188,6 +188,9 @@ def test_host_forward_config_and_workspace(spark):
     video = spark.make_shape(1, 24, 175680 + 512, 128, 512)
     assert (spark.forward_host_workspace_bytes(video, spark.fwd_config())
             == spark.forward_host_workspace_bytes(video, spark.fwd_config(heads_per_group=1)))
+    # with Reblock, automatic groups hold at least 8 heads (its first levels need the CTAs)
+    assert (spark.forward_host_workspace_bytes(video, spark.fwd_config(reblock=1))
+            == spark.forward_host_workspace_bytes(video, spark.fwd_config(reblock=1, heads_per_group=8)))
     mid = spark.make_shape(1, 24, 4096, 64, 0)   # 1.5 MiB of Q/K/V per head: 22 heads
     assert (spark.forward_host_workspace_bytes(mid, spark.fwd_config())
             == spark.forward_host_workspace_bytes(mid, spark.fwd_config(heads_per_group=22)))
