@@ -13,13 +13,16 @@
 //   retried with 1e-6 tr(M)/d on the diagonal, identity if that fails too);
 //   x_i = L^T q_i / |L^T q_i| (fp32);
 //   every node of m > 1 blocks: centred covariance of its x (fp64 accumulation), leading
-//   eigenvector v (fp64 Householder tridiagonalisation, Sturm multisection, inverse
-//   iteration), projections x.v signed so their third central moment is >= 0, the
+//   eigenvector v (fp64 Lanczos; Householder tridiagonalisation, Sturm multisection and
+//   inverse iteration when it does not converge), projections x.v signed so their third
+//   central moment is >= 0, the
 //   floor(m/2)*64-th smallest (projection, token) by radix select, stable partition;
 //   leaves ordered by smallest token, tokens ascending; Q/K/V rows gathered.
 // The tree shape depends only on nb, so the host walks it; nodes at most 64 blocks big are
 // split together with their whole subtree by one CTA, larger nodes (the first few levels)
-// accumulate their covariance over many CTAs with fp64 atomics.
+// accumulate their raw moment sums over many CTAs with fp64 atomics: the root and every
+// left child over its tokens, every right child as its parent's sums minus its left
+// sibling's.
 #pragma once
 #include <vector>
 
@@ -731,8 +734,8 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
 // Leading eigenvector by the Lanczos method (Lanczos 1950; the three-term recurrence with
 // one local re-orthogonalisation against the newest vector), with C in registers as in
 // eigen_top. Pass 1 runs the recurrence and checks the top eigenpair (theta, s) of the
-// Lanczos tridiagonal T_n every kLzCheck steps (multisection on Sturm counts, inverse
-// iteration) until the Ritz residual beta_n |s_n| is below kLzTol * theta. Pass 2 runs the
+// Lanczos tridiagonal T_n every kLzCheck steps from kLzFirst on (multisection on Sturm
+// counts, inverse iteration) until the Ritz residual beta_n |s_n| is below kLzTol * theta. Pass 2 runs the
 // same recurrence again from the same start - the same operations in the same order, so
 // the same vectors bit for bit - and sums the Ritz vector v = sum_j s_j q_j in fp64 as it
 // goes, so no basis is stored. The true residual |C v - theta v| is then measured; the call
@@ -741,6 +744,10 @@ __device__ void eigen_top(double* C, double* scr, double* v) {
 // below 1e-9 theta the eigenvector error is below 1e-9 / relative gap: 1e-5 at the 1e-4
 // gap under which a node counts as a tie.
 constexpr int kLzCheck = 16;
+// first check after 48 steps: on whitened covariances (nearly flat spectra) none of 503
+// solves sampled at 1344x768x240 converged in fewer, and a check (a multisection and an
+// inverse iteration) costs as much as about 30 steps
+constexpr int kLzFirst = 3 * kLzCheck;
 constexpr double kLzTol = 1e-12;
 constexpr double kLzAccept = 1e-9;
 
@@ -953,23 +960,38 @@ __device__ bool eigen_top_lanczos(double* C, double* v, unsigned char* work) {
     double r[M], w[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) w[m] = w_out[lane + 32 * m];
-    double t = 0.0;
+    // two reductions per step, each of two sums at once: (q.w, q.q), then (q.r, r.r)
+    double t0 = 0.0, t1 = 0.0;
 #pragma unroll
-    for (int m = 0; m < M; ++m) t = fma(q[m], w[m], t);
-    double alpha = warp_sum_d(t);
+    for (int m = 0; m < M; ++m) {
+      t0 = fma(q[m], w[m], t0);
+      t1 = fma(q[m], q[m], t1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      t0 += __shfl_xor_sync(0xffffffffu, t0, o);
+      t1 += __shfl_xor_sync(0xffffffffu, t1, o);
+    }
+    double alpha = t0;
 #pragma unroll
     for (int m = 0; m < M; ++m) r[m] = w[m] - alpha * q[m] - beta_prev * qp[m];
-    t = 0.0;  // one local re-orthogonalisation against q_j
+    double u0 = 0.0, u1 = 0.0;  // one local re-orthogonalisation against q_j
 #pragma unroll
-    for (int m = 0; m < M; ++m) t = fma(q[m], r[m], t);
-    const double c2 = warp_sum_d(t);
+    for (int m = 0; m < M; ++m) {
+      u0 = fma(q[m], r[m], u0);
+      u1 = fma(r[m], r[m], u1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      u0 += __shfl_xor_sync(0xffffffffu, u0, o);
+      u1 += __shfl_xor_sync(0xffffffffu, u1, o);
+    }
+    const double c2 = u0;
 #pragma unroll
     for (int m = 0; m < M; ++m) r[m] -= c2 * q[m];
     alpha += c2;
-    double bb = 0.0;
-#pragma unroll
-    for (int m = 0; m < M; ++m) bb = fma(r[m], r[m], bb);
-    const double beta = sqrt(warp_sum_d(bb));
+    // |r - c2 q|^2 = r.r - 2 c2 (q.r) + c2^2 (q.q), with q.r = c2
+    const double beta = sqrt(fmax(u1 - c2 * c2 * (2.0 - t1), 0.0));
     const bool invariant = !(beta > 1e-13 * (fabs(alpha) + 1e-300));
     const double inv = invariant ? 0.0 : 1.0 / beta;
     if (warp == 0 && lane == 0) {
@@ -998,7 +1020,7 @@ __device__ bool eigen_top_lanczos(double* C, double* v, unsigned char* work) {
     }
     const bool invariant = step(j);
     n = j + 1;
-    if (invariant || (n >= 2 * kLzCheck && n % kLzCheck == 0) || n == K) {
+    if (invariant || (n >= kLzFirst && n % kLzCheck == 0) || n == K) {
       __syncthreads();  // al / be of step j are written
       theta = tridiag_top_value(al, be, b2, n, red, misc);
       if (tid == 0) {
@@ -1263,18 +1285,21 @@ __device__ __forceinline__ void carve(unsigned char* smem, double** C, double** 
   *sc = reinterpret_cast<SplitScratch*>(smem + S::kC + S::kVec + EigScratch<D>::kBytes + S::kStage);
 }
 
-// Large levels, step 1: covariance sums of every node over chunks of its tokens, fp64
-// atomics into nacc[node][bh] = (S2 [D x D], S1 [D]). grid (nodes * cpn, BH).
+// Large levels, step 1: raw sums of the summed nodes (labels stride * i: every node at the
+// root, the left children below it) over chunks of their tokens, fp64 atomics into
+// nacc[node][bh] = (S2 = sum x x^T [D x D], S1 = sum x [D]). grid (summed nodes * cpn, BH).
+// A left leaf is summed too: its right sibling (3-block parents) needs it.
 template <int D>
-__global__ void __launch_bounds__(kThreads) node_moments_kernel(LevelArgs a, int cpn, double* __restrict__ nacc) {
+__global__ void __launch_bounds__(kThreads) node_moments_kernel(LevelArgs a, int cpn, int stride,
+                                                                double* __restrict__ nacc) {
   extern __shared__ __align__(16) unsigned char smem[];
   double* S2 = reinterpret_cast<double*>(smem);
   double* S1 = S2 + D * D;
   float* stage = reinterpret_cast<float*>(S1 + D);
-  const int c = blockIdx.x / cpn, chunk = blockIdx.x % cpn;
+  const int c = stride * (blockIdx.x / cpn), chunk = blockIdx.x % cpn;
   const size_t bh = blockIdx.y;
   int st, m;
-  if (!node_of(a.nb, a.level, c, &st, &m) || m <= 1) return;
+  if (!node_of(a.nb, a.level, c, &st, &m) || m < 1 || (stride == 1 && m == 1)) return;
   const int t0 = chunk * kChunkTok;
   const int n = min(kChunkTok, m * kBlock - t0);
   if (n <= 0) return;
@@ -1290,7 +1315,8 @@ __global__ void __launch_bounds__(kThreads) node_moments_kernel(LevelArgs a, int
 // Large levels, step 2: one CTA per node finishes the covariance, finds the eigenvector and
 // splits (or carries a leaf). grid (nodes, BH).
 template <int D>
-__global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, const double* __restrict__ nacc) {
+__global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, double* __restrict__ nacc,
+                                                              const double* __restrict__ nacc_up) {
   extern __shared__ __align__(16) unsigned char smem[];
   double *C, *mu, *v, *scr;
   float* stage;
@@ -1307,7 +1333,14 @@ __global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, const
     return;
   }
   const int n = m * kBlock;
-  const double* src = nacc + ((size_t)c * gridDim.y + bh) * (D * D + D);
+  double* src = nacc + ((size_t)c * gridDim.y + bh) * (D * D + D);
+  if (nacc_up != nullptr && (c & 1)) {
+    // a right child: its parent's raw sums minus its left sibling's, kept for its children
+    const double* up = nacc_up + ((size_t)(c >> 1) * gridDim.y + bh) * (D * D + D);
+    const double* left = nacc + ((size_t)(c - 1) * gridDim.y + bh) * (D * D + D);
+    for (int e = threadIdx.x; e < D * D + D; e += kThreads) src[e] = up[e] - left[e];
+    __syncthreads();
+  }
   const double inv = 1.0 / n;
   for (int i = threadIdx.x; i < D; i += kThreads) mu[i] = src[D * D + i] * inv;
   __syncthreads();
@@ -1450,7 +1483,7 @@ struct Plan {
   int levels = 0, first_small = 0;  // levels < first_small use the multi-CTA path
   int max_large_nodes = 0;
   std::vector<int> cpn;             // chunks per node at each large level
-  size_t off_macc, off_lmat, off_x, off_tok0, off_tok1, off_proj, off_nacc, off_mark, off_order, total;
+  size_t off_macc, off_lmat, off_x, off_tok0, off_tok1, off_proj, off_nacc, off_nacc2, off_mark, off_order, total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1481,6 +1514,7 @@ inline Plan make_plan(int bh, int nb, int d) {
   P.off_tok1 = o;  o = align256(o + (size_t)bh * nv * 4);
   P.off_proj = o;  o = align256(o + (size_t)bh * nv * 4);
   P.off_nacc = o;  o = align256(o + (size_t)P.max_large_nodes * bh * ((size_t)d * d + d) * 8);
+  P.off_nacc2 = o; o = align256(o + (size_t)P.max_large_nodes * bh * ((size_t)d * d + d) * 8);
   P.off_mark = o;  o = align256(o + (size_t)bh * nv * 4);
   P.off_order = o; o = align256(o + (size_t)bh * nb * 4);
   P.total = o;
@@ -1512,7 +1546,7 @@ int partition_run(int bh, int N, int nb, const uint16_t* A, const uint16_t* Bm, 
     int32_t* tok0 = reinterpret_cast<int32_t*>(w + P.off_tok0);
     int32_t* tok1 = reinterpret_cast<int32_t*>(w + P.off_tok1);
     float* proj = reinterpret_cast<float*>(w + P.off_proj);
-    double* nacc = reinterpret_cast<double*>(w + P.off_nacc);
+    double* nacc_buf[2] = {reinterpret_cast<double*>(w + P.off_nacc), reinterpret_cast<double*>(w + P.off_nacc2)};
     int32_t* mark = reinterpret_cast<int32_t*>(w + P.off_mark);
     int32_t* order = reinterpret_cast<int32_t*>(w + P.off_order);
     const size_t tree_stride = (size_t)(P.levels + 1) * nv;
@@ -1543,15 +1577,21 @@ int partition_run(int bh, int N, int nb, const uint16_t* A, const uint16_t* Bm, 
     cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
     const int smem_nm = (D * D + D) * 8 + 2 * kTile * (D + 4) * 4;
     cudaFuncSetAttribute(node_moments_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_nm);
+    // level l keeps its nodes' raw sums in nacc_buf[l & 1]; below the root only the left
+    // children are summed over their tokens, a right child's sums are its parent's minus its
+    // left sibling's (node_split_kernel derives and stores them)
     for (int l = 0; l < P.first_small; ++l) {
       a.level = l;
       a.tin = (l & 1) ? tok1 : tok0;
       a.tout = (l & 1) ? tok0 : tok1;
       const int nodes = 1 << l;
+      double* nacc = nacc_buf[l & 1];
+      const double* nacc_up = l > 0 ? nacc_buf[(l - 1) & 1] : nullptr;
       if (cudaMemsetAsync(nacc, 0, (size_t)nodes * bh * ((size_t)D * D + D) * 8, cs) != cudaSuccess)
         return SPARK_ECUDA;
-      node_moments_kernel<D><<<dim3(nodes * P.cpn[l], bh), kThreads, smem_nm, cs>>>(a, P.cpn[l], nacc);
-      node_split_kernel<D><<<dim3(nodes, bh), kThreads, smem_split, cs>>>(a, nacc);
+      const int summed = l > 0 ? nodes / 2 : 1;
+      node_moments_kernel<D><<<dim3(summed * P.cpn[l], bh), kThreads, smem_nm, cs>>>(a, P.cpn[l], l > 0 ? 2 : 1, nacc);
+      node_split_kernel<D><<<dim3(nodes, bh), kThreads, smem_split, cs>>>(a, nacc, nacc_up);
       SPARK_LAUNCH_CHECK();
       note_launches(2);
     }
