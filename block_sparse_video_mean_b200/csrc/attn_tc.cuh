@@ -263,9 +263,14 @@ __global__ void __launch_bounds__(384, 1)
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* ring = smem;
   unsigned char* vring = ring + C::kStages * C::kTileBytes;
+  // [slot][stage]: the stage holds this slot's tile. The two slots' tiles alternate over the
+  // shared stages and an issuer waits only for its own tiles, so with one barrier per stage
+  // its parity wait could be satisfied by the phase of its own previous tile while the other
+  // slot's tile in between is still in flight (copies need not land in issue order); with a
+  // barrier per slot every phase of a barrier is waited for by its one consumer.
   uint64_t* kfull = reinterpret_cast<uint64_t*>(ring + C::kRingBytes);
-  uint64_t* vfull = kfull + C::kStages;
-  uint64_t* kempty = vfull + C::kStages;   // K stage free: its S MMAs completed
+  uint64_t* vfull = kfull + 2 * C::kStages;
+  uint64_t* kempty = vfull + 2 * C::kStages;  // K stage free: its S MMAs completed
   uint64_t* vempty = kempty + C::kStages;  // V stage free: its PV MMAs completed
   uint64_t* sfull = vempty + C::kStages;   // [slot][S buffer]
   uint64_t* pfull = sfull + 4;             // [slot][S buffer]
@@ -286,10 +291,14 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ring + C::kRingBytes + C::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  static_assert((6 * C::kStages + 20 + 4 * kQueueLen) * 8 + 8 + 2 * kQueueLen * 4 <= C::kBarBytes,
+                "barriers, queues and flags exceed their shared-memory region");
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
+    for (int i = 0; i < 2 * C::kStages; ++i) {
       tc::mbar_init(&kfull[i], 1);
       tc::mbar_init(&vfull[i], 1);
+    }
+    for (int i = 0; i < C::kStages; ++i) {
       tc::mbar_init(&kempty[i], 1);
       tc::mbar_init(&vempty[i], 1);
     }
@@ -396,6 +405,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     uint32_t q = 0;
+    uint32_t fc[2 * C::kStages] = {};  // copies issued per (slot, stage) barrier
     while (ok && (have[0] || have[1])) {
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
@@ -433,16 +443,17 @@ __global__ void __launch_bounds__(384, 1)
             // issuing lane and warp, so spreading a tile's boxes over lanes raises the
             // delivery rate (measured on this SM: 22 B/clk with one lane, 31 with four)
             unsigned char* st = rbase + stage * C::kTileBytes;
-            if (lane == 0) tc::mbar_expect_tx(&full[stage], C::kTileBytes);
+            uint64_t* fb = &full[s * C::kStages + stage];
+            if (lane == 0) tc::mbar_expect_tx(fb, C::kTileBytes);
             __syncwarp();
             if (lane < 2 * C::kPanels) {
               const int hf = lane / C::kPanels, pn = lane % C::kPanels;
               const int sk = hf ? src[1] : src[0];
               tc::tma_load_2d(st + pn * C::kPanelBytes + hf * C::kHalfBytes,
-                              sk == 1 ? map_p : (sk == 2 ? map_e : map_x), pn * 64, hf ? y[1] : y[0],
-                              &full[stage]);
+                              sk == 1 ? map_p : (sk == 2 ? map_e : map_x), pn * 64, hf ? y[1] : y[0], fb);
             }
             __syncwarp();
+            ++fc[s * C::kStages + stage];
             ++q;
             if (++t[s] == cur[s].ntiles) {
               t[s] = 0;
@@ -462,9 +473,11 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     if ((!ok || *abort_flag) && lane == 0) {
-      // drain every copy that may still be in flight before the CTA leaves
-      const uint32_t first = q > (uint32_t)C::kStages ? q - C::kStages : 0;
-      for (uint32_t j = first; j < q; ++j) mbar_drain(&full[j % C::kStages], (j / C::kStages) & 1);
+      // drain every copy that may still be in flight before the CTA leaves: the latest
+      // phase of each (slot, stage) barrier (a stage is reused only after its earlier copy
+      // was consumed)
+      for (int i = 0; i < 2 * C::kStages; ++i)
+        if (fc[i] > 0) mbar_drain(&full[i], (fc[i] - 1) & 1);
     }
   } else if (warp == 9 || warp == 11) {
     // ================================================================ MMA issuers
@@ -504,11 +517,13 @@ __global__ void __launch_bounds__(384, 1)
       bool pfirst = false, plast = false;
       const uint32_t ring_addr = tc::smem_addr(ring);
       const uint32_t vring_addr = tc::smem_addr(vring);
+      uint32_t kuse[C::kStages] = {}, vuse[C::kStages] = {};  // this slot's tiles per stage so far
       auto issue_pv = [&]() -> bool {
         const uint32_t b = pg & 1;
         if (!tc::mbar_wait(&pfull[2 * s + b], (pg >> 1) & 1, abort_flag, p.wait_clocks)) return false;
         const int stage = pq % C::kStages;
-        if (!tc::mbar_wait(&vfull[stage], (pq / C::kStages) & 1, abort_flag, p.wait_clocks)) return false;
+        if (!tc::mbar_wait(&vfull[s * C::kStages + stage], vuse[stage]++ & 1, abort_flag, p.wait_clocks))
+          return false;
         if (pfirst && pitem > 0 && !tc::mbar_wait(&ofree[s], (pitem - 1) & 1, abort_flag, p.wait_clocks)) return false;
         tc::tc_fence_after();
         const uint32_t st = vring_addr + stage * C::kTileBytes;
@@ -530,7 +545,8 @@ __global__ void __launch_bounds__(384, 1)
               const uint32_t qb = nitem & 1;
               bool good = t[o] != 0 || tc::mbar_wait(&qfull[2 * s + qb], (nitem >> 1) & 1, abort_flag, p.wait_clocks);
               const int stage = q % C::kStages;
-              good = good && tc::mbar_wait(&kfull[stage], (q / C::kStages) & 1, abort_flag, p.wait_clocks);
+              good = good && tc::mbar_wait(&kfull[s * C::kStages + stage], kuse[stage]++ & 1, abort_flag,
+                                           p.wait_clocks);
               if (!good) {
                 ok = false;
               } else {
