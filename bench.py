@@ -138,7 +138,7 @@ def load_peaks():
 # go out head by head, so the traffic grows with the heads), scaled by 24 / 4
 # (profiles/attn_tc_1152x640x243_h4_dram.md). A workload without a capture of its current
 # kernel reports None.
-ATTN_TRAFFIC_BYTES = {"1152x640x243": (13.70267e9 + 0.18733e9) * 6}
+ATTN_TRAFFIC_BYTES = {"1152x640x243": (4.544962e9 + 0.188276e9) * 6}
 
 
 class ClockSampler:

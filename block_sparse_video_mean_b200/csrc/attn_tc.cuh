@@ -405,7 +405,9 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     uint32_t q = 0;
-    uint32_t fc[2 * C::kStages] = {};  // copies issued per (slot, stage) barrier
+    // per (slot, stage) barrier, bit slot * kStages + stage: a copy was issued on it; the
+    // parity of the number of copies issued on it
+    uint32_t fused = 0, fpar = 0;
     while (ok && (have[0] || have[1])) {
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
@@ -453,7 +455,8 @@ __global__ void __launch_bounds__(384, 1)
                               sk == 1 ? map_p : (sk == 2 ? map_e : map_x), pn * 64, hf ? y[1] : y[0], fb);
             }
             __syncwarp();
-            ++fc[s * C::kStages + stage];
+            fused |= 1u << (s * C::kStages + stage);
+            fpar ^= 1u << (s * C::kStages + stage);
             ++q;
             if (++t[s] == cur[s].ntiles) {
               t[s] = 0;
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(384, 1)
       // phase of each (slot, stage) barrier (a stage is reused only after its earlier copy
       // was consumed)
       for (int i = 0; i < 2 * C::kStages; ++i)
-        if (fc[i] > 0) mbar_drain(&full[i], (fc[i] - 1) & 1);
+        if ((fused >> i) & 1u) mbar_drain(&full[i], ((fpar >> i) & 1u) ^ 1u);
     }
   } else if (warp == 9 || warp == 11) {
     // ================================================================ MMA issuers
@@ -517,13 +520,15 @@ __global__ void __launch_bounds__(384, 1)
       bool pfirst = false, plast = false;
       const uint32_t ring_addr = tc::smem_addr(ring);
       const uint32_t vring_addr = tc::smem_addr(vring);
-      uint32_t kuse[C::kStages] = {}, vuse[C::kStages] = {};  // this slot's tiles per stage so far
+      // parity of this slot's tiles on each stage so far (bit = stage), K and V rings
+      uint32_t kpar = 0, vpar = 0;
       auto issue_pv = [&]() -> bool {
         const uint32_t b = pg & 1;
         if (!tc::mbar_wait(&pfull[2 * s + b], (pg >> 1) & 1, abort_flag, p.wait_clocks)) return false;
         const int stage = pq % C::kStages;
-        if (!tc::mbar_wait(&vfull[s * C::kStages + stage], vuse[stage]++ & 1, abort_flag, p.wait_clocks))
-          return false;
+        const uint32_t vp = (vpar >> stage) & 1u;
+        vpar ^= 1u << stage;
+        if (!tc::mbar_wait(&vfull[s * C::kStages + stage], vp, abort_flag, p.wait_clocks)) return false;
         if (pfirst && pitem > 0 && !tc::mbar_wait(&ofree[s], (pitem - 1) & 1, abort_flag, p.wait_clocks)) return false;
         tc::tc_fence_after();
         const uint32_t st = vring_addr + stage * C::kTileBytes;
@@ -545,8 +550,9 @@ __global__ void __launch_bounds__(384, 1)
               const uint32_t qb = nitem & 1;
               bool good = t[o] != 0 || tc::mbar_wait(&qfull[2 * s + qb], (nitem >> 1) & 1, abort_flag, p.wait_clocks);
               const int stage = q % C::kStages;
-              good = good && tc::mbar_wait(&kfull[s * C::kStages + stage], kuse[stage]++ & 1, abort_flag,
-                                           p.wait_clocks);
+              const uint32_t kp = (kpar >> stage) & 1u;
+              kpar ^= 1u << stage;
+              good = good && tc::mbar_wait(&kfull[s * C::kStages + stage], kp, abort_flag, p.wait_clocks);
               if (!good) {
                 ok = false;
               } else {

@@ -10,7 +10,8 @@
 // which two blocks count as tied). A CTA holds the score rows of RT query blocks in
 // shared memory as order-preserving uint32 keys; one warp per row then finds the k-th
 // largest key by a 4-pass MSB radix select over warp-private 256-bin histograms, and
-// writes the kept indices in ascending order with ballots (ties: lower index first).
+// writes the kept indices with ballots (ties: lower index first) in the row's sweep order
+// (select_sweep_start), which the attention kernels follow.
 #pragma once
 #include "spark_common.cuh"
 #include "tc_util.cuh"
@@ -119,13 +120,27 @@ struct SelectParams {
   int32_t* cnt;
   const double* thr;  // [B*H] (tau mode)
   int nq, nb, kcap, k, mode, rt;  // nq score rows (query blocks or tiles), nb key blocks
+  int sweep;  // query tiles the attention kernel runs at once (0: plain ascending rows)
   float scale;
 };
 
+// Start of row i's sweep order: the kept blocks of a row are written ascending from the
+// first one at or above this position, then wrapping around to the ones below it. The
+// attention kernels visit a row's blocks in the order written, and they run the query
+// tiles of a head in ascending order, `sweep` at a time: as the start position advances
+// by nb / sweep per row, the tiles at work at any moment read K/V near one position of
+// the head, which then stays in L2 for all of them. Multiple of 32 (one warp chunk).
+__host__ __device__ inline int select_sweep_start(int i, int nb, int sweep) {
+  if (sweep <= 0) return 0;
+  return (int)(((long long)(i % sweep) * nb) / sweep) & ~31;
+}
+
 // One warp selects the kept blocks of one score row kr[0 .. nb) (order-preserving keys):
 // top-k by a 4-pass MSB radix select over a warp-private 256-bin histogram h, or the
-// head's tau threshold; writes the ascending indices of the kept blocks to row orow of
-// idx (at most kcap) and their count to cnt[orow].
+// head's tau threshold; writes the indices of the kept blocks to row orow of idx in the
+// row's sweep order (select_sweep_start; at most kcap, the first ones in that order) and
+// their count to cnt[orow]. Ties at the top-k cut go to the lower block indices whatever
+// the order they are written in.
 __device__ __forceinline__ void select_row_warp(const SelectParams& p, const uint32_t* kr,
                                                 size_t bh, size_t orow, uint32_t* h, int lane) {
   const int nb = p.nb;
@@ -188,9 +203,24 @@ __device__ __forceinline__ void select_row_warp(const SelectParams& p, const uin
     T = prefix;
     take_eq = kk;
   }
-  // ---- ascending output pass
-  int written = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < nb; j0 += 32) {
+  // ---- output pass in sweep order: chunks of 32 blocks from the start position to the
+  // end of the row, then from 0. Ties are ranked by block index: the first segment starts
+  // with the ties below the start position counted.
+  const int i_row = (int)(orow - bh * (size_t)p.nq);
+  const int start = select_sweep_start(i_row, nb, p.sweep);
+  const int nch = (nb + 31) / 32;
+  int eq_seen = 0;
+  if (!use_thr) {
+    for (int j0 = 0; j0 < start; j0 += 32) {
+      const int j = j0 + lane;
+      eq_seen += __popc(__ballot_sync(0xffffffffu, j < nb && kr[j] == T));
+    }
+  }
+  int written = 0;
+  for (int c = 0; c < nch; ++c) {
+    int j0 = start + 32 * c;
+    if (j0 >= 32 * nch) j0 -= 32 * nch;
+    if (j0 == 0) eq_seen = 0;  // wrapped (or no rotation): ties ranked from the row start
     const int j = j0 + lane;
     bool keep = false;
     if (use_thr) {

@@ -447,6 +447,9 @@ int score_select_impl(const spark_shape* s, const float* q_pool, const float* k_
   sp.mode = mode;
   sp.rt = rt;
   sp.scale = scale;
+  // query tiles the attention kernel runs at once: one CTA per SM, two 64-query items
+  // per CTA or one 128-query tile
+  sp.sweep = num_sms() * (q_tile_of(s) == 2 * kBlock ? 1 : 2);
   if (!fused) {
     const int nbp = (int)select_row_stride(nb);
     uint32_t* skeys = reinterpret_cast<uint32_t*>(static_cast<unsigned char*>(ws) + select_scores_offset(bh));

@@ -129,9 +129,16 @@ int spark_pool_kv(const spark_shape* s, const uint16_t* Q, const uint16_t* K, co
  *       mu and sigma (population) over all nt*nb scores of the head, obtained in fp64
  *       from the d x d second moments of q_pool and k_pool. No per-row floor: a row
  *       may keep nothing. More than kcap kept blocks truncates the row to its first
- *       kcap indices and records SPARK_ECAPACITY (kcap = nb never overflows).
- * Outputs: idx int32 [B, H, nt, kcap] (per row, ascending block indices in the first
- * cnt slots; later slots unspecified), cnt int32 [B, H, nt].
+ *       kcap indices in the row's order (below) and records SPARK_ECAPACITY (kcap = nb
+ *       never overflows).
+ * Outputs: idx int32 [B, H, nt, kcap], cnt int32 [B, H, nt]. Row i holds its cnt kept
+ * block indices in the first cnt slots (later slots unspecified) in sweep order: ascending
+ * from the first one at or above p_i = floor((i mod W) * nb / W) rounded down to a
+ * multiple of 32, then the ones below p_i, ascending, with W the number of query tiles
+ * spark_attn_fwd runs at once on the current device (2 per SM for q_tile = 64, 1 per SM
+ * for q_tile = 128). spark_attn_fwd visits a row's blocks in the order given (any order is
+ * valid input); in this one the tiles at work at any moment read K/V near one position of
+ * the head. The order changes no kept set: top-k ties still go to the lower indices.
  * The scores are computed by a tiled fp32 kernel into ws and each row is selected from
  * there (per score: even and odd d terms in two fp32 chains, then scaled).
  * ws: spark_workspace_bytes(s, SPARK_CALL_SELECT) bytes, 16-byte aligned (both modes). */

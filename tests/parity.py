@@ -13,10 +13,27 @@ LSE_ABS = 5e-3      # natural-log LSE, |l - r|
 
 
 def gpu_rows(idx, cnt):
-    """List of ascending index arrays from the device's idx/cnt of one head."""
+    """List of ascending index arrays (the kept sets) from the device's idx/cnt of one
+    head; the device writes each row in its sweep order (see sweep_start)."""
     idx = np.asarray(idx)
     cnt = np.asarray(cnt)
-    return [idx[i, : cnt[i]].astype(np.int64) for i in range(cnt.shape[0])]
+    return [np.sort(idx[i, : cnt[i]].astype(np.int64)) for i in range(cnt.shape[0])]
+
+
+def sweep_start(i, nb, sweep):
+    """First block position of row i's sweep order: floor((i mod sweep) * nb / sweep)
+    rounded down to a multiple of 32 (sweep = query tiles the attention kernel runs at
+    once: 2 per SM for 64-query tiles, 1 per SM for 128-query tiles)."""
+    return ((i % sweep) * nb // sweep) & ~31
+
+
+def check_sweep_order(row, i, nb, sweep):
+    """True when a device row lists its kept blocks ascending from the first one at or
+    above sweep_start(i), then the ones below it, ascending."""
+    row = np.asarray(row, dtype=np.int64)
+    s = np.sort(row)
+    st = sweep_start(i, nb, sweep)
+    return np.array_equal(row, np.concatenate([s[s >= st], s[s < st]]))
 
 
 def check_selection_row(gsel, s_row, mode, param, thr=None):

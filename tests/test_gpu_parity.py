@@ -9,7 +9,7 @@ import torch
 
 import oracle.spark_oracle as orc
 from block_sparse_video_mean_b200.inputs import make_qkv
-from tests.parity import (check_lse, check_output, check_selection_row, gpu_rows)
+from tests.parity import (check_lse, check_output, check_selection_row, check_sweep_order, gpu_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +38,13 @@ def head_f64(Q, K, V, b, h):
     return tuple(orc.to_f64(t[b, h]) for t in (Q, K, V))
 
 
+def sweep_width(q_tile):
+    """Query tiles the attention kernel runs at once: 2 per SM (64-query items) or 1 per
+    SM (128-query tiles); the selection writes each row in the sweep order it implies."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    return sms * (1 if q_tile == 128 else 2)
+
+
 def compare_head(plan, O, L, Q, K, V, b, h, ns, cfg, qblocks=None, check_pool=True, dense=True):
     """Compare one head (all or sampled query tiles: blocks, or pairs of blocks on the
     128-query route) against the oracle."""
@@ -55,6 +62,11 @@ def compare_head(plan, O, L, Q, K, V, b, h, ns, cfg, qblocks=None, check_pool=Tr
         np.testing.assert_allclose(gp["v_summ"], P.vtil, atol=2e-5, rtol=0)
         np.testing.assert_allclose(gp["beta"], P.beta, atol=2e-5, rtol=0)
     sel = gpu_rows(plan.idx[b, h].cpu().numpy(), plan.cnt[b, h].cpu().numpy()) if nb else []
+    raw = plan.idx[b, h].cpu().numpy()
+    cnt = plan.cnt[b, h].cpu().numpy()
+    W = sweep_width(qt)
+    for i in (blocks if nb else []):
+        assert check_sweep_order(raw[i, : cnt[i]], i, nb, W), (b, h, i)
     thr = None
     if cfg.mode == "tau" and nb:
         thr = orc.tau_threshold(orc.block_scores(P.qbar, P.kbar, scale), cfg.param)
@@ -153,13 +165,37 @@ def test_repeat_calls_are_bitwise_stable(spark, q_tile, extra, nv, H):
     cfg = spark.ForwardConfig("topk", 0.1, True, q_tile=q_tile, extra_tokens=extra)
     plan, O, L = run_plan(spark, Q, K, V, 20, cfg)
     O1, L1, idx1 = O.clone(), L.clone(), plan.idx.clone()
-    for _ in range(3):
+    # at full length 12 repeats: a ring-barrier hazard of the 64-query kernel (a wait
+    # satisfied by an earlier phase) changed one query block in about 1 run of 6
+    for _ in range(12 if nv > 100_000 else 3):
         plan.run(Q, K, V)
         torch.cuda.synchronize()
         assert torch.equal(O1, plan.O) and torch.equal(L1, plan.lse) and torch.equal(idx1, plan.idx)
 
 
 # ------------------------------------------------------------------- device-side faults
+
+@pytest.mark.parametrize("q_tile", [64, 128])
+@pytest.mark.parametrize("mode,param", [("topk", 0.1), ("topk", 0.5), ("tau", 1.0), ("tau", -0.5)])
+def test_rows_are_written_in_sweep_order(spark, q_tile, mode, param):
+    """Many rows (more than the tiles in flight, so the start position wraps) over many
+    blocks: every row holds the oracle's kept set, ascending from its sweep start and
+    then wrapping, and the forward through that order matches the oracle on sampled tiles."""
+    nb, ns, d = 700, 40, 64
+    Q, K, V = make_qkv(1, 2, nb * 64, ns, d, seed=31)
+    cfg = spark.ForwardConfig(mode, param, True, q_tile=q_tile)
+    plan, O, L = run_plan(spark, Q, K, V, ns, cfg)
+    assert spark.device_error() == 0
+    W = sweep_width(q_tile)
+    starts = set()
+    for h in range(2):
+        raw, cnt = plan.idx[0, h].cpu().numpy(), plan.cnt[0, h].cpu().numpy()
+        for i in range(plan.nt):
+            assert check_sweep_order(raw[i, : cnt[i]], i, nb, W), (h, i)
+            starts.add(((i % W) * nb // W) & ~31)
+        compare_head(plan, O, L, Q, K, V, 0, h, ns, cfg, qblocks=sample_blocks(plan.nt, 12, h))
+    assert len(starts) > 8                     # the rows really are rotated
+
 
 def test_out_of_range_index_is_skipped_and_reported(spark):
     Q, K, V = make_qkv(1, 1, 64 * 8, 8, 64, seed=3)
