@@ -1150,17 +1150,14 @@ __device__ uint32_t radix_select(int n, int r, KeyF key, FiltF filt, SplitScratc
   return prefix;
 }
 
-// Splits one node of m > 1 blocks (n = 64 m tokens): projections on v (fp64 dot products,
-// stored as fp32), sign from the third central moment, the floor(m/2)*64-th smallest
-// (projection, token) and a stable partition of tin into tout (left part first). Writes
-// the children's labels 2c / 2c + 1 into tree_next when it is not null.
+// Projections proj[i] = x[tin[i]] . v of n tokens (fp64 dot products, stored as fp32) by
+// the CTA; returns the thread's share of their fp64 sum. 8 lanes per token, 4 tokens per
+// warp at a time (PL = D / 8 components per lane, as float4 loads), so each warp keeps
+// several row gathers in flight.
 template <int D>
-__device__ void split_node(const double* v, const float* __restrict__ Xh, const int32_t* tin,
-                           int32_t* tout, float* proj, int n, int m, int label,
-                           int32_t* tree_next, SplitScratch* sc) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // projections: 8 lanes per token, 4 tokens per warp at a time (PL = D / 8 components
-  // per lane, as float4 loads), so each warp keeps several row gathers in flight
+__device__ double project_tokens(const double* v, const float* __restrict__ Xh, const int32_t* tin,
+                                 float* proj, int n) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int PL = D / 8;
   const int sub = lane >> 3, sl = lane & 7;
   double vl[PL];
@@ -1188,8 +1185,16 @@ __device__ void split_node(const double* v, const float* __restrict__ Xh, const 
       psum += d;
     }
   }
-  __syncthreads();
-  const double pbar = block_sum_d(psum, sc->red) / n;
+  return psum;
+}
+
+// Splits one node of m > 1 blocks (n = 64 m tokens) whose projections are in proj and
+// whose projection mean is pbar: sign from the third central moment, the floor(m/2)*64-th
+// smallest (projection, token) and a stable partition of tin into tout (left part first).
+// Writes the children's labels 2c / 2c + 1 into tree_next when it is not null.
+__device__ void split_projected(const int32_t* tin, int32_t* tout, const float* proj, double pbar, int n,
+                                int m, int label, int32_t* tree_next, SplitScratch* sc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   double m3 = 0.0;
   for (int i = tid; i < n; i += kThreads) {
     const double c = (double)proj[i] - pbar;
@@ -1241,6 +1246,17 @@ __device__ void split_node(const double* v, const float* __restrict__ Xh, const 
     nl_base += total;
   }
   __syncthreads();
+}
+
+// Projections on v by the CTA, then the split (small nodes: one CTA does both).
+template <int D>
+__device__ void split_node(const double* v, const float* __restrict__ Xh, const int32_t* tin,
+                           int32_t* tout, float* proj, int n, int m, int label,
+                           int32_t* tree_next, SplitScratch* sc) {
+  const double psum = project_tokens<D>(v, Xh, tin, proj, n);
+  __syncthreads();
+  const double pbar = block_sum_d(psum, sc->red) / n;
+  split_projected(tin, tout, proj, pbar, n, m, label, tree_next, sc);
 }
 
 // A leaf carried to the next level: same tokens, label 2c.
@@ -1312,11 +1328,13 @@ __global__ void __launch_bounds__(kThreads) node_moments_kernel(LevelArgs a, int
   for (int i = threadIdx.x; i < D * D + D; i += kThreads) atomicAdd(dst + i, S2[i]);
 }
 
-// Large levels, step 2: one CTA per node finishes the covariance, finds the eigenvector and
-// splits (or carries a leaf). grid (nodes, BH).
+// Large levels, step 2: one CTA per node finishes the covariance (a right child's sums are
+// its parent's minus its left sibling's; they are kept for its children) and writes the
+// leading eigenvector to vbuf[node][bh]. grid (nodes, BH).
 template <int D>
-__global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, double* __restrict__ nacc,
-                                                              const double* __restrict__ nacc_up) {
+__global__ void __launch_bounds__(kThreads) node_eig_kernel(LevelArgs a, double* __restrict__ nacc,
+                                                            const double* __restrict__ nacc_up,
+                                                            double* __restrict__ vbuf) {
   extern __shared__ __align__(16) unsigned char smem[];
   double *C, *mu, *v, *scr;
   float* stage;
@@ -1325,17 +1343,10 @@ __global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, doubl
   const int c = blockIdx.x;
   const size_t bh = blockIdx.y;
   int st, m;
-  if (!node_of(a.nb, a.level, c, &st, &m)) return;
-  const size_t hoff = bh * (size_t)a.nv + st * kBlock;
-  int32_t* tree_next = a.tree ? a.tree + bh * (size_t)(a.levels + 1) * a.nv + (size_t)(a.level + 1) * a.nv : nullptr;
-  if (m == 1) {
-    carry_leaf(a.tin + hoff, a.tout + hoff, c, tree_next);
-    return;
-  }
+  if (!node_of(a.nb, a.level, c, &st, &m) || m == 1) return;
   const int n = m * kBlock;
   double* src = nacc + ((size_t)c * gridDim.y + bh) * (D * D + D);
   if (nacc_up != nullptr && (c & 1)) {
-    // a right child: its parent's raw sums minus its left sibling's, kept for its children
     const double* up = nacc_up + ((size_t)(c >> 1) * gridDim.y + bh) * (D * D + D);
     const double* left = nacc + ((size_t)(c - 1) * gridDim.y + bh) * (D * D + D);
     for (int e = threadIdx.x; e < D * D + D; e += kThreads) src[e] = up[e] - left[e];
@@ -1347,8 +1358,47 @@ __global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a, doubl
   for (int e = threadIdx.x; e < D * D; e += kThreads) C[e] = src[e] * inv - mu[e / D] * mu[e % D];
   __syncthreads();
   leading_eigvec<D>(C, scr, reinterpret_cast<unsigned char*>(stage), v);
-  split_node<D>(v, a.X + bh * (size_t)a.nv * D, a.tin + hoff, a.tout + hoff, a.proj + hoff, n, m, c,
-                tree_next, sc);
+  double* vout = vbuf + ((size_t)c * gridDim.y + bh) * D;
+  for (int i = threadIdx.x; i < D; i += kThreads) vout[i] = v[i];
+}
+
+// Large levels, step 3: projections of every node's tokens on its eigenvector, in chunks of
+// kChunkTok tokens per CTA (one CTA per node would keep too few row gathers in flight for
+// the 10^5 tokens of a top-level node). grid (nodes * cpn, BH).
+template <int D>
+__global__ void __launch_bounds__(kThreads) node_project_kernel(LevelArgs a, int cpn, const double* __restrict__ vbuf) {
+  const int c = blockIdx.x / cpn, chunk = blockIdx.x % cpn;
+  const size_t bh = blockIdx.y;
+  int st, m;
+  if (!node_of(a.nb, a.level, c, &st, &m) || m == 1) return;
+  const int t0 = chunk * kChunkTok;
+  const int n = min(kChunkTok, m * kBlock - t0);
+  if (n <= 0) return;
+  const size_t hoff = bh * (size_t)a.nv + st * kBlock + t0;
+  project_tokens<D>(vbuf + ((size_t)c * gridDim.y + bh) * D, a.X + bh * (size_t)a.nv * D, a.tin + hoff,
+                    a.proj + hoff, n);
+}
+
+// Large levels, step 4: one CTA per node splits it from its projections (or carries a
+// leaf). grid (nodes, BH).
+__global__ void __launch_bounds__(kThreads) node_split_kernel(LevelArgs a) {
+  __shared__ SplitScratch sc;
+  const int c = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  int st, m;
+  if (!node_of(a.nb, a.level, c, &st, &m)) return;
+  const size_t hoff = bh * (size_t)a.nv + st * kBlock;
+  int32_t* tree_next = a.tree ? a.tree + bh * (size_t)(a.levels + 1) * a.nv + (size_t)(a.level + 1) * a.nv : nullptr;
+  if (m == 1) {
+    carry_leaf(a.tin + hoff, a.tout + hoff, c, tree_next);
+    return;
+  }
+  const int n = m * kBlock;
+  const float* proj = a.proj + hoff;
+  double psum = 0.0;
+  for (int i = threadIdx.x; i < n; i += kThreads) psum += (double)proj[i];
+  const double pbar = block_sum_d(psum, sc.red) / n;
+  split_projected(a.tin + hoff, a.tout + hoff, proj, pbar, n, m, c, tree_next, &sc);
 }
 
 // Small nodes: one CTA per node of level `level` splits it and its whole subtree down to
@@ -1483,7 +1533,8 @@ struct Plan {
   int levels = 0, first_small = 0;  // levels < first_small use the multi-CTA path
   int max_large_nodes = 0;
   std::vector<int> cpn;             // chunks per node at each large level
-  size_t off_macc, off_lmat, off_x, off_tok0, off_tok1, off_proj, off_nacc, off_nacc2, off_mark, off_order, total;
+  size_t off_macc, off_lmat, off_x, off_tok0, off_tok1, off_proj, off_nacc, off_nacc2, off_vbuf, off_mark, off_order,
+      total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1515,6 +1566,7 @@ inline Plan make_plan(int bh, int nb, int d) {
   P.off_proj = o;  o = align256(o + (size_t)bh * nv * 4);
   P.off_nacc = o;  o = align256(o + (size_t)P.max_large_nodes * bh * ((size_t)d * d + d) * 8);
   P.off_nacc2 = o; o = align256(o + (size_t)P.max_large_nodes * bh * ((size_t)d * d + d) * 8);
+  P.off_vbuf = o;  o = align256(o + (size_t)P.max_large_nodes * bh * d * 8);
   P.off_mark = o;  o = align256(o + (size_t)bh * nv * 4);
   P.off_order = o; o = align256(o + (size_t)bh * nb * 4);
   P.total = o;
@@ -1547,6 +1599,7 @@ int partition_run(int bh, int N, int nb, const uint16_t* A, const uint16_t* Bm, 
     int32_t* tok1 = reinterpret_cast<int32_t*>(w + P.off_tok1);
     float* proj = reinterpret_cast<float*>(w + P.off_proj);
     double* nacc_buf[2] = {reinterpret_cast<double*>(w + P.off_nacc), reinterpret_cast<double*>(w + P.off_nacc2)};
+    double* vbuf = reinterpret_cast<double*>(w + P.off_vbuf);
     int32_t* mark = reinterpret_cast<int32_t*>(w + P.off_mark);
     int32_t* order = reinterpret_cast<int32_t*>(w + P.off_order);
     const size_t tree_stride = (size_t)(P.levels + 1) * nv;
@@ -1573,13 +1626,14 @@ int partition_run(int bh, int N, int nb, const uint16_t* A, const uint16_t* Bm, 
     a.nb = nb;
     a.levels = P.levels;
     const int smem_split = SplitSmem<D>::kBytes;
-    cudaFuncSetAttribute(node_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
+    cudaFuncSetAttribute(node_eig_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
     cudaFuncSetAttribute(subtree_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_split);
     const int smem_nm = (D * D + D) * 8 + 2 * kTile * (D + 4) * 4;
     cudaFuncSetAttribute(node_moments_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_nm);
     // level l keeps its nodes' raw sums in nacc_buf[l & 1]; below the root only the left
     // children are summed over their tokens, a right child's sums are its parent's minus its
-    // left sibling's (node_split_kernel derives and stores them)
+    // left sibling's (node_eig_kernel derives and stores them); then the eigenvectors (one
+    // CTA per node), the projections (many CTAs per node) and the splits (one CTA per node)
     for (int l = 0; l < P.first_small; ++l) {
       a.level = l;
       a.tin = (l & 1) ? tok1 : tok0;
@@ -1591,9 +1645,11 @@ int partition_run(int bh, int N, int nb, const uint16_t* A, const uint16_t* Bm, 
         return SPARK_ECUDA;
       const int summed = l > 0 ? nodes / 2 : 1;
       node_moments_kernel<D><<<dim3(summed * P.cpn[l], bh), kThreads, smem_nm, cs>>>(a, P.cpn[l], l > 0 ? 2 : 1, nacc);
-      node_split_kernel<D><<<dim3(nodes, bh), kThreads, smem_split, cs>>>(a, nacc, nacc_up);
+      node_eig_kernel<D><<<dim3(nodes, bh), kThreads, smem_split, cs>>>(a, nacc, nacc_up, vbuf);
+      node_project_kernel<D><<<dim3(nodes * P.cpn[l], bh), kThreads, 0, cs>>>(a, P.cpn[l], vbuf);
+      node_split_kernel<<<dim3(nodes, bh), kThreads, 0, cs>>>(a);
       SPARK_LAUNCH_CHECK();
-      note_launches(2);
+      note_launches(4);
     }
     if (P.first_small < P.levels) {
       a.level = P.first_small;
