@@ -86,8 +86,12 @@ __device__ __forceinline__ double block_sum_d(double v, double* red) {
 
 // ------------------------------------------------------------------ second moments
 // Adds sum over `rows` of r r^T (and sum of r when S1 != nullptr) into fp64 accumulators
-// held in shared memory (S2: D x D, S1: D). Rows are staged 64 at a time as fp32; each
-// thread owns an (D/16) x (D/16) sub-block, sums a tile in fp32, then adds it in fp64.
+// held in shared memory (S2: D x D, S1: D). Rows are staged 64 at a time as fp32; thread
+// (ti, tj) owns rows ti (D/16) .. + D/16 - 1 and columns tj + 16 b of S2, sums a tile in
+// fp32, then adds it in fp64: consecutive tj touch consecutive doubles, so the fp64
+// read-modify-writes are free of bank conflicts (a contiguous column block would put the
+// 16 tj of a warp 8 doubles apart). Each element sums the same products in the same order
+// whichever thread owns it.
 // `load_row(i, dst)` writes row i (0 <= i < n) as D floats into dst.
 template <int D, class LoadRow>
 __device__ void accumulate_moments(int n, LoadRow load_row, float* stage, double* S2, double* S1) {
@@ -118,7 +122,7 @@ __device__ void accumulate_moments(int n, LoadRow load_row, float* stage, double
 #pragma unroll
       for (int a = 0; a < S; ++a) {
         xa[a] = row[ti * S + a];
-        xb[a] = row[tj * S + a];
+        xb[a] = row[tj + 16 * a];
       }
 #pragma unroll
       for (int a = 0; a < S; ++a)
@@ -128,7 +132,7 @@ __device__ void accumulate_moments(int n, LoadRow load_row, float* stage, double
 #pragma unroll
     for (int a = 0; a < S; ++a)
 #pragma unroll
-      for (int b = 0; b < S; ++b) S2[(ti * S + a) * D + tj * S + b] += (double)acc[a][b];
+      for (int b = 0; b < S; ++b) S2[(ti * S + a) * D + tj + 16 * b] += (double)acc[a][b];
     if (S1 != nullptr && tid < D) {
       float cs = 0.f;
       for (int r = 0; r < kTile; ++r) cs += stage[r * LD + tid];
@@ -186,10 +190,10 @@ __device__ void accumulate_moments_rows(int n, RowPtr row_ptr, float* stage, dou
 #pragma unroll
       for (int a = 0; a < S; a += 4) {
         const float4 va = *reinterpret_cast<const float4*>(row + ti * S + a);
-        const float4 vb = *reinterpret_cast<const float4*>(row + tj * S + a);
         xa[a] = va.x; xa[a + 1] = va.y; xa[a + 2] = va.z; xa[a + 3] = va.w;
-        xb[a] = vb.x; xb[a + 1] = vb.y; xb[a + 2] = vb.z; xb[a + 3] = vb.w;
       }
+#pragma unroll
+      for (int b = 0; b < S; ++b) xb[b] = row[tj + 16 * b];
 #pragma unroll
       for (int a = 0; a < S; ++a)
 #pragma unroll
@@ -198,7 +202,7 @@ __device__ void accumulate_moments_rows(int n, RowPtr row_ptr, float* stage, dou
 #pragma unroll
     for (int a = 0; a < S; ++a)
 #pragma unroll
-      for (int b = 0; b < S; ++b) S2[(ti * S + a) * D + tj * S + b] += (double)acc[a][b];
+      for (int b = 0; b < S; ++b) S2[(ti * S + a) * D + tj + 16 * b] += (double)acc[a][b];
     if (S1 != nullptr && tid < D) {
       float cs = 0.f;
       for (int r = 0; r < kTile; ++r) cs += cur[r * LD + tid];
