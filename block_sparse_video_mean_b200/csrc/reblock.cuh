@@ -836,52 +836,77 @@ __device__ double tridiag_top_value(const double* a, const double* e, const doub
 
 // Unit eigenvector y of the n x n tridiagonal (a, e) at the eigenvalue theta by two steps
 // of inverse iteration (LU with partial pivoting, Newton-refined reciprocals); one thread.
+// The factorisation and both solves carry their recurrences in registers (the next pivot,
+// the next superdiagonal entry, the neighbouring solution entries) and keep in shared
+// memory only what a later pass reads, so no step waits on a shared-memory round trip;
+// the operations and their order are those of the plain LAPACK-style loops.
 __device__ void tridiag_inverse_iteration(const double* a, const double* e, int n, double theta,
                                           double* dd, double* du, double* du2, double* dl, int* piv,
                                           double* y) {
   const double tiny = 1e-30 * (fabs(theta) + 1e-300);
-  for (int i = 0; i < n; ++i) {
-    dd[i] = a[i] - theta;
-    if (i < n - 1) dl[i] = du[i] = e[i];
-    du2[i] = 0.0;
-  }
+  // factorisation: dd holds the reciprocals of the pivots
+  double d0 = a[0] - theta;               // pivot candidate of row i
+  double u0 = n > 1 ? e[0] : 0.0;         // superdiagonal entry of row i
   for (int i = 0; i < n - 1; ++i) {
-    if (fabs(dd[i]) >= fabs(dl[i])) {
-      if (dd[i] == 0.0) dd[i] = tiny;
-      const double f = dl[i] * rcp_nr(dd[i]);
+    const double li = e[i];               // subdiagonal entry below row i
+    const double dn = a[i + 1] - theta;   // diagonal of row i + 1
+    const double un = i < n - 2 ? e[i + 1] : 0.0;  // superdiagonal of row i + 1
+    if (fabs(d0) >= fabs(li)) {
+      if (d0 == 0.0) d0 = tiny;
+      const double r = rcp_nr(d0);
+      const double f = li * r;
+      dd[i] = r;
       dl[i] = f;
-      dd[i + 1] -= f * du[i];
+      du[i] = u0;
+      du2[i] = 0.0;
       piv[i] = 0;
+      d0 = dn - f * u0;
+      u0 = un;
     } else {
-      const double f = dd[i] * rcp_nr(dl[i]);
-      dd[i] = dl[i];
+      const double r = rcp_nr(li);
+      const double f = d0 * r;
+      dd[i] = r;
       dl[i] = f;
-      const double tmp = du[i];
-      du[i] = dd[i + 1];
-      dd[i + 1] = tmp - f * dd[i + 1];
-      if (i < n - 2) {
-        du2[i] = du[i + 1];
-        du[i + 1] = -f * du[i + 1];
-      }
+      du[i] = dn;
+      du2[i] = un;
       piv[i] = 1;
+      d0 = u0 - f * dn;
+      u0 = -f * un;
     }
   }
-  if (dd[n - 1] == 0.0) dd[n - 1] = tiny;
-  for (int i = 0; i < n; ++i) dd[i] = rcp_nr(dd[i]);
+  if (d0 == 0.0) d0 = tiny;
+  dd[n - 1] = rcp_nr(d0);
   for (int i = 0; i < n; ++i) y[i] = 1.0 + 0.001 * i;
   for (int it = 0; it < 2; ++it) {
+    // forward: apply the row interchanges and L^-1; yi carries y[i]
+    double yi = y[0];
     for (int i = 0; i < n - 1; ++i) {
+      const double yn = y[i + 1];
       if (piv[i] == 0) {
-        y[i + 1] -= dl[i] * y[i];
+        y[i] = yi;
+        yi = yn - dl[i] * yi;
       } else {
-        const double tmp = y[i] - dl[i] * y[i + 1];
-        y[i] = y[i + 1];
-        y[i + 1] = tmp;
+        y[i] = yn;
+        yi = yi - dl[i] * yn;
       }
     }
-    y[n - 1] *= dd[n - 1];
-    if (n >= 2) y[n - 2] = (y[n - 2] - du[n - 2] * y[n - 1]) * dd[n - 2];
-    for (int i = n - 3; i >= 0; --i) y[i] = (y[i] - du[i] * y[i + 1] - du2[i] * y[i + 2]) * dd[i];
+    y[n - 1] = yi;
+    // back substitution with U (diagonal reciprocals dd, superdiagonals du, du2)
+    double y1 = y[n - 1] * dd[n - 1];      // y[i + 1]
+    y[n - 1] = y1;
+    double y2 = 0.0;                        // y[i + 2]
+    if (n >= 2) {
+      const double t = (y[n - 2] - du[n - 2] * y1) * dd[n - 2];
+      y[n - 2] = t;
+      y2 = y1;
+      y1 = t;
+    }
+    for (int i = n - 3; i >= 0; --i) {
+      const double t = (y[i] - du[i] * y1 - du2[i] * y2) * dd[i];
+      y[i] = t;
+      y2 = y1;
+      y1 = t;
+    }
     double nn = 0.0;
     for (int i = 0; i < n; ++i) nn += y[i] * y[i];
     const double inv = 1.0 / sqrt(nn);
