@@ -9,9 +9,10 @@
 // pipe: a bf16/tf32 product would move scores by ~1e-3, far beyond the 1e-4 window in
 // which two blocks count as tied). A CTA holds the score rows of RT query blocks in
 // shared memory as order-preserving uint32 keys; one warp per row then finds the k-th
-// largest key by a 4-pass MSB radix select over warp-private 256-bin histograms, and
-// writes the kept indices with ballots (ties: lower index first) in the row's sweep order
-// (select_sweep_start), which the attention kernels follow.
+// largest key from a warp-private 256-bin histogram of the row's values between its
+// minimum and maximum and an exact ranking of the cut bin's keys (a 4-pass MSB radix select
+// where that does not apply), and writes the kept indices with ballots (ties: lower index
+// first) in the row's sweep order (select_sweep_start), which the attention kernels follow.
 #pragma once
 #include "spark_common.cuh"
 #include "tc_util.cuh"
@@ -135,12 +136,164 @@ __host__ __device__ inline int select_sweep_start(int i, int nb, int sweep) {
   return (int)(((long long)(i % sweep) * nb) / sweep) & ~31;
 }
 
+// The bin of the 256-bin histogram h in which the count from the top reaches kk (1 <= kk
+// <= the histogram's total), the count in the bins above it and the bin's own count; every
+// lane gets all three. Lane l scans bins 255 - 8l .. 248 - 8l.
+__device__ __forceinline__ void top_bin(const uint32_t* h, int kk, int lane, int* bin_out,
+                                        int* above_out, uint32_t* count_out) {
+  uint32_t cntb[8];
+  uint32_t tot = 0;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    cntb[t] = h[255 - 8 * lane - t];
+    tot += cntb[t];
+  }
+  uint32_t incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const uint32_t excl = incl - tot;
+  const bool mine = excl < (uint32_t)kk && (uint32_t)kk <= incl;
+  const uint32_t who = __ballot_sync(0xffffffffu, mine);
+  const int src = __ffs(who) - 1;
+  int bin = 0, above = 0;
+  uint32_t c = 0;
+  if (lane == src) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (run + cntb[t] >= (uint32_t)kk) {
+        bin = 255 - 8 * lane - t;
+        above = (int)run;
+        c = cntb[t];
+        break;
+      }
+      run += cntb[t];
+    }
+  }
+  *bin_out = __shfl_sync(0xffffffffu, bin, src);
+  *above_out = __shfl_sync(0xffffffffu, above, src);
+  *count_out = __shfl_sync(0xffffffffu, c, src);
+}
+
+// The top-k cut of the row kr[0 .. nb): its k-th largest key T and the number of keys
+// equal to T that the top k keep (k minus the keys above T), by a 4-pass MSB radix select
+// over the warp's 256-bin histogram h.
+__device__ __forceinline__ void radix_cut(const uint32_t* kr, int nb, int k, uint32_t* h, int lane,
+                                          uint32_t* T_out, int* take_out) {
+  uint32_t prefix = 0, mask = 0;
+  int kk = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = lane; b < 256; b += 32) h[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < nb; j += 32) {
+      const uint32_t key = kr[j];
+      if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    int bin, above;
+    uint32_t c;
+    top_bin(h, kk, lane, &bin, &above, &c);
+    kk -= above;
+    prefix |= (uint32_t)bin << shift;
+    mask |= 255u << shift;
+    __syncwarp();
+  }
+  *T_out = prefix;
+  *take_out = kk;
+}
+
+// The same cut from value bins, in one histogram pass instead of four: the row's scores are
+// binned over [min, max] into 256 equal-width bins, bin(v) = min(floor((v - min) * 256 /
+// (max - min)), 255) in fp32 with every operation rounded to nearest, which never
+// decreases as the key grows, so every key in a bin above the cut bin lies above T. The
+// cut bin's keys (a dozen or two on Gaussian-like rows; the radix select's first pass, on
+// the sign and exponent bits, puts most of a row into two or three bins and serialises
+// the warp's atomics) are gathered into h and ranked exactly. Returns false, with no
+// result, when the row's range is not finite and positive or the cut bin holds more than
+// 256 keys (many equal scores); the caller then runs radix_cut.
+__device__ __forceinline__ bool binned_cut(const uint32_t* kr, int nb, int k, uint32_t* h, int lane,
+                                           uint32_t* T_out, int* take_out) {
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int j = lane; j < nb; j += 32) {
+    const uint32_t key = kr[j];
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  const float vmin = key_to_float(kmin), vmax = key_to_float(kmax);
+  const float range = __fsub_rn(vmax, vmin);
+  const float inv = __fdiv_rn(256.f, range);
+  if (!(isfinite(vmin) && isfinite(vmax) && range > 0.f && isfinite(range) && isfinite(inv)))
+    return false;
+  auto bin_of = [&](uint32_t key) -> int {
+    const float t = __fmul_rn(__fsub_rn(key_to_float(key), vmin), inv);  // in [0, 256]
+    return min((int)t, 255);
+  };
+  for (int b = lane; b < 256; b += 32) h[b] = 0;
+  __syncwarp();
+  for (int j = lane; j < nb; j += 32) atomicAdd(&h[bin_of(kr[j])], 1u);
+  __syncwarp();
+  int bin, above;
+  uint32_t cst;
+  top_bin(h, k, lane, &bin, &above, &cst);
+  __syncwarp();  // every lane has read h
+  if (cst > 256u) return false;
+  // the cut bin's keys to h[0 .. cst), in row order
+  int base = 0;
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < nb ? kr[j] : 0u;
+    const bool in = j < nb && bin_of(key) == bin;
+    const uint32_t m = __ballot_sync(0xffffffffu, in);
+    const int pos = base + __popc(m & lanemask_lt());
+    if (in && pos < 256) h[pos] = key;
+    base += __popc(m);
+  }
+  __syncwarp();
+  // the candidate x with #(candidates > x) < kk <= #(candidates >= x) is T
+  const int kk = k - above;  // 1 <= kk <= cst
+  bool found = false;
+  uint32_t T = 0;
+  int take = 0;
+  for (int i0 = 0; i0 < (int)cst; i0 += 32) {
+    const int i = i0 + lane;
+    uint32_t x = 0;
+    int g = 0, e = 0;
+    if (i < (int)cst) {
+      x = h[i];
+      for (int t = 0; t < (int)cst; ++t) {
+        const uint32_t y = h[t];
+        g += y > x ? 1 : 0;
+        e += y >= x ? 1 : 0;
+      }
+    }
+    const uint32_t hm = __ballot_sync(0xffffffffu, i < (int)cst && g < kk && kk <= e);
+    if (hm) {
+      const int src = __ffs(hm) - 1;
+      T = __shfl_sync(0xffffffffu, x, src);
+      take = kk - __shfl_sync(0xffffffffu, g, src);
+      found = true;
+      break;
+    }
+  }
+  __syncwarp();  // h is read before the caller reuses it
+  if (!found) return false;
+  *T_out = T;
+  *take_out = take;
+  return true;
+}
+
 // One warp selects the kept blocks of one score row kr[0 .. nb) (order-preserving keys):
-// top-k by a 4-pass MSB radix select over a warp-private 256-bin histogram h, or the
-// head's tau threshold; writes the indices of the kept blocks to row orow of idx in the
-// row's sweep order (select_sweep_start; at most kcap, the first ones in that order) and
-// their count to cnt[orow]. Ties at the top-k cut go to the lower block indices whatever
-// the order they are written in.
+// top-k by the cut of binned_cut (radix_cut where that declines), or the head's tau
+// threshold; writes the indices of the kept blocks to row orow of idx in the row's sweep
+// order (select_sweep_start; at most kcap, the first ones in that order) and their count
+// to cnt[orow]. Ties at the top-k cut go to the lower block indices whatever the order they
+// are written in.
 __device__ __forceinline__ void select_row_warp(const SelectParams& p, const uint32_t* kr,
                                                 size_t bh, size_t orow, uint32_t* h, int lane) {
   const int nb = p.nb;
@@ -150,58 +303,7 @@ __device__ __forceinline__ void select_row_warp(const SelectParams& p, const uin
   const bool use_thr = (p.mode == SPARK_SELECT_TAU);
   const double thr = use_thr ? p.thr[bh] : 0.0;
   if (!use_thr) {
-    uint32_t prefix = 0, mask = 0;
-    int kk = p.k;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int b = lane; b < 256; b += 32) h[b] = 0;
-      __syncwarp();
-      for (int j = lane; j < nb; j += 32) {
-        const uint32_t key = kr[j];
-        if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
-      }
-      __syncwarp();
-      // lane l owns bins 255-8l .. 248-8l (descending); find the bin where the count
-      // from the top reaches kk.
-      uint32_t cntb[8];
-      uint32_t tot = 0;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        cntb[t] = h[255 - 8 * lane - t];
-        tot += cntb[t];
-      }
-      uint32_t incl = tot;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      const uint32_t excl = incl - tot;
-      const bool mine = excl < (uint32_t)kk && (uint32_t)kk <= incl;
-      const uint32_t who = __ballot_sync(0xffffffffu, mine);
-      const int src = __ffs(who) - 1;
-      int bin = 0, above = 0;
-      if (lane == src) {
-        uint32_t run = excl;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          if (run + cntb[t] >= (uint32_t)kk) {
-            bin = 255 - 8 * lane - t;
-            above = (int)run;
-            break;
-          }
-          run += cntb[t];
-        }
-      }
-      bin = __shfl_sync(0xffffffffu, bin, src);
-      above = __shfl_sync(0xffffffffu, above, src);
-      kk -= above;
-      prefix |= (uint32_t)bin << shift;
-      mask |= 255u << shift;
-      __syncwarp();
-    }
-    T = prefix;
-    take_eq = kk;
+    if (!binned_cut(kr, nb, p.k, h, lane, &T, &take_eq)) radix_cut(kr, nb, p.k, h, lane, &T, &take_eq);
   }
   // ---- output pass in sweep order: chunks of 32 blocks from the start position to the
   // end of the row, then from 0. Ties are ranked by block index: the first segment starts
@@ -326,8 +428,9 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
   for (int d0 = 0; d0 < D; d0 += kScDC) {
     __syncthreads();
     // stage q rows i0.. (64 x 32) and k rows j0.. (128 x 32), transposed to [d][row]
+    // consecutive lanes take consecutive rows, so the transposed stores hit 32 banks
     for (int e = tid; e < kScI * kScDC / 4; e += 256) {
-      const int rr = e / (kScDC / 4), cc = (e % (kScDC / 4)) * 4;
+      const int rr = e % kScI, cc = (e / kScI) * 4;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (i0 + rr < nq) v = *reinterpret_cast<const float4*>(qp + (size_t)(i0 + rr) * D + d0 + cc);
       qs[cc][rr] = v.x;
@@ -336,7 +439,7 @@ __global__ void __launch_bounds__(256) score_tile_kernel(const float* __restrict
       qs[cc + 3][rr] = v.w;
     }
     for (int e = tid; e < kScJ * kScDC / 4; e += 256) {
-      const int rr = e / (kScDC / 4), cc = (e % (kScDC / 4)) * 4;
+      const int rr = e % kScJ, cc = (e / kScJ) * 4;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j0 + rr < nb) v = *reinterpret_cast<const float4*>(kp + (size_t)(j0 + rr) * D + d0 + cc);
       ks[cc][rr] = v.x;

@@ -197,6 +197,36 @@ def test_rows_are_written_in_sweep_order(spark, q_tile, mode, param):
     assert len(starts) > 8                     # the rows really are rotated
 
 
+@pytest.mark.parametrize("patterns,ratio,q_tile", [(1, 0.1, 64), (2, 0.1, 64), (5, 0.1, 64), (5, 0.5, 64),
+                                                    (40, 0.1, 64), (40, 0.5, 64), (5, 0.1, 128)])
+def test_topk_cut_inside_runs_of_equal_scores(spark, patterns, ratio, q_tile):
+    """Key blocks copied from a few patterns give rows of exactly equal scores, so the top-k
+    cut falls inside a run of equal keys: one pattern makes every score of a row equal, two
+    put more than 256 equal keys in the cut's value bin, five and forty leave a few hundred
+    or a few dozen. Every row must keep the oracle's set up to near-ties, and of each
+    pattern's blocks (equal scores, bit for bit) the lowest-index ones: the tie rule."""
+    nb, ns, d = 700, 16, 64
+    Q, K, V = make_qkv(1, 2, nb * 64, ns, d, seed=47)
+    g = torch.Generator().manual_seed(47)
+    pat = torch.randint(0, patterns, (2, nb), generator=g)
+    for h in range(2):
+        base = K[0, h, : patterns * 64].clone().view(patterns, 64, d)
+        K[0, h, : nb * 64] = base[pat[h]].reshape(nb * 64, d)
+    cfg = spark.ForwardConfig("topk", ratio, True, q_tile=q_tile)
+    plan, O, L = run_plan(spark, Q, K, V, ns, cfg)
+    assert spark.device_error() == 0
+    for h in range(2):
+        sel = gpu_rows(plan.idx[0, h].cpu().numpy(), plan.cnt[0, h].cpu().numpy())
+        ph = pat[h].numpy()
+        for i in range(plan.nt):
+            kept = np.zeros(nb, dtype=bool)
+            kept[sel[i]] = True
+            for p in range(patterns):
+                run = kept[ph == p]
+                assert np.all(run[: run.sum()]), (h, i, p)   # a prefix of the pattern's blocks
+        compare_head(plan, O, L, Q, K, V, 0, h, ns, cfg, qblocks=sample_blocks(plan.nt, 24, h))
+
+
 def test_out_of_range_index_is_skipped_and_reported(spark):
     Q, K, V = make_qkv(1, 1, 64 * 8, 8, 64, seed=3)
     Qd, Kd, Vd = Q.to(DEV), K.to(DEV), V.to(DEV)
