@@ -349,9 +349,12 @@ __global__ void __launch_bounds__(384, 1)
             // keys 16kk .. 16kk + 15: P of key half kk / 4 lives at columns 64 (kk / 4) ..
             tc::mma_ts(tbase + C::kColO, tbase + C::kColS + 128 * b + 64 * (kk >> 2) + 8 * (kk & 3),
                        tc_vdesc<D>(st, kk), idPV, (t == 0 && kk == 0) ? 0u : 1u);
+          // oready first: a softmax warp waits for it only on the tiles where it rescales O,
+          // which is sound while PV(g - 2)'s oready arrival precedes its sfree arrival (the
+          // one that lets S(g) start)
+          tc::mma_commit(oready);
           tc::mma_commit(&vempty[stage]);
           tc::mma_commit(&sfree[b]);
-          tc::mma_commit(oready);
           if (t + 1 == cur.ntiles) tc::mma_commit(odone);
         }
         ++g;
