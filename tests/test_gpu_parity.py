@@ -202,8 +202,9 @@ def test_rows_are_written_in_sweep_order(spark, q_tile, mode, param):
 def test_topk_cut_inside_runs_of_equal_scores(spark, patterns, ratio, q_tile):
     """Key blocks copied from a few patterns give rows of exactly equal scores, so the top-k
     cut falls inside a run of equal keys: one pattern makes every score of a row equal, two
-    put more than 256 equal keys in the cut's value bin, five and forty leave a few hundred
-    or a few dozen. Every row must keep the oracle's set up to near-ties, and of each
+    put about 350 equal keys (more than the 256 the cut's value bin takes) in the cut bin,
+    five and forty leave about 140 or 18. Every row must keep the oracle's set up to
+    near-ties, and of each
     pattern's blocks (equal scores, bit for bit) the lowest-index ones: the tie rule."""
     nb, ns, d = 700, 16, 64
     Q, K, V = make_qkv(1, 2, nb * 64, ns, d, seed=47)
