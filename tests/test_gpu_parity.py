@@ -204,8 +204,8 @@ def test_topk_cut_inside_runs_of_equal_scores(spark, patterns, ratio, q_tile):
     cut falls inside a run of equal keys: one pattern makes every score of a row equal, two
     put about 350 equal keys (more than the 256 the cut's value bin takes) in the cut bin,
     five and forty leave about 140 or 18. Every row must keep the oracle's set up to
-    near-ties, and of each
-    pattern's blocks (equal scores, bit for bit) the lowest-index ones: the tie rule."""
+    near-ties, and of each pattern's blocks (equal scores, bit for bit) the lowest-index
+    ones: the tie rule."""
     nb, ns, d = 700, 16, 64
     Q, K, V = make_qkv(1, 2, nb * 64, ns, d, seed=47)
     g = torch.Generator().manual_seed(47)
